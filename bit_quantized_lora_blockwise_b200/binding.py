@@ -1,0 +1,261 @@
+"""ctypes binding of libqlora.so (C ABI in include/qlora.h).
+
+Argument marshalling only: torch tensors are checked for dtype, device,
+shape and contiguity, and their raw device pointers are handed to the
+library together with the current CUDA stream. Every step of the QLoRA path
+runs in the library's CUDA kernels; there is no CPU fallback, and loading
+fails loudly when the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqlora.so")
+
+BLOCK = 64
+DQ_BLOCK = 256
+
+_lib = None
+_lock = threading.Lock()
+
+_STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_NULL", 2: "QLORA_ERR_SHAPE", 3: "QLORA_ERR_ALIGN",
+           4: "QLORA_ERR_RANGE", 5: "QLORA_ERR_CUDA", 6: "QLORA_ERR_UNSUPPORTED",
+           7: "QLORA_ERR_WORKSPACE", 8: "QLORA_ERR_TABLE"}
+
+# every symbol include/qlora.h declares
+EXPORTS = ("qlora_status_string", "qlora_abi_version", "qlora_nf4_levels", "qlora_dq_levels",
+           "qlora_workspace_bytes", "qlora_quantize_nf4", "qlora_double_quant", "qlora_dequant",
+           "qlora_linear_fwd", "qlora_linear_bwd", "qlora_device_error")
+
+
+class QLoRAError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        super().__init__(f"{call} failed: {_STATUS.get(status, status)}")
+
+
+def load(path: str | None = None):
+    """Load libqlora.so (raises OSError if it is missing: no fallback)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise OSError(f"libqlora.so not found at {p}; build it with "
+                          "`python -m bit_quantized_lora_blockwise_b200.build`")
+        lib = ctypes.CDLL(p)
+        P, I64, I32, F32, SZ = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float,
+                                ctypes.c_size_t)
+        lib.qlora_status_string.argtypes = [I32]
+        lib.qlora_status_string.restype = ctypes.c_char_p
+        lib.qlora_abi_version.restype = I32
+        lib.qlora_nf4_levels.argtypes = [P]
+        lib.qlora_dq_levels.argtypes = [P]
+        lib.qlora_workspace_bytes.argtypes = [I64, I64, I64, I32]
+        lib.qlora_workspace_bytes.restype = SZ
+        lib.qlora_quantize_nf4.argtypes = [P, I64, I64, P, P, P, P]
+        lib.qlora_double_quant.argtypes = [P, I64, P, P, P, P]
+        lib.qlora_dequant.argtypes = [P, P, P, I64, I64, P, P, P, P]
+        lib.qlora_linear_fwd.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, P, I32, F32, P, P, P, SZ, P]
+        lib.qlora_linear_bwd.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, P, P, P, I32, F32, P, P, P,
+                                         P, SZ, P]
+        lib.qlora_device_error.argtypes = [I32]
+        lib.qlora_device_error.restype = ctypes.c_uint32
+        for fn in ("qlora_quantize_nf4", "qlora_double_quant", "qlora_dequant", "qlora_linear_fwd",
+                   "qlora_linear_bwd"):
+            getattr(lib, fn).restype = I32
+        _lib = lib
+        return lib
+
+
+def _check(status: int, call: str):
+    if status != 0:
+        raise QLoRAError(status, call)
+
+
+def _ptr(t) -> ctypes.c_void_p | None:
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _req(t, name, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+class _HostTables:
+    """Host float arrays for the code tables, kept alive across calls."""
+
+    def __init__(self, nf4=None, t8=None):
+        lib = load()
+        if nf4 is None:
+            self.nf4 = (ctypes.c_float * 16)()
+            lib.qlora_nf4_levels(self.nf4)
+        else:
+            self.nf4 = (ctypes.c_float * 16)(*np.asarray(nf4, np.float32).tolist())
+        if t8 is None:
+            self.t8 = (ctypes.c_float * 256)()
+            lib.qlora_dq_levels(self.t8)
+        else:
+            self.t8 = (ctypes.c_float * 256)(*np.asarray(t8, np.float32).tolist())
+
+
+_default_tables = None
+
+
+def _tables(nf4, t8) -> _HostTables:
+    global _default_tables
+    if nf4 is None and t8 is None:
+        if _default_tables is None:
+            _default_tables = _HostTables()
+        return _default_tables
+    return _HostTables(nf4, t8)
+
+
+def nf4_levels() -> np.ndarray:
+    """The library's default 16 NF4 levels (host computation)."""
+    out = (ctypes.c_float * 16)()
+    load().qlora_nf4_levels(out)
+    return np.frombuffer(out, dtype=np.float32).copy()
+
+
+def dq_levels() -> np.ndarray:
+    out = (ctypes.c_float * 256)()
+    load().qlora_dq_levels(out)
+    return np.frombuffer(out, dtype=np.float32).copy()
+
+
+def abi_version() -> int:
+    return int(load().qlora_abi_version())
+
+
+def workspace_bytes(M: int, N: int, K: int, r: int) -> int:
+    return int(load().qlora_workspace_bytes(M, N, K, r))
+
+
+def device_error(clear: bool = False) -> int:
+    return int(load().qlora_device_error(1 if clear else 0))
+
+
+def quantize_nf4(W: torch.Tensor, nf4=None, packed=None, absmax=None):
+    """W bf16 [N, K] -> (packed uint8 [N*K/2], absmax fp32 [N*K/64])."""
+    N, K = W.shape
+    _req(W, "W", torch.bfloat16)
+    if packed is None:
+        packed = torch.empty(N * K // 2, dtype=torch.uint8, device=W.device)
+    if absmax is None:
+        absmax = torch.empty(N * K // BLOCK, dtype=torch.float32, device=W.device)
+    _req(packed, "packed", torch.uint8, (N * K // 2,))
+    _req(absmax, "absmax", torch.float32, (N * K // BLOCK,))
+    tb = _tables(nf4, None)
+    _check(load().qlora_quantize_nf4(_ptr(W), N, K, tb.nf4, _ptr(packed), _ptr(absmax), _stream()),
+           "qlora_quantize_nf4")
+    return packed, absmax
+
+
+def double_quant(absmax: torch.Tensor, t8=None, q=None, scale2=None):
+    """absmax fp32 [nb] -> (q uint8 [nb], scale2 fp32 [ceil(nb/256)])."""
+    _req(absmax, "absmax", torch.float32)
+    nb = absmax.numel()
+    ng = (nb + DQ_BLOCK - 1) // DQ_BLOCK
+    if q is None:
+        q = torch.empty(nb, dtype=torch.uint8, device=absmax.device)
+    if scale2 is None:
+        scale2 = torch.empty(ng, dtype=torch.float32, device=absmax.device)
+    _req(q, "q", torch.uint8, (nb,))
+    _req(scale2, "scale2", torch.float32, (ng,))
+    tb = _tables(None, t8)
+    _check(load().qlora_double_quant(_ptr(absmax), nb, tb.t8, _ptr(q), _ptr(scale2), _stream()),
+           "qlora_double_quant")
+    return q, scale2
+
+
+def dequant(packed, q, scale2, N: int, K: int, nf4=None, t8=None, out=None) -> torch.Tensor:
+    """-> W' bf16 [N, K]."""
+    _req(packed, "packed", torch.uint8, (N * K // 2,))
+    _req(q, "q", torch.uint8, (N * K // BLOCK,))
+    _req(scale2, "scale2", torch.float32)
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.bfloat16, device=packed.device)
+    _req(out, "out", torch.bfloat16, (N, K))
+    tb = _tables(nf4, t8)
+    _check(load().qlora_dequant(_ptr(packed), _ptr(q), _ptr(scale2), N, K, tb.nf4, tb.t8, _ptr(out),
+                                _stream()), "qlora_dequant")
+    return out
+
+
+def _workspace(workspace, M, N, K, r, device):
+    need = workspace_bytes(M, N, K, r)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+    _req(workspace, "workspace", torch.uint8)
+    return workspace
+
+
+def linear_fwd(packed, q, scale2, X, A, B, alpha: float, N: int, K: int, nf4=None, t8=None,
+               Y=None, XA_out=None, workspace=None):
+    """Y = X W'^T + (alpha/r) (X A) B  -> Y bf16 [M, N] (and XA_out if given)."""
+    M = X.shape[0]
+    r = A.shape[1]
+    _req(X, "X", torch.bfloat16, (M, K))
+    _req(A, "A", torch.bfloat16, (K, r))
+    _req(B, "B", torch.bfloat16, (r, N))
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _req(Y, "Y", torch.bfloat16, (M, N))
+    if XA_out is not None:
+        _req(XA_out, "XA_out", torch.bfloat16, (M, r))
+    workspace = _workspace(workspace, M, N, K, r, X.device)
+    tb = _tables(nf4, t8)
+    _check(load().qlora_linear_fwd(_ptr(packed), _ptr(q), _ptr(scale2), tb.nf4, tb.t8, M, N, K, _ptr(X),
+                                   _ptr(A), _ptr(B), r, float(alpha), _ptr(Y), _ptr(XA_out),
+                                   _ptr(workspace), workspace.numel(), _stream()), "qlora_linear_fwd")
+    return Y
+
+
+def linear_bwd(packed, q, scale2, X, dY, A, B, alpha: float, N: int, K: int, XA=None, nf4=None, t8=None,
+               dX=None, dA=None, dB=None, workspace=None):
+    """-> (dX bf16 [M, K], dA bf16 [K, r], dB bf16 [r, N]); no dW (W is frozen)."""
+    M = X.shape[0]
+    r = A.shape[1]
+    _req(X, "X", torch.bfloat16, (M, K))
+    _req(dY, "dY", torch.bfloat16, (M, N))
+    _req(A, "A", torch.bfloat16, (K, r))
+    _req(B, "B", torch.bfloat16, (r, N))
+    if XA is not None:
+        _req(XA, "XA", torch.bfloat16, (M, r))
+    dev = X.device
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev) if dX is None else dX
+    dA = torch.empty((K, r), dtype=torch.bfloat16, device=dev) if dA is None else dA
+    dB = torch.empty((r, N), dtype=torch.bfloat16, device=dev) if dB is None else dB
+    _req(dX, "dX", torch.bfloat16, (M, K))
+    _req(dA, "dA", torch.bfloat16, (K, r))
+    _req(dB, "dB", torch.bfloat16, (r, N))
+    workspace = _workspace(workspace, M, N, K, r, dev)
+    tb = _tables(nf4, t8)
+    _check(load().qlora_linear_bwd(_ptr(packed), _ptr(q), _ptr(scale2), tb.nf4, tb.t8, M, N, K, _ptr(X),
+                                   _ptr(dY), _ptr(A), _ptr(B), _ptr(XA), r, float(alpha), _ptr(dX), _ptr(dA),
+                                   _ptr(dB), _ptr(workspace), workspace.numel(), _stream()),
+           "qlora_linear_bwd")
+    return dX, dA, dB

@@ -1,0 +1,238 @@
+// NF4 codec kernels: blockwise absmax + nearest-level encode + nibble pack,
+// double quantization of the absmax constants, and dequantization to bf16.
+//
+// Method (QLoRA pages): intvml.com "DL0087 QLoRA: 4-bit Quantized LoRA",
+// components (1)-(3) and the formulation's symbol list; promptingindex.com
+// "QLoRA: Finetuning 65B Models on a Single GPU", sections "4-bit
+// NormalFloat" and "Double Quantization and Paged Optimizers".
+//
+// All three kernels are HBM-bound streaming kernels: 128-bit loads, one warp
+// lane per 8 (quantize) or 16 (dequant) consecutive weights, warp shuffles
+// for the per-block reduction, grid-stride loops over a grid sized to the
+// SM count.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace qlora {
+
+struct CodecTables {
+  float nf4[16];
+  float t8[256];
+};
+
+// ------------------------------------------------------------------------
+// NF4 code of x: the number of fp32 midpoints m_i = (L_i + L_{i+1}) * 0.5
+// strictly below x, by a 4-step binary search over the 15 sorted midpoints
+// (mid[] in shared memory, mid7 in a register).
+__device__ __forceinline__ uint32_t nf4_code(float x, const float *mid, float mid7) {
+  uint32_t c = (x > mid7) ? 8u : 0u;
+  c += (x > mid[c + 3]) ? 4u : 0u;
+  c += (x > mid[c + 1]) ? 2u : 0u;
+  c += (x > mid[c]) ? 1u : 0u;
+  return c;
+}
+
+// Correctly rounded x = w / c from the correctly rounded reciprocal
+// r = RN(1/c): q0 = RN(w r), residual e = w - q0 c (exact with one FMA),
+// x = RN(q0 + e r). Markstein's theorem (P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990) gives x = RN(w / c) when r is within half an ulp of 1/c
+// and q0 within one ulp of w / c, barring underflow. The caller routes
+// blocks whose c lies outside [2^-125, 2^125] (1/c near overflow or
+// subnormal) through the IEEE divide; a quotient that underflows is far
+// below every NF4 midpoint, so its rounding cannot change the code.
+__device__ __forceinline__ float div_by_recip(float w, float c, float r) {
+  const float q0 = __fmul_rn(w, r);
+  const float e = __fmaf_rn(-q0, c, w);
+  return __fmaf_rn(e, r, q0);
+}
+
+// One 64-weight block per 8 lanes; each lane encodes 8 consecutive weights
+// (one 16-byte load) into one 32-bit word of 8 nibbles.
+__global__ void __launch_bounds__(256) quantize_nf4_kernel(const uint4 *__restrict__ W,
+                                                           int64_t nblocks,
+                                                           uint32_t *__restrict__ packed,
+                                                           float *__restrict__ absmax,
+                                                           const CodecTables tabs) {
+  __shared__ float s_mid[16];
+  if (threadIdx.x < 15)
+    s_mid[threadIdx.x] = __fmul_rn(__fadd_rn(tabs.nf4[threadIdx.x], tabs.nf4[threadIdx.x + 1]), 0.5f);
+  __syncthreads();
+  const float mid7 = s_mid[7];
+  const uint32_t sub = threadIdx.x & 7u;
+  const uint32_t lane = threadIdx.x & 31u;
+  const int64_t nwords = nblocks * 8;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  // The loop runs per warp (base is warp-uniform) so the shuffles below
+  // always see all 32 lanes; lanes past the end compute on zeros.
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31u);
+       base < nwords; base += stride) {
+    const int64_t t = base + lane;
+    const bool valid = t < nwords;
+    const int64_t b = t >> 3;
+    const uint4 v = valid ? __ldg(&W[t]) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(wd[i] << 16);
+      f[2 * i + 1] = __uint_as_float(wd[i] & 0xFFFF0000u);
+    }
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+    // each 8-lane group (one 64-block) reduces independently
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+    const float c = m;
+    uint32_t word = 0;
+    if (c == 0.0f) {
+      const uint32_t z = nf4_code(0.0f, s_mid, mid7);
+      word = z * 0x11111111u;
+    } else if (c >= 0x1p-125f && c <= 0x1p125f) {
+      const float r = __frcp_rn(c);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) word |= nf4_code(div_by_recip(f[i], c, r), s_mid, mid7) << (4 * i);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) word |= nf4_code(__fdiv_rn(f[i], c), s_mid, mid7) << (4 * i);
+    }
+    if (!valid) continue;
+    packed[t] = word;
+    if (sub == 0) absmax[b] = c;
+  }
+}
+
+// ------------------------------------------------------------------------
+// Double quantization: one warp per group of 256 constants, 8 per lane.
+// S = group max; q = number of fp32 midpoints of t8 strictly below c / S
+// (8-step binary search over the 255 midpoints); a group of zeros -> x = 0.
+__global__ void __launch_bounds__(256) double_quant_kernel(const float *__restrict__ absmax,
+                                                           int64_t nb, uint8_t *__restrict__ q,
+                                                           float *__restrict__ scale2,
+                                                           const CodecTables tabs) {
+  __shared__ float s_mid[256];
+  if (threadIdx.x < 255)
+    s_mid[threadIdx.x] = __fmul_rn(__fadd_rn(tabs.t8[threadIdx.x], tabs.t8[threadIdx.x + 1]), 0.5f);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t ng = (nb + 255) / 256;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       g < ng; g += warps) {
+    const int64_t base = g * 256 + lane * 8;
+    float c[8];
+    if (base + 8 <= nb) {
+      const float4 a = __ldg(reinterpret_cast<const float4 *>(absmax + base));
+      const float4 b = __ldg(reinterpret_cast<const float4 *>(absmax + base + 4));
+      c[0] = a.x; c[1] = a.y; c[2] = a.z; c[3] = a.w;
+      c[4] = b.x; c[5] = b.y; c[6] = b.z; c[7] = b.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c[i] = (base + i < nb) ? absmax[base + i] : 0.0f;
+    }
+    float s = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s = fmaxf(s, c[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s = fmaxf(s, __shfl_xor_sync(0xFFFFFFFFu, s, o));
+    uint32_t codes[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float x = (s == 0.0f) ? 0.0f : __fdiv_rn(c[i], s);
+      uint32_t k = 0;
+#pragma unroll
+      for (uint32_t step = 128; step > 0; step >>= 1)
+        if (x > s_mid[k + step - 1]) k += step;
+      codes[i] = k;
+    }
+    if (base + 8 <= nb) {
+      uint2 packed8;
+      packed8.x = codes[0] | (codes[1] << 8) | (codes[2] << 16) | (codes[3] << 24);
+      packed8.y = codes[4] | (codes[5] << 8) | (codes[6] << 16) | (codes[7] << 24);
+      *reinterpret_cast<uint2 *>(q + base) = packed8;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (base + i < nb) q[base + i] = static_cast<uint8_t>(codes[i]);
+    }
+    if (lane == 0) scale2[g] = s;
+  }
+}
+
+// ------------------------------------------------------------------------
+// NF4 decode of one block: the 16 products bf16(L_i * c') are formed once
+// (fp32 multiply, RNE to bf16) and split into four 8-byte planes (low and
+// high bytes of entries 0-7 and 8-15); each 4-bit code then picks its two
+// bytes with byte permutes, with no memory lookups.
+struct Nf4Planes {
+  uint32_t alo0, alo1, ahi0, ahi1, blo0, blo1, bhi0, bhi1;
+};
+
+__device__ __forceinline__ Nf4Planes make_planes(const float (&L)[16], float cp) {
+  uint32_t t[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) t[j] = pack_bf16x2(__fmul_rn(L[2 * j], cp), __fmul_rn(L[2 * j + 1], cp));
+  Nf4Planes p;
+  p.alo0 = prmt(t[0], t[1], 0x6420u);
+  p.alo1 = prmt(t[2], t[3], 0x6420u);
+  p.ahi0 = prmt(t[0], t[1], 0x7531u);
+  p.ahi1 = prmt(t[2], t[3], 0x7531u);
+  p.blo0 = prmt(t[4], t[5], 0x6420u);
+  p.blo1 = prmt(t[6], t[7], 0x6420u);
+  p.bhi0 = prmt(t[4], t[5], 0x7531u);
+  p.bhi1 = prmt(t[6], t[7], 0x7531u);
+  return p;
+}
+
+// 8 codes (nibble i of w = element i) -> 8 bf16 in out[0..3]
+// (out[k] = element 2k in the low half, 2k+1 in the high half).
+__device__ __forceinline__ void nf4_lookup8(const Nf4Planes &P, uint32_t w, uint32_t (&out)[4]) {
+  const uint32_t m = w & 0x77777777u;                       // code & 7 of every nibble
+  const uint32_t s = ((w >> 1) & 0x44444444u) | 0x32103210u;  // byte k or k+4 by code bit 3
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t mh = h ? (m >> 16) : m;
+    const uint32_t sh = h ? (s >> 16) : s;
+    const uint32_t la = prmt(P.alo0, P.alo1, mh);
+    const uint32_t lb = prmt(P.blo0, P.blo1, mh);
+    const uint32_t ha = prmt(P.ahi0, P.ahi1, mh);
+    const uint32_t hb = prmt(P.bhi0, P.bhi1, mh);
+    const uint32_t lo = prmt(la, lb, sh);
+    const uint32_t hi = prmt(ha, hb, sh);
+    out[2 * h] = prmt(lo, hi, 0x5140u);
+    out[2 * h + 1] = prmt(lo, hi, 0x7362u);
+  }
+}
+
+// Standalone dequantization: one lane per 16 consecutive weights
+// (a quarter of a 64-block): 8 packed bytes in, 32 bytes of bf16 out.
+__global__ void __launch_bounds__(256) dequant_kernel(const uint2 *__restrict__ packed,
+                                                      const uint8_t *__restrict__ q,
+                                                      const float *__restrict__ scale2,
+                                                      int64_t nquarters, uint4 *__restrict__ out,
+                                                      const CodecTables tabs) {
+  __shared__ float s_t8[256];
+  s_t8[threadIdx.x] = tabs.t8[threadIdx.x];
+  __syncthreads();
+  float L[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) L[i] = tabs.nf4[i];
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < nquarters;
+       t += nthreads) {
+    const int64_t b = t >> 2;
+    const uint2 pk = __ldg(&packed[t]);
+    const float cp = __fmul_rn(s_t8[__ldg(&q[b])], __ldg(&scale2[b >> 8]));
+    const Nf4Planes P = make_planes(L, cp);
+    uint32_t o0[4], o1[4];
+    nf4_lookup8(P, pk.x, o0);
+    nf4_lookup8(P, pk.y, o1);
+    out[2 * t] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+    out[2 * t + 1] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+  }
+}
+
+}  // namespace qlora

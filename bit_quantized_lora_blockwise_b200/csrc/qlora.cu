@@ -1,0 +1,576 @@
+// libqlora.so — C ABI (include/qlora.h) over the sm_100a kernels in
+// codec.cuh and gemm.cuh. Host side: argument checks, the default code
+// tables, TMA tensor-map encoding, workspace carving and the launch order of
+// the forward and backward passes. Single translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "qlora.h"
+#include "codec.cuh"
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+using namespace qlora;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// ------------------------------------------------------------ utilities --
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct DeviceInfo {
+  bool init = false;
+  bool sm100 = false;
+  int sms = 0;
+};
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+qlora_status device_info(DeviceInfo *out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo &d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    d.sm100 = (major == 10 && minor == 0);
+    d.sms = sms;
+    d.init = true;
+  }
+  *out = d;
+  return d.sm100 ? QLORA_OK : QLORA_ERR_UNSUPPORTED;
+}
+
+// Code tables: finite and strictly ascending; the NF4 table holds 0.0f.
+qlora_status check_tables(const float *nf4, const float *t8) {
+  if (nf4 != nullptr) {
+    bool zero = false;
+    for (int i = 0; i < 16; ++i) {
+      if (!std::isfinite(nf4[i])) return QLORA_ERR_TABLE;
+      if (i > 0 && !(nf4[i] > nf4[i - 1])) return QLORA_ERR_TABLE;
+      if (nf4[i] == 0.0f) zero = true;
+    }
+    if (!zero) return QLORA_ERR_TABLE;
+  }
+  if (t8 != nullptr) {
+    for (int i = 0; i < 256; ++i) {
+      if (!std::isfinite(t8[i])) return QLORA_ERR_TABLE;
+      if (i > 0 && !(t8[i] > t8[i - 1])) return QLORA_ERR_TABLE;
+    }
+  }
+  return QLORA_OK;
+}
+
+CodecTables make_tables(const float *nf4, const float *t8) {
+  CodecTables t;
+  std::memset(&t, 0, sizeof t);
+  if (nf4) std::memcpy(t.nf4, nf4, sizeof t.nf4);
+  if (t8) std::memcpy(t.t8, t8, sizeof t.t8);
+  return t;
+}
+
+int grid_for(int64_t work_items, int per_cta, int sms, int waves) {
+  const int64_t want = cdiv(work_items, per_cta);
+  const int64_t cap = static_cast<int64_t>(sms) * waves;
+  return static_cast<int>(want < 1 ? 1 : (want < cap ? want : cap));
+}
+
+// ------------------------------------------------------------ TMA maps --
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [outer, inner] with row pitch `row_bytes`; box
+// {box_inner, box_outer}; out-of-range elements read as zero.
+bool make_map(CUtensorMap *map, const void *base, bool bf16, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                        const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// bf16 operand [outer rows, inner] read as K-major tiles (box {64, box_rows})
+bool map_kmajor(CUtensorMap *m, const void *p, int64_t inner, int64_t outer, uint32_t box_rows) {
+  return make_map(m, p, true, inner, outer, inner * 2, 64, box_rows, true);
+}
+// bf16 operand [outer rows, inner] read as MN-major 64x64 chunks
+bool map_mnmajor(CUtensorMap *m, const void *p, int64_t inner, int64_t outer) {
+  return make_map(m, p, true, inner, outer, inner * 2, 64, 64, true);
+}
+
+// ------------------------------------------------------- GEMM launcher --
+template <class C>
+qlora_status launch_gemm(const GemmArgs &args, int sms, cudaStream_t stream) {
+  static std::once_flag once[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(once[dev], [&] {
+    attr_err = cudaFuncSetAttribute(qgemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return QLORA_ERR_CUDA;
+  const int row_tiles = (args.rows + 127) / 128;
+  const int col_tiles = (args.cols + C::BN - 1) / C::BN;
+  const int tiles = row_tiles * col_tiles * args.splits;
+  const int grid = tiles < sms ? tiles : sms;
+  qgemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(args);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status launch_reduce(const float *part, int splits, int rows, int cols, int64_t rows_pad,
+                           int64_t cols_pad, float scale, void *out, int64_t ld, float scale2, void *out2,
+                           int64_t ld2, bool transpose, int sms, cudaStream_t stream) {
+  const int64_t total = static_cast<int64_t>(rows) * cols;
+  const int grid = grid_for(total, 256, sms, 8);
+  splitk_reduce_kernel<<<grid, 256, 0, stream>>>(part, splits, rows, cols, rows_pad, cols_pad, scale,
+                                                 reinterpret_cast<__nv_bfloat16 *>(out), ld, scale2,
+                                                 reinterpret_cast<__nv_bfloat16 *>(out2), ld2,
+                                                 transpose ? 1 : 0);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// ------------------------------------------------------- skinny GEMMs --
+// out[rows, r] (or its transpose) = scale * sum_k Aop[row, k] Bop[j, k],
+// with the K range split across CTAs into fp32 partials, then reduced.
+enum SkinnyKind { SK_XA, SK_G, SK_DA, SK_DB };
+
+int rank_tile(int r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
+
+struct SkinnyPlan {
+  int rows, kblocks, splits, bn;
+  size_t part_bytes;
+};
+
+SkinnyPlan plan_skinny(int64_t rows, int64_t kdim, int r, int sms) {
+  SkinnyPlan p;
+  p.rows = static_cast<int>(rows);
+  p.kblocks = static_cast<int>(cdiv(kdim, 64));
+  p.bn = rank_tile(r);
+  const int row_tiles = static_cast<int>(cdiv(rows, 128));
+  int splits = static_cast<int>(cdiv(sms, row_tiles));
+  if (splits > p.kblocks) splits = p.kblocks;
+  if (splits < 1) splits = 1;
+  p.splits = splits;
+  p.part_bytes = align256(static_cast<size_t>(splits) * row_tiles * 128 * p.bn * 4);
+  return p;
+}
+
+template <int BN, int AS, int BS>
+qlora_status run_skinny_bn(const GemmArgs &a, int sms, cudaStream_t st) {
+  using C = GemmCfg<BN, AS, BS, L2_NONE, EPI_F32, (BN == 256 ? 4 : 6), 0>;
+  return launch_gemm<C>(a, sms, st);
+}
+
+template <int AS, int BS>
+qlora_status run_skinny(const GemmArgs &a, int bn, int sms, cudaStream_t st) {
+  if (bn == 64) return run_skinny_bn<64, AS, BS>(a, sms, st);
+  if (bn == 128) return run_skinny_bn<128, AS, BS>(a, sms, st);
+  return run_skinny_bn<256, AS, BS>(a, sms, st);
+}
+
+// kind: SK_XA   Aop = X [M,K] (K-major),   Bop = A  [K,r] (MN-major), rows = M, kdim = K
+//       SK_G    Aop = dY [M,N] (K-major),  Bop = B  [r,N] (K-major),  rows = M, kdim = N
+//       SK_DA   Aop = X^T (MN-major),      Bop = Gs [M,r] (MN-major), rows = K, kdim = M
+//       SK_DB   Aop = dY^T (MN-major),     Bop = XA [M,r] (MN-major), rows = N, kdim = M
+qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a_outer, const void *bop,
+                    int64_t b_inner, int64_t b_outer, int64_t rows, int64_t kdim, int r, float scale,
+                    void *out, int64_t ld, float scale2, void *out2, int64_t ld2, bool transpose,
+                    float *part, int sms, cudaStream_t st) {
+  const SkinnyPlan p = plan_skinny(rows, kdim, r, sms);
+  GemmArgs a;
+  std::memset(&a, 0, sizeof a);
+  bool ok = true;
+  switch (kind) {
+    case SK_XA:
+      ok = map_kmajor(&a.tm_a, aop, a_inner, a_outer, 128) && map_mnmajor(&a.tm_b, bop, b_inner, b_outer);
+      break;
+    case SK_G:
+      ok = map_kmajor(&a.tm_a, aop, a_inner, a_outer, 128) &&
+           map_kmajor(&a.tm_b, bop, b_inner, b_outer, p.bn);
+      break;
+    case SK_DA:
+    case SK_DB:
+      ok = map_mnmajor(&a.tm_a, aop, a_inner, a_outer) && map_mnmajor(&a.tm_b, bop, b_inner, b_outer);
+      break;
+  }
+  if (!ok) return QLORA_ERR_CUDA;
+  a.out = part;
+  a.rows = p.rows;
+  a.cols = r;
+  a.kblocks = p.kblocks;
+  a.splits = p.splits;
+  a.lora_kblocks = 0;
+  a.out_scale = 1.0f;
+  qlora_status s;
+  switch (kind) {
+    case SK_XA: s = run_skinny<A_TMA_K, B_TMA_MN>(a, p.bn, sms, st); break;
+    case SK_G: s = run_skinny<A_TMA_K, B_TMA_K>(a, p.bn, sms, st); break;
+    default: s = run_skinny<A_TMA_MN, B_TMA_MN>(a, p.bn, sms, st); break;
+  }
+  if (s != QLORA_OK) return s;
+  const int64_t rows_pad = cdiv(rows, 128) * 128;
+  return launch_reduce(part, p.splits, static_cast<int>(rows), r, rows_pad, p.bn, scale, out, ld, scale2,
+                       out2, ld2, transpose, sms, st);
+}
+
+// -------------------------------------------------------- fused GEMMs --
+struct FusedPlan {
+  int bn, splits;
+  size_t part_bytes;
+};
+
+FusedPlan plan_fused(int64_t M, int64_t rows, int64_t kblocks, int sms) {
+  FusedPlan p;
+  p.bn = M <= 32 ? 32 : 256;
+  const int64_t tiles = cdiv(rows, 128) * cdiv(M, p.bn);
+  int64_t splits = 1;
+  if (tiles < sms) {
+    splits = sms / tiles;
+    if (splits > kblocks) splits = kblocks;
+    if (splits < 1) splits = 1;
+  }
+  p.splits = static_cast<int>(splits);
+  p.part_bytes = p.splits > 1 ? align256(static_cast<size_t>(p.splits) * cdiv(rows, 128) * 128 *
+                                         cdiv(M, p.bn) * p.bn * 4)
+                              : 0;
+  return p;
+}
+
+template <int BN, int AS, int L2>
+qlora_status run_fused_bn(const GemmArgs &a, int sms, cudaStream_t st) {
+  if (a.splits > 1) return launch_gemm<GemmCfg<BN, AS, B_TMA_K, L2, EPI_F32, (BN > 64 ? 4 : 8), 8>>(a, sms, st);
+  return launch_gemm<GemmCfg<BN, AS, B_TMA_K, L2, EPI_BF16_T, (BN > 64 ? 4 : 8), 8>>(a, sms, st);
+}
+
+// Layer sizes shared by forward and backward.
+struct Shape {
+  int64_t M, N, K;
+  int r;
+};
+
+size_t fwd_ws_bytes(const Shape &s, int sms) {
+  const size_t xas = align256(static_cast<size_t>(s.M) * s.r * 2);
+  const SkinnyPlan xa = plan_skinny(s.M, s.K, s.r, sms);
+  const FusedPlan fp = plan_fused(s.M, s.N, s.K / 64, sms);
+  return xas + (xa.part_bytes > fp.part_bytes ? xa.part_bytes : fp.part_bytes);
+}
+
+size_t bwd_ws_bytes(const Shape &s, int sms) {
+  const size_t mr = align256(static_cast<size_t>(s.M) * s.r * 2);
+  size_t part = plan_skinny(s.M, s.N, s.r, sms).part_bytes;                 // G
+  part = std::max(part, plan_skinny(s.K, s.M, s.r, sms).part_bytes);         // dA
+  part = std::max(part, plan_skinny(s.N, s.M, s.r, sms).part_bytes);         // dB
+  part = std::max(part, plan_skinny(s.M, s.K, s.r, sms).part_bytes);         // XA recompute
+  part = std::max(part, plan_fused(s.M, s.K, s.N / 64, sms).part_bytes);     // dX split-K
+  return 2 * mr + part;
+}
+
+qlora_status check_linear(const uint8_t *packed, const uint8_t *q, const float *scale2, const float *nf4,
+                          const float *t8, const Shape &s, float alpha) {
+  if (!packed || !q || !scale2 || !nf4 || !t8) return QLORA_ERR_NULL;
+  if (s.M < 1 || s.N < 64 || s.K < 64 || s.N % 64 || s.K % 64) return QLORA_ERR_SHAPE;
+  if (s.M > (int64_t(1) << 30) || s.N > (int64_t(1) << 30) || s.K > (int64_t(1) << 30))
+    return QLORA_ERR_SHAPE;
+  if (s.r < 1 || s.r > QLORA_MAX_RANK || s.r % 8) return QLORA_ERR_RANGE;
+  if (!std::isfinite(alpha)) return QLORA_ERR_RANGE;
+  if (!aligned16(packed) || !aligned16(q) || !aligned16(scale2)) return QLORA_ERR_ALIGN;
+  return check_tables(nf4, t8);
+}
+
+}  // namespace
+
+// ====================================================================== ABI
+extern "C" {
+
+const char *qlora_status_string(qlora_status s) {
+  switch (s) {
+    case QLORA_OK: return "QLORA_OK";
+    case QLORA_ERR_NULL: return "QLORA_ERR_NULL";
+    case QLORA_ERR_SHAPE: return "QLORA_ERR_SHAPE";
+    case QLORA_ERR_ALIGN: return "QLORA_ERR_ALIGN";
+    case QLORA_ERR_RANGE: return "QLORA_ERR_RANGE";
+    case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA";
+    case QLORA_ERR_UNSUPPORTED: return "QLORA_ERR_UNSUPPORTED";
+    case QLORA_ERR_WORKSPACE: return "QLORA_ERR_WORKSPACE";
+    case QLORA_ERR_TABLE: return "QLORA_ERR_TABLE";
+  }
+  return "QLORA_ERR_UNKNOWN";
+}
+
+int qlora_abi_version(void) { return QLORA_ABI_VERSION; }
+
+// Standard-normal quantile by Newton's method on the CDF written with erfc
+// (double precision), from z = 0: z <- z - (Phi(z) - p) / phi(z).
+static double normal_quantile(double p) {
+  double z = 0.0;
+  for (int it = 0; it < 100; ++it) {
+    const double cdf = 0.5 * std::erfc(-z / std::sqrt(2.0));
+    const double pdf = std::exp(-0.5 * z * z) / std::sqrt(2.0 * M_PI);
+    const double step = (cdf - p) / pdf;
+    z -= step;
+    if (std::fabs(step) < 1e-17 * (1.0 + std::fabs(z))) break;
+  }
+  return z;
+}
+
+void qlora_nf4_levels(float out[16]) {
+  if (out == nullptr) return;
+  const double delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0));
+  const double zmax = normal_quantile(delta);
+  for (int i = 0; i < 7; ++i) out[i] = static_cast<float>(-normal_quantile(delta + i * (0.5 - delta) / 7.0) / zmax);
+  out[7] = 0.0f;
+  for (int j = 0; j < 8; ++j) out[15 - j] = static_cast<float>(normal_quantile(delta + j * (0.5 - delta) / 8.0) / zmax);
+}
+
+void qlora_dq_levels(float out[256]) {
+  if (out == nullptr) return;
+  for (int k = 0; k < 256; ++k) out[k] = static_cast<float>(k) / 255.0f;
+}
+
+size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
+  if (M < 1 || N < 64 || K < 64 || N % 64 || K % 64 || r < 1 || r > QLORA_MAX_RANK || r % 8) return 0;
+  DeviceInfo d;
+  int sms = 148;
+  if (device_info(&d) == QLORA_OK) sms = d.sms;
+  const Shape s{M, N, K, r};
+  const size_t f = fwd_ws_bytes(s, sms), b = bwd_ws_bytes(s, sms);
+  return f > b ? f : b;
+}
+
+qlora_status qlora_quantize_nf4(const qlora_bf16 *W, int64_t N, int64_t K, const float nf4[16], uint8_t *packed,
+                                float *absmax, qlora_stream_t stream) {
+  if (!W || !nf4 || !packed || !absmax) return QLORA_ERR_NULL;
+  if (N < 1 || K < 64 || K % 64) return QLORA_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(absmax)) return QLORA_ERR_ALIGN;
+  qlora_status st = check_tables(nf4, nullptr);
+  if (st != QLORA_OK) return st;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != QLORA_OK) return st;
+  const int64_t nblocks = N * (K / 64);
+  const int grid = grid_for(nblocks * 8, 256, d.sms, 16);
+  quantize_nf4_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint4 *>(W), nblocks, reinterpret_cast<uint32_t *>(packed), absmax,
+      make_tables(nf4, nullptr));
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_double_quant(const float *absmax, int64_t nb, const float t8[256], uint8_t *q, float *scale2,
+                                qlora_stream_t stream) {
+  if (!absmax || !t8 || !q || !scale2) return QLORA_ERR_NULL;
+  if (nb < 1) return QLORA_ERR_SHAPE;
+  if (!aligned16(absmax) || !aligned16(q) || !aligned16(scale2)) return QLORA_ERR_ALIGN;
+  qlora_status st = check_tables(nullptr, t8);
+  if (st != QLORA_OK) return st;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != QLORA_OK) return st;
+  const int64_t ng = cdiv(nb, 256);
+  const int grid = grid_for(ng, 8, d.sms, 16);
+  double_quant_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(absmax, nb, q, scale2,
+                                                                            make_tables(nullptr, t8));
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_dequant(const uint8_t *packed, const uint8_t *q, const float *scale2, int64_t N, int64_t K,
+                           const float nf4[16], const float t8[256], qlora_bf16 *W_out, qlora_stream_t stream) {
+  if (!packed || !q || !scale2 || !nf4 || !t8 || !W_out) return QLORA_ERR_NULL;
+  if (N < 1 || K < 64 || K % 64) return QLORA_ERR_SHAPE;
+  if (!aligned16(packed) || !aligned16(q) || !aligned16(scale2) || !aligned16(W_out)) return QLORA_ERR_ALIGN;
+  qlora_status st = check_tables(nf4, t8);
+  if (st != QLORA_OK) return st;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != QLORA_OK) return st;
+  const int64_t quarters = N * K / 16;
+  const int grid = grid_for(quarters, 256, d.sms, 16);
+  dequant_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint2 *>(packed), q, scale2, quarters, reinterpret_cast<uint4 *>(W_out),
+      make_tables(nf4, t8));
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const float *scale2, const float nf4[16],
+                              const float t8[256], int64_t M, int64_t N, int64_t K, const qlora_bf16 *X,
+                              const qlora_bf16 *A, const qlora_bf16 *B, int r, float alpha, qlora_bf16 *Y,
+                              qlora_bf16 *XA_out, void *workspace, size_t workspace_bytes,
+                              qlora_stream_t stream) {
+  const Shape s{M, N, K, r};
+  qlora_status st = check_linear(packed, q, scale2, nf4, t8, s, alpha);
+  if (st != QLORA_OK) return st;
+  if (!X || !A || !B || !Y) return QLORA_ERR_NULL;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || (XA_out && !aligned16(XA_out)) ||
+      !aligned16(workspace))
+    return QLORA_ERR_ALIGN;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != QLORA_OK) return st;
+  if (!workspace || workspace_bytes < fwd_ws_bytes(s, d.sms)) return QLORA_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const float scl = alpha / static_cast<float>(r);
+
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  qlora_bf16 *xas = reinterpret_cast<qlora_bf16 *>(ws);
+  float *part = reinterpret_cast<float *>(ws + align256(static_cast<size_t>(M) * r * 2));
+
+  // 1) XA = X A (split-K partials) -> XA_out = bf16(XA), xas = bf16(s XA)
+  if (XA_out != nullptr)
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, 1.0f, XA_out, r, scl, xas, r, false, part, d.sms, cs);
+  else
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, scl, xas, r, 0.0f, nullptr, 0, false, part, d.sms, cs);
+  if (st != QLORA_OK) return st;
+
+  // 2) Y^T[n, m] = W'[n, :] . X[m, :] + B^T[n, :] . xas[m, :]
+  const FusedPlan fp = plan_fused(M, N, K / 64, d.sms);
+  GemmArgs a;
+  std::memset(&a, 0, sizeof a);
+  if (!map_kmajor(&a.tm_b, X, K, M, fp.bn) ||
+      !make_map(&a.tm_pk, packed, false, K / 2, N, K / 2, 32, 128, false) ||
+      !map_mnmajor(&a.tm_a2, B, N, r) || !map_kmajor(&a.tm_b2, xas, r, M, fp.bn))
+    return QLORA_ERR_CUDA;
+  a.q = q;
+  a.scale2 = scale2;
+  a.w_kblocks = K / 64;
+  a.w_rows = static_cast<int>(N);
+  a.rows = static_cast<int>(N);
+  a.cols = static_cast<int>(M);
+  a.kblocks = static_cast<int>(K / 64);
+  a.splits = fp.splits;
+  a.lora_kblocks = static_cast<int>(cdiv(r, 64));
+  a.out_scale = 1.0f;
+  std::memcpy(a.nf4, nf4, sizeof a.nf4);
+  std::memcpy(a.t8, t8, sizeof a.t8);
+  if (fp.splits == 1) {
+    a.out = Y;
+    a.out_ld = N;
+  } else {
+    a.out = part;
+  }
+  st = fp.bn == 32 ? run_fused_bn<32, A_DEQ_K, L2_A_MN>(a, d.sms, cs)
+                   : run_fused_bn<256, A_DEQ_K, L2_A_MN>(a, d.sms, cs);
+  if (st != QLORA_OK || fp.splits == 1) return st;
+  return launch_reduce(part, fp.splits, static_cast<int>(N), static_cast<int>(M), cdiv(N, 128) * 128,
+                       cdiv(M, fp.bn) * fp.bn, 1.0f, Y, N, 0.0f, nullptr, 0, true, d.sms, cs);
+}
+
+qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const float *scale2, const float nf4[16],
+                              const float t8[256], int64_t M, int64_t N, int64_t K, const qlora_bf16 *X,
+                              const qlora_bf16 *dY, const qlora_bf16 *A, const qlora_bf16 *B, const qlora_bf16 *XA,
+                              int r, float alpha, qlora_bf16 *dX, qlora_bf16 *dA, qlora_bf16 *dB, void *workspace,
+                              size_t workspace_bytes, qlora_stream_t stream) {
+  const Shape s{M, N, K, r};
+  qlora_status st = check_linear(packed, q, scale2, nf4, t8, s, alpha);
+  if (st != QLORA_OK) return st;
+  if (!X || !dY || !A || !B || !dX || !dA || !dB) return QLORA_ERR_NULL;
+  if (!aligned16(X) || !aligned16(dY) || !aligned16(A) || !aligned16(B) || (XA && !aligned16(XA)) ||
+      !aligned16(dX) || !aligned16(dA) || !aligned16(dB) || !aligned16(workspace))
+    return QLORA_ERR_ALIGN;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != QLORA_OK) return st;
+  if (!workspace || workspace_bytes < bwd_ws_bytes(s, d.sms)) return QLORA_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const float scl = alpha / static_cast<float>(r);
+
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const size_t mr = align256(static_cast<size_t>(M) * r * 2);
+  qlora_bf16 *gs = reinterpret_cast<qlora_bf16 *>(ws);
+  qlora_bf16 *xa_ws = reinterpret_cast<qlora_bf16 *>(ws + mr);
+  float *part = reinterpret_cast<float *>(ws + 2 * mr);
+
+  // 1) Gs = bf16(s * dY B^T)
+  st = skinny(SK_G, dY, N, M, B, N, r, M, N, r, scl, gs, r, 0.0f, nullptr, 0, false, part, d.sms, cs);
+  if (st != QLORA_OK) return st;
+
+  // 2) dX^T[k, m] = W'^T[k, :] . dY[m, :] + A[k, :] . Gs[m, :]
+  const FusedPlan fp = plan_fused(M, K, N / 64, d.sms);
+  GemmArgs a;
+  std::memset(&a, 0, sizeof a);
+  if (!map_kmajor(&a.tm_b, dY, N, M, fp.bn) ||
+      !make_map(&a.tm_pk, packed, false, K / 2, N, K / 2, 64, 64, false) || !map_kmajor(&a.tm_a2, A, r, K, 128) ||
+      !map_kmajor(&a.tm_b2, gs, r, M, fp.bn))
+    return QLORA_ERR_CUDA;
+  a.q = q;
+  a.scale2 = scale2;
+  a.w_kblocks = K / 64;
+  a.w_rows = static_cast<int>(N);
+  a.rows = static_cast<int>(K);
+  a.cols = static_cast<int>(M);
+  a.kblocks = static_cast<int>(N / 64);
+  a.splits = fp.splits;
+  a.lora_kblocks = static_cast<int>(cdiv(r, 64));
+  a.out_scale = 1.0f;
+  std::memcpy(a.nf4, nf4, sizeof a.nf4);
+  std::memcpy(a.t8, t8, sizeof a.t8);
+  if (fp.splits == 1) {
+    a.out = dX;
+    a.out_ld = K;
+  } else {
+    a.out = part;
+  }
+  st = fp.bn == 32 ? run_fused_bn<32, A_DEQ_MN, L2_A_K>(a, d.sms, cs)
+                   : run_fused_bn<256, A_DEQ_MN, L2_A_K>(a, d.sms, cs);
+  if (st != QLORA_OK) return st;
+  if (fp.splits > 1) {
+    st = launch_reduce(part, fp.splits, static_cast<int>(K), static_cast<int>(M), cdiv(K, 128) * 128,
+                       cdiv(M, fp.bn) * fp.bn, 1.0f, dX, K, 0.0f, nullptr, 0, true, d.sms, cs);
+    if (st != QLORA_OK) return st;
+  }
+
+  // 3) dA = X^T Gs   ([K, r])
+  st = skinny(SK_DA, X, K, M, gs, r, M, K, M, r, 1.0f, dA, r, 0.0f, nullptr, 0, false, part, d.sms, cs);
+  if (st != QLORA_OK) return st;
+
+  // 4) XA (saved or recomputed), then dB = s XA^T dY   ([r, N], from dB^T[n, j])
+  const qlora_bf16 *xa = XA;
+  if (xa == nullptr) {
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, 1.0f, xa_ws, r, 0.0f, nullptr, 0, false, part, d.sms, cs);
+    if (st != QLORA_OK) return st;
+    xa = xa_ws;
+  }
+  return skinny(SK_DB, dY, N, M, xa, r, M, N, M, r, scl, dB, N, 0.0f, nullptr, 0, true, part, d.sms, cs);
+}
+
+uint32_t qlora_device_error(int clear) {
+  unsigned int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return 0xFFFFFFFFu;
+  if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof v) != cudaSuccess) return 0xFFFFFFFFu;
+  if (clear) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &z, sizeof z) != cudaSuccess) return 0xFFFFFFFFu;
+  }
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,193 @@
+/*
+ * qlora.h — C ABI of libqlora.so: the frozen-base linear layer of QLoRA on
+ * one B200 (sm_100a).
+ *
+ * The method (QLoRA pages: intvml.com "DL0087 QLoRA: 4-bit Quantized LoRA";
+ * promptingindex.com "QLoRA: Finetuning 65B Models on a Single GPU";
+ * systemoverflow.com "QLoRA ... at Extreme Scale"): a frozen weight W [N, K]
+ * is stored as 4-bit NF4 codes in blocks of 64 with one absmax constant per
+ * block; the constants are themselves quantized to 8 bits with one fp32
+ * scale per 256 constants ("double quantization"). On every forward and
+ * backward pass each block is dequantized to bf16 just before the matmul and
+ * discarded, and the bf16 low-rank adapters A [K, r], B [r, N] (scale
+ * alpha / r) are the only tensors that receive gradients.
+ *
+ * Conventions for every call
+ *   - Pointers named *device* live in device memory of the current device;
+ *     tables (nf4, t8) are HOST pointers, read during the call.
+ *   - Matrices are dense, row-major, contiguous. bf16 values travel as their
+ *     16-bit patterns (qlora_bf16).
+ *   - The caller owns every buffer. The library allocates no device memory;
+ *     scratch space is the caller's `workspace` (size from
+ *     qlora_workspace_bytes).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t, passed as void*;
+ *     NULL = legacy default stream). Arguments are checked on the host
+ *     before anything is launched: a failed check returns its status and
+ *     launches nothing. A launch failure returns QLORA_ERR_CUDA. The library
+ *     never exits, traps or prints.
+ *   - Every device-side wait is bounded; a wait that runs out sets a bit in
+ *     the device error word (qlora_device_error) and the kernel returns.
+ *   - Outputs are overwritten, never accumulated into.
+ */
+#ifndef QLORA_H_
+#define QLORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#define QLORA_ABI_VERSION 1
+#define QLORA_BLOCK 64          /* weights per absmax constant (DL0087 component 2)        */
+#define QLORA_DQ_BLOCK 256      /* constants per second-level fp32 scale (DL0087 comp. 3) */
+#define QLORA_NF4_LEVELS 16     /* 4-bit code -> level table                              */
+#define QLORA_DQ_LEVELS 256     /* 8-bit code -> constant level table                     */
+#define QLORA_MAX_RANK 256      /* largest adapter rank r accepted                        */
+
+typedef uint16_t qlora_bf16;    /* bf16 bit pattern                                       */
+typedef void *qlora_stream_t;   /* a cudaStream_t                                         */
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_NULL = 1,        /* a required pointer is NULL                               */
+  QLORA_ERR_SHAPE = 2,       /* a size is out of range or not a multiple it must be      */
+  QLORA_ERR_ALIGN = 3,       /* a device pointer is not 16-byte aligned                  */
+  QLORA_ERR_RANGE = 4,       /* a scalar (r, alpha) is out of range                      */
+  QLORA_ERR_CUDA = 5,        /* a CUDA runtime/driver call or a launch failed            */
+  QLORA_ERR_UNSUPPORTED = 6, /* the current device is not sm_100                         */
+  QLORA_ERR_WORKSPACE = 7,   /* workspace NULL or smaller than qlora_workspace_bytes     */
+  QLORA_ERR_TABLE = 8        /* a code table is not finite and strictly ascending, or the
+                                NF4 table has no exact 0.0f                              */
+} qlora_status;
+
+/* Human-readable name of a status (static string). */
+QLORA_API const char *qlora_status_string(qlora_status s);
+
+/* QLORA_ABI_VERSION of the built library. */
+QLORA_API int qlora_abi_version(void);
+
+/*
+ * The library's default code tables (host, no device work).
+ *
+ * qlora_nf4_levels: the 16 ascending NF4 levels — standard-normal quantiles
+ * rescaled to [-1, 1] with an exact zero, equal probability mass per level
+ * on each side (promptingindex.com "4-bit NormalFloat"; DL0087 formulation
+ * list). Sixteen is even, so the split is 7 negative, 0, 8 positive; the
+ * outermost probability is delta = ((1 - 1/30) + (1 - 1/32)) / 2.
+ * qlora_dq_levels: the 256 ascending 8-bit constant levels k/255 (the pages
+ * fix only "8-bit"; an unsigned linear map is taken, the constants being
+ * non-negative). Any other ascending tables may be passed to the calls.
+ */
+QLORA_API void qlora_nf4_levels(float out[16]);
+QLORA_API void qlora_dq_levels(float out[256]);
+
+/*
+ * Bytes of scratch that qlora_linear_fwd / qlora_linear_bwd need for this
+ * shape (the larger of the two). Returns 0 for shapes the calls reject.
+ */
+QLORA_API size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+
+/*
+ * Blockwise NF4 quantization (DL0087 components 1-2; sandgarden.com "QLoRA",
+ * workflow step "Load and Quantize").
+ *   W       device bf16 [N, K]
+ *   nf4     host float[16], ascending, finite, containing 0.0f
+ *   packed  device uint8 [N*K/2]: element 2j in the low nibble of byte j,
+ *           element 2j+1 in the high nibble
+ *   absmax  device float [N*K/64]: c_b = max |w| over the 64 consecutive
+ *           row-major elements of block b
+ * Code of an element: the count of fp32 midpoints (L[i]+L[i+1])*0.5f that
+ * lie strictly below x = w / c_b (IEEE fp32 division); a block of zeros
+ * encodes x = 0.
+ * Requires N >= 1, K >= 64, K % 64 == 0, 16-byte aligned W, packed, absmax.
+ */
+QLORA_API qlora_status qlora_quantize_nf4(const qlora_bf16 *W, int64_t N, int64_t K, const float nf4[16],
+                                uint8_t *packed, float *absmax, qlora_stream_t stream);
+
+/*
+ * Double quantization of the absmax constants (DL0087 component 3;
+ * promptingindex.com "Double Quantization and Paged Optimizers").
+ *   absmax  device float [nb] (non-negative)
+ *   t8      host float[256], ascending, finite
+ *   q       device uint8 [nb]: nearest 8-bit level of c / S_g (same
+ *           midpoint rule as the NF4 code; a group of zeros encodes 0)
+ *   scale2  device float [ceil(nb/256)]: S_g = max of the 256 consecutive
+ *           constants of group g (the last group may be shorter; groups
+ *           straddle weight rows)
+ * Requires nb >= 1, 16-byte aligned pointers.
+ */
+QLORA_API qlora_status qlora_double_quant(const float *absmax, int64_t nb, const float t8[256],
+                                uint8_t *q, float *scale2, qlora_stream_t stream);
+
+/*
+ * Dequantization to bf16 (DL0087, opening paragraph and Figure 1):
+ *   W_out[e] = bf16_rne( nf4[code_e] * c'_b ),  c'_b = t8[q_b] * scale2[b/256],
+ * both products in fp32. Bit-identical to the bf16 weight the two linear
+ * calls feed to their tensor-core MMAs (they never write it to memory).
+ *   packed, q, scale2 as produced above; W_out device bf16 [N, K].
+ */
+QLORA_API qlora_status qlora_dequant(const uint8_t *packed, const uint8_t *q, const float *scale2,
+                           int64_t N, int64_t K, const float nf4[16], const float t8[256],
+                           qlora_bf16 *W_out, qlora_stream_t stream);
+
+/*
+ * QLoRA linear forward (DL0087 Figure 1 and formulation list):
+ *   Y = X W'^T + s (X A) B,   s = alpha / r,
+ * W' the dequantized weight, rebuilt tile by tile inside the GEMM mainloop.
+ *   X [M, K], A [K, r], B [r, N], Y [M, N]: device bf16.
+ *   XA_out: device bf16 [M, r] receiving X A (unscaled) for the backward, or
+ *           NULL.
+ *   workspace: device scratch of at least qlora_workspace_bytes(M, N, K, r).
+ * Accumulation in fp32; (X A) is rounded to bf16 (times s) before its
+ * rank-r product. Requires M >= 1, N % 64 == 0, K % 64 == 0, N, K >= 64,
+ * 1 <= r <= 256, r % 8 == 0, alpha finite, 16-byte aligned pointers.
+ */
+QLORA_API qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const float *scale2,
+                              const float nf4[16], const float t8[256],
+                              int64_t M, int64_t N, int64_t K,
+                              const qlora_bf16 *X, const qlora_bf16 *A, const qlora_bf16 *B,
+                              int r, float alpha, qlora_bf16 *Y, qlora_bf16 *XA_out,
+                              void *workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/*
+ * QLoRA linear backward through the frozen base (DL0087 component 4;
+ * sandgarden.com workflow "Fine-Tune the Adapters"): W' is dequantized
+ * again inside the mainloop (recompute, no stored bf16 copy) and gradients
+ * stop at the adapters — there is no dW.
+ *   G  = dY B^T
+ *   dX = dY W' + s G A^T
+ *   dA = s X^T G
+ *   dB = s (X A)^T dY
+ *   X [M, K], dY [M, N], A [K, r], B [r, N]: device bf16.
+ *   XA: device bf16 [M, r] saved by the forward, or NULL to recompute X A.
+ *   dX [M, K], dA [K, r], dB [r, N]: device bf16 outputs.
+ * Same requirements as qlora_linear_fwd.
+ */
+QLORA_API qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const float *scale2,
+                              const float nf4[16], const float t8[256],
+                              int64_t M, int64_t N, int64_t K,
+                              const qlora_bf16 *X, const qlora_bf16 *dY,
+                              const qlora_bf16 *A, const qlora_bf16 *B, const qlora_bf16 *XA,
+                              int r, float alpha, qlora_bf16 *dX, qlora_bf16 *dA, qlora_bf16 *dB,
+                              void *workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/*
+ * The device error word of the current device: bit 0 = a bounded pipeline
+ * wait ran out (the kernel returned early; its outputs are undefined).
+ * Synchronizes the device. clear != 0 resets the word. Returns 0xFFFFFFFF if
+ * the word cannot be read.
+ */
+QLORA_API uint32_t qlora_device_error(int clear);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_H_ */

@@ -1,0 +1,94 @@
+"""CPU-only checks of the C ABI: the library loads, exports every symbol that
+include/qlora.h declares, and its host-side argument checks return the
+documented status codes before anything touches a GPU (no compute calls).
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from bit_quantized_lora_blockwise_b200 import binding
+from bit_quantized_lora_blockwise_b200.build import LIB, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlora.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"QLORA_API\s+[\w\s\*]*?\b(qlora_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_five_calls():
+    syms = declared_symbols()
+    for name in ("qlora_quantize_nf4", "qlora_double_quant", "qlora_dequant", "qlora_linear_fwd",
+                 "qlora_linear_bwd"):
+        assert name in syms
+    assert set(syms) == set(binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert lib.qlora_abi_version() == 1
+
+
+def test_library_has_sm100a_code():
+    # the fatbin section must hold sm_100a code; nvcc records the arch in the ELF notes
+    data = open(LIB, "rb").read()
+    assert b"sm_100a" in data
+
+
+def test_status_strings(lib):
+    for code, name in binding._STATUS.items():
+        assert lib.qlora_status_string(code).decode() == name
+
+
+def test_host_tables_match_oracle(lib):
+    import oracle
+    assert np.array_equal(binding.nf4_levels(), oracle.nf4_levels())
+    assert np.array_equal(binding.dq_levels(), oracle.dq_levels())
+
+
+def _fake(addr=0x10000):
+    return ctypes.c_void_p(addr)
+
+
+def test_argument_checks_before_any_launch(lib):
+    tb = binding._tables(None, None)
+    s = ctypes.c_void_p(0)
+    # NULL pointers
+    assert lib.qlora_quantize_nf4(None, 64, 64, tb.nf4, _fake(), _fake(), s) == 1
+    assert lib.qlora_double_quant(_fake(), 10, tb.t8, None, _fake(), s) == 1
+    # shapes: K % 64, K < 64, N < 1
+    assert lib.qlora_quantize_nf4(_fake(), 64, 96, tb.nf4, _fake(), _fake(), s) == 2
+    assert lib.qlora_quantize_nf4(_fake(), 0, 64, tb.nf4, _fake(), _fake(), s) == 2
+    assert lib.qlora_double_quant(_fake(), 0, tb.t8, _fake(), _fake(), s) == 2
+    # alignment
+    assert lib.qlora_quantize_nf4(_fake(0x10008), 64, 64, tb.nf4, _fake(), _fake(), s) == 3
+    # tables: not ascending / no exact zero
+    bad = (ctypes.c_float * 16)(*np.linspace(-1, 1, 16).astype(np.float32))  # no exact 0
+    assert lib.qlora_quantize_nf4(_fake(), 64, 64, bad, _fake(), _fake(), s) == 8
+    desc = (ctypes.c_float * 256)(*np.linspace(1, 0, 256).astype(np.float32))
+    assert lib.qlora_double_quant(_fake(), 10, desc, _fake(), _fake(), s) == 8
+    # linear: r range, r % 8, N % 64, alpha finite
+    args = dict(M=16, N=128, K=128, r=8, alpha=16.0)
+
+    def fwd(**kw):
+        a = {**args, **kw}
+        return lib.qlora_linear_fwd(_fake(), _fake(), _fake(), tb.nf4, tb.t8, a["M"], a["N"], a["K"],
+                                    _fake(), _fake(), _fake(), a["r"], a["alpha"], _fake(), None,
+                                    _fake(), 1 << 30, s)
+    assert fwd(r=0) == 4 and fwd(r=300) == 4 and fwd(r=12) == 4
+    assert fwd(N=96) == 2 and fwd(K=32) == 2 and fwd(M=0) == 2
+    assert fwd(alpha=float("inf")) == 4
+    assert lib.qlora_workspace_bytes(16, 96, 128, 8) == 0
+    assert lib.qlora_workspace_bytes(16, 128, 128, 8) > 0
