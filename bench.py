@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA frozen-base linear hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Workload: the 7B-shaped linear set (q, k, v, o 4096x4096; gate, up
+4096->11008; down 11008->4096), M = 4 x 512 = 2048 tokens, r = 64,
+alpha = 16, W ~ N(0, 0.02) with 0.1 % outliers at +-10 sigma; synthetic
+seeded inputs, generated on the device before timing.
+
+One step = for every linear: qlora_quantize_nf4, qlora_double_quant,
+qlora_dequant, qlora_linear_fwd (saving XA), qlora_linear_bwd — every row of
+the hot path once. Under torchrun each rank runs its own batch (weak
+scaling, data parallel over tokens) and the adapter gradients dA, dB of
+every linear are summed across ranks with one NCCL all-reduce per step.
+
+`value` = fwd+bwd algorithmic FLOPs of all ranks / step time (max over
+ranks), sum over linears of 4MNK + 6Mr(N+K). The codec phases are reported
+in GB/s beside it. The reference arm (--impl reference) times the CPU
+oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "llama7b_set"
+METRIC = "QLoRA linear fwd+bwd TFLOP/s and quant/dequant GB/s, % of roofline, 1 B200"
+UNIT = "TFLOP/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["bit_quantized_lora_blockwise_b200/csrc/gemm.cuh",
+                  "bit_quantized_lora_blockwise_b200/csrc/codec.cuh",
+                  "bit_quantized_lora_blockwise_b200/csrc/ptx.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--linears", default="", help="comma list of linear names to keep (profiling runs)")
+    return ap.parse_args()
+
+
+def linear_flops(M, N, K, r):
+    return 4 * M * N * K + 6 * M * r * (N + K)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_key: str):
+    """Per-launch DRAM bytes of `kernel_key` from the committed ncu summary,
+    or None when there is none or the kernels changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    src = None
+    val = None
+    for ln in lines:
+        if ln.startswith("kernel_source_hash:"):
+            src = ln.split(":", 1)[1].strip()
+        if ln.startswith(kernel_key + ":"):
+            val = float(ln.split(":", 1)[1].strip())
+    if src != kernel_source_hash():
+        return None
+    return val
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle --
+def oracle_sample_step(wl, li=0, tokens=64):
+    """One bounded oracle step: the full codec chain on linear `li` and the
+    float64 forward+backward for `tokens` tokens. Returns its algorithmic
+    FLOPs (same convention as the GPU value)."""
+    import numpy as np
+    import torch
+    import oracle
+    from bit_quantized_lora_blockwise_b200.inputs import layer_inputs, bf16_bits
+    lin = wl.linears[li]
+    inp = layer_inputs(wl, li, tokens, device="cpu")
+    wb = bf16_bits(inp["W"])
+    pk, am = oracle.quantize_nf4(wb)
+    q, s2 = oracle.double_quant(am)
+    wq = oracle.dequant(pk, q, s2, lin.N * lin.K).reshape(lin.N, lin.K)
+    X, A, B, dY = (bf16_bits(inp[k]) for k in ("X", "A", "B", "dY"))
+    Y, XA = oracle.linear_fwd(X, wq, A, B, wl.alpha, wl.r)
+    dX, dA, dB = oracle.linear_bwd(X, dY, wq, A, B, wl.alpha, wl.r)
+    return linear_flops(tokens, lin.N, lin.K, wl.r), f"linear '{lin.name}' {lin.N}x{lin.K}: codec on all " \
+        f"{lin.N * lin.K} weights + fp64 fwd/bwd on {tokens} of {wl.M[0]} tokens"
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def cpu_baseline(wl, budget_s=12.0):
+    t0 = time.perf_counter()
+    flops = 0
+    n = 0
+    sample = ""
+    while True:
+        f, sample = oracle_sample_step(wl)
+        flops += f
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{n} x ({sample}); {dt:.1f} s"}
+
+
+def run_reference(args, rank):
+    from bit_quantized_lora_blockwise_b200.inputs import WORKLOADS
+    if rank != 0:
+        return
+    wl = WORKLOADS[WORKLOAD]
+    for _ in range(args.warmup):
+        oracle_sample_step(wl)
+    t0 = time.perf_counter()
+    flops = 0
+    sample = ""
+    for _ in range(args.steps):
+        f, sample = oracle_sample_step(wl)
+        flops += f
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD, "sample_per_step": sample, "M": wl.M[0], "r": wl.r},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ native --
+class LinearState:
+    def __init__(self, wl, li, M, device):
+        import torch
+        from bit_quantized_lora_blockwise_b200 import binding
+        from bit_quantized_lora_blockwise_b200.inputs import layer_inputs
+        lin = wl.linears[li]
+        self.name, self.N, self.K, self.M, self.r, self.alpha = lin.name, lin.N, lin.K, M, wl.r, wl.alpha
+        inp = layer_inputs(wl, li, M, device=device)
+        self.W, self.X, self.A, self.B, self.dY = (inp[k] for k in ("W", "X", "A", "B", "dY"))
+        N, K, r = self.N, self.K, self.r
+        e = dict(device=device)
+        self.packed = torch.empty(N * K // 2, dtype=torch.uint8, **e)
+        self.absmax = torch.empty(N * K // 64, dtype=torch.float32, **e)
+        self.q = torch.empty(N * K // 64, dtype=torch.uint8, **e)
+        self.scale2 = torch.empty((N * K // 64 + 255) // 256, dtype=torch.float32, **e)
+        self.Wq = torch.empty((N, K), dtype=torch.bfloat16, **e)
+        self.Y = torch.empty((M, N), dtype=torch.bfloat16, **e)
+        self.XA = torch.empty((M, r), dtype=torch.bfloat16, **e)
+        self.dX = torch.empty((M, K), dtype=torch.bfloat16, **e)
+        self.dA = torch.empty((K, r), dtype=torch.bfloat16, **e)
+        self.dB = torch.empty((r, N), dtype=torch.bfloat16, **e)
+        self.ws_bytes = binding.workspace_bytes(M, N, K, r)
+
+    def flops(self):
+        return linear_flops(self.M, self.N, self.K, self.r)
+
+    def codec_bytes(self):
+        n = self.N * self.K
+        return {"quantize": n * 2 + n // 2 + n // 64 * 4,
+                "double_quant": n // 64 * 4 + n // 64 + ((n // 64 + 255) // 256) * 4,
+                "dequant": n // 2 + n // 64 + ((n // 64 + 255) // 256) * 4 + n * 2}
+
+
+def run_native(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from bit_quantized_lora_blockwise_b200 import binding
+    from bit_quantized_lora_blockwise_b200.build import build
+    from bit_quantized_lora_blockwise_b200.inputs import WORKLOADS
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    build()
+    binding.load()
+    wl = WORKLOADS[WORKLOAD]
+    M = wl.M[0]
+    keep = [n for n in args.linears.split(",") if n]
+    layers = [LinearState(wl, i, M, dev) for i in range(len(wl.linears))
+              if not keep or wl.linears[i].name in keep]
+    ws = torch.empty(max(l.ws_bytes for l in layers), dtype=torch.uint8, device=dev)
+    nl = len(layers)
+
+    def ev():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        return e
+
+    # per step, per linear: events around the codec calls and the fused GEMMs
+    def make_events():
+        return [{k: (ev(), ev()) for k in ("quantize", "double_quant", "dequant", "fwd_gemm", "bwd_gemm")}
+                for _ in range(nl)]
+
+    def step(evs=None):
+        for i, L in enumerate(layers):
+            e = evs[i] if evs else None
+            if e: e["quantize"][0].record()
+            binding.quantize_nf4(L.W, packed=L.packed, absmax=L.absmax)
+            if e: e["quantize"][1].record(); e["double_quant"][0].record()
+            binding.double_quant(L.absmax, q=L.q, scale2=L.scale2)
+            if e: e["double_quant"][1].record(); e["dequant"][0].record()
+            binding.dequant(L.packed, L.q, L.scale2, L.N, L.K, out=L.Wq)
+            if e: e["dequant"][1].record(); binding.set_trace_events(*e["fwd_gemm"])
+            binding.linear_fwd(L.packed, L.q, L.scale2, L.X, L.A, L.B, L.alpha, L.N, L.K, Y=L.Y,
+                               XA_out=L.XA, workspace=ws)
+            if e: binding.set_trace_events(*e["bwd_gemm"])
+            binding.linear_bwd(L.packed, L.q, L.scale2, L.X, L.dY, L.A, L.B, L.alpha, L.N, L.K, XA=L.XA,
+                               dX=L.dX, dA=L.dA, dB=L.dB, workspace=ws)
+            if e: binding.set_trace_events(None, None)
+        if world > 1:
+            # data parallel over tokens: sum the adapter gradients of all ranks
+            flat = torch.cat([t.view(-1) for L in layers for t in (L.dA, L.dB)]).float()
+            dist.all_reduce(flat)
+            off = 0
+            for L in layers:
+                for t in (L.dA, L.dB):
+                    n = t.numel()
+                    t.copy_(flat[off:off + n].view_as(t))
+                    off += n
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    evs_steps = [make_events() for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    launches0 = binding.launch_count()
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start.record()
+    for k in range(args.steps):
+        step(evs_steps[k])
+    t_stop.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = binding.launch_count() - launches0
+    clocks = sampler.stop()
+    ms = t_start.elapsed_time(t_stop) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    err = binding.device_error()
+
+    step_flops = sum(L.flops() for L in layers)
+    value = step_flops * world / (ms * 1e-3) / 1e12
+
+    # per-phase device times (mean over the timed steps)
+    phase = {k: [] for k in ("quantize", "double_quant", "dequant", "fwd_gemm", "bwd_gemm")}
+    for evs in evs_steps:
+        for k in phase:
+            phase[k].append(sum(evs[i][k][0].elapsed_time(evs[i][k][1]) for i in range(nl)))
+    phase_ms = {k: sum(v) / len(v) for k, v in phase.items()}
+    codec_bytes = {k: sum(L.codec_bytes()[k] for L in layers) for k in ("quantize", "double_quant", "dequant")}
+    gemm_flops = {"fwd_gemm": sum(2 * M * L.N * L.K + 2 * M * L.r * L.N for L in layers),
+                  "bwd_gemm": sum(2 * M * L.N * L.K + 2 * M * L.r * L.K for L in layers)}
+    pk, pk_kind = peaks()
+    hbm = pk["hbm_gbs"]
+    tc = pk["bf16_tflops_sustained"] if "bf16_tflops_sustained" in pk else pk["bf16_tflops"]
+    phases = {}
+    for k in ("quantize", "double_quant", "dequant"):
+        gbs = codec_bytes[k] / (phase_ms[k] * 1e-3) / 1e9
+        phases[k] = {"ms": round(phase_ms[k], 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
+    for k in ("fwd_gemm", "bwd_gemm"):
+        tf = gemm_flops[k] / (phase_ms[k] * 1e-3) / 1e12
+        phases[k] = {"ms": round(phase_ms[k], 4), "TFLOP/s": round(tf, 1), "frac_tensor": round(tf / tc, 3)}
+    # dominant kernel: the fused backward dequant-GEMM (largest share of the step)
+    dom = max(("fwd_gemm", "bwd_gemm"), key=lambda k: phase_ms[k])
+    achieved = gemm_flops[dom] / nl / (phase_ms[dom] / nl * 1e-3) / 1e12
+    traffic = profiled_traffic("qgemm_" + dom)
+    roofline = {"bound": "tensor", "kernel": f"fused dequant-GEMM ({dom.split('_')[0]}), per-launch average "
+                "over the 7 linears", "achieved": round(achieved, 1), "peak": tc,
+                "peak_kind": f"{pk_kind} bf16_tflops_sustained (kernel timed inside a long step)",
+                "unit": "TFLOP/s", "frac": round(achieved / tc, 4),
+                "traffic": traffic}
+
+    # ------------------------------------------------------------ e2e leg --
+    e2e = None
+    if not args.no_e2e:
+        host = []
+        for L in layers:
+            host.append({k: getattr(L, k).cpu().pin_memory() for k in ("W", "X", "A", "B", "dY")})
+        h2d = sum(t.numel() * t.element_size() for h in host for t in h.values())
+        outs = [(torch.empty_like(L.dA, device="cpu").pin_memory(), torch.empty_like(L.dB, device="cpu").pin_memory())
+                for L in layers]
+        d2h = sum(a.numel() * a.element_size() + b.numel() * b.element_size() for a, b in outs)
+
+        def e2e_step():
+            for L, h in zip(layers, host):
+                for k, t in h.items():
+                    getattr(L, k).copy_(t, non_blocking=True)
+            step()
+            for L, (a, b) in zip(layers, outs):
+                a.copy_(L.dA, non_blocking=True)
+                b.copy_(L.dB, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        e2e_steps = max(2, min(args.steps, 5))
+        if world > 1:
+            dist.barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for _ in range(e2e_steps):
+            e2e_step()
+        a1.record()
+        torch.cuda.synchronize()
+        ems = a0.elapsed_time(a1) / e2e_steps
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": step_flops * world / (ems * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ems,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "linears": [f"{L.name}:{L.N}x{L.K}" for L in layers],
+                           "M": M, "r": wl.r, "alpha": wl.alpha, "per_rank_tokens": M,
+                           "parallelism": f"dp{world}",
+                           "l2": "inputs larger than L2 (405 MB of bf16 weights + 320 MB of activations per step)",
+                           "step": "per linear: quantize_nf4, double_quant, dequant, linear_fwd, linear_bwd"},
+                "phases": phases, "roofline": roofline, "gpu_launches": launches,
+                "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "device_error": err}
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        if args.impl == "reference":
+            if rank == 0:
+                run_reference(args, rank)
+            return
+        import torch
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        try:
+            run_native(args, rank, world, local_rank)
+        finally:
+            dist.destroy_process_group()
+        return
+    if args.impl == "reference":
+        run_reference(args, rank)
+    else:
+        run_native(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -31,7 +31,8 @@ _STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_NULL", 2: "QLORA_ERR_SHAPE", 3: "QLORA_E
 # every symbol include/qlora.h declares
 EXPORTS = ("qlora_status_string", "qlora_abi_version", "qlora_nf4_levels", "qlora_dq_levels",
            "qlora_workspace_bytes", "qlora_quantize_nf4", "qlora_double_quant", "qlora_dequant",
-           "qlora_linear_fwd", "qlora_linear_bwd", "qlora_device_error")
+           "qlora_linear_fwd", "qlora_linear_bwd", "qlora_device_error", "qlora_set_trace_events",
+           "qlora_launch_count")
 
 
 class QLoRAError(RuntimeError):
@@ -68,6 +69,9 @@ def load(path: str | None = None):
                                          P, SZ, P]
         lib.qlora_device_error.argtypes = [I32]
         lib.qlora_device_error.restype = ctypes.c_uint32
+        lib.qlora_set_trace_events.argtypes = [P, P]
+        lib.qlora_set_trace_events.restype = None
+        lib.qlora_launch_count.restype = ctypes.c_uint64
         for fn in ("qlora_quantize_nf4", "qlora_double_quant", "qlora_dequant", "qlora_linear_fwd",
                    "qlora_linear_bwd"):
             getattr(lib, fn).restype = I32
@@ -156,6 +160,20 @@ def workspace_bytes(M: int, N: int, K: int, r: int) -> int:
 
 def device_error(clear: bool = False) -> int:
     return int(load().qlora_device_error(1 if clear else 0))
+
+
+def launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(load().qlora_launch_count())
+
+
+def set_trace_events(start=None, stop=None):
+    """Record torch.cuda.Event `start`/`stop` around the fused GEMM kernel of
+    the following linear_fwd / linear_bwd calls (None, None to stop)."""
+    if start is None or stop is None:
+        load().qlora_set_trace_events(None, None)
+    else:
+        load().qlora_set_trace_events(ctypes.c_void_p(start.cuda_event), ctypes.c_void_p(stop.cuda_event))
 
 
 def quantize_nf4(W: torch.Tensor, nf4=None, packed=None, absmax=None):

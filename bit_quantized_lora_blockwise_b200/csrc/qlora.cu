@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -34,6 +35,15 @@ struct DeviceInfo {
 };
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
+std::atomic<uint64_t> g_launches{0};
+thread_local cudaEvent_t t_trace_start = nullptr;
+thread_local cudaEvent_t t_trace_stop = nullptr;
+
+// Every kernel launch goes through here: counts it and maps a launch error.
+qlora_status launched() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
 
 qlora_status device_info(DeviceInfo *out) {
   int dev = 0;
@@ -150,7 +160,7 @@ qlora_status launch_gemm(const GemmArgs &args, int sms, cudaStream_t stream) {
   const int tiles = row_tiles * col_tiles * args.splits;
   const int grid = tiles < sms ? tiles : sms;
   qgemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(args);
-  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return launched();
 }
 
 qlora_status launch_reduce(const float *part, int splits, int rows, int cols, int64_t rows_pad,
@@ -162,7 +172,7 @@ qlora_status launch_reduce(const float *part, int splits, int rows, int cols, in
                                                  reinterpret_cast<__nv_bfloat16 *>(out), ld, scale2,
                                                  reinterpret_cast<__nv_bfloat16 *>(out2), ld2,
                                                  transpose ? 1 : 0);
-  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return launched();
 }
 
 // ------------------------------------------------------- skinny GEMMs --
@@ -301,6 +311,13 @@ size_t bwd_ws_bytes(const Shape &s, int sms) {
   return 2 * mr + part;
 }
 
+void trace_begin(cudaStream_t s) {
+  if (t_trace_start && t_trace_stop) cudaEventRecord(t_trace_start, s);
+}
+void trace_end(cudaStream_t s) {
+  if (t_trace_start && t_trace_stop) cudaEventRecord(t_trace_stop, s);
+}
+
 qlora_status check_linear(const uint8_t *packed, const uint8_t *q, const float *scale2, const float *nf4,
                           const float *t8, const Shape &s, float alpha) {
   if (!packed || !q || !scale2 || !nf4 || !t8) return QLORA_ERR_NULL;
@@ -387,7 +404,7 @@ qlora_status qlora_quantize_nf4(const qlora_bf16 *W, int64_t N, int64_t K, const
   quantize_nf4_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const uint4 *>(W), nblocks, reinterpret_cast<uint32_t *>(packed), absmax,
       make_tables(nf4, nullptr));
-  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return launched();
 }
 
 qlora_status qlora_double_quant(const float *absmax, int64_t nb, const float t8[256], uint8_t *q, float *scale2,
@@ -403,7 +420,7 @@ qlora_status qlora_double_quant(const float *absmax, int64_t nb, const float t8[
   const int grid = grid_for(ng, 8, d.sms, 16);
   double_quant_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(absmax, nb, q, scale2,
                                                                             make_tables(nullptr, t8));
-  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return launched();
 }
 
 qlora_status qlora_dequant(const uint8_t *packed, const uint8_t *q, const float *scale2, int64_t N, int64_t K,
@@ -420,7 +437,7 @@ qlora_status qlora_dequant(const uint8_t *packed, const uint8_t *q, const float 
   dequant_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const uint2 *>(packed), q, scale2, quarters, reinterpret_cast<uint4 *>(W_out),
       make_tables(nf4, t8));
-  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return launched();
 }
 
 qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const float *scale2, const float nf4[16],
@@ -478,8 +495,10 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   } else {
     a.out = part;
   }
+  trace_begin(cs);
   st = fp.bn == 32 ? run_fused_bn<32, A_DEQ_K, L2_A_MN>(a, d.sms, cs)
                    : run_fused_bn<256, A_DEQ_K, L2_A_MN>(a, d.sms, cs);
+  trace_end(cs);
   if (st != QLORA_OK || fp.splits == 1) return st;
   return launch_reduce(part, fp.splits, static_cast<int>(N), static_cast<int>(M), cdiv(N, 128) * 128,
                        cdiv(M, fp.bn) * fp.bn, 1.0f, Y, N, 0.0f, nullptr, 0, true, d.sms, cs);
@@ -539,8 +558,10 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   } else {
     a.out = part;
   }
+  trace_begin(cs);
   st = fp.bn == 32 ? run_fused_bn<32, A_DEQ_MN, L2_A_K>(a, d.sms, cs)
                    : run_fused_bn<256, A_DEQ_MN, L2_A_K>(a, d.sms, cs);
+  trace_end(cs);
   if (st != QLORA_OK) return st;
   if (fp.splits > 1) {
     st = launch_reduce(part, fp.splits, static_cast<int>(K), static_cast<int>(M), cdiv(K, 128) * 128,
@@ -561,6 +582,13 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   }
   return skinny(SK_DB, dY, N, M, xa, r, M, N, M, r, scl, dB, N, 0.0f, nullptr, 0, true, part, d.sms, cs);
 }
+
+void qlora_set_trace_events(void *start, void *stop) {
+  t_trace_start = static_cast<cudaEvent_t>(start);
+  t_trace_stop = static_cast<cudaEvent_t>(stop);
+}
+
+uint64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 uint32_t qlora_device_error(int clear) {
   unsigned int v = 0;

@@ -187,6 +187,21 @@ QLORA_API qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q,
  */
 QLORA_API uint32_t qlora_device_error(int clear);
 
+/*
+ * Measurement instrumentation (no counterpart on the pages).
+ *
+ * qlora_set_trace_events: when both are non-NULL, the next qlora_linear_fwd
+ * and qlora_linear_bwd calls on this host thread record `start` (a
+ * cudaEvent_t) on their stream just before their fused dequant-GEMM kernel
+ * and `stop` just after it, so a caller can time that kernel alone with
+ * cudaEventElapsedTime. Pass NULL, NULL to stop. The events stay owned by the
+ * caller.
+ * qlora_launch_count: the number of kernels this library has launched in
+ * this process (all devices, all threads).
+ */
+QLORA_API void qlora_set_trace_events(void *start, void *stop);
+QLORA_API uint64_t qlora_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif
