@@ -258,6 +258,7 @@ def run_native(args, rank, world, local_rank):
     import torch.distributed as dist
     from bit_quantized_lora_blockwise_b200 import binding
     from bit_quantized_lora_blockwise_b200.build import build
+    from bit_quantized_lora_blockwise_b200.dp import allreduce_adapter_grads
     from bit_quantized_lora_blockwise_b200.inputs import WORKLOADS
 
     if not torch.cuda.is_available():
@@ -302,14 +303,7 @@ def run_native(args, rank, world, local_rank):
             if e: binding.set_trace_events(None, None)
         if world > 1:
             # data parallel over tokens: sum the adapter gradients of all ranks
-            flat = torch.cat([t.view(-1) for L in layers for t in (L.dA, L.dB)]).float()
-            dist.all_reduce(flat)
-            off = 0
-            for L in layers:
-                for t in (L.dA, L.dB):
-                    n = t.numel()
-                    t.copy_(flat[off:off + n].view_as(t))
-                    off += n
+            allreduce_adapter_grads([t for L in layers for t in (L.dA, L.dB)])
 
     for _ in range(args.warmup):
         step()
