@@ -32,7 +32,9 @@ _STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_NULL", 2: "QLORA_ERR_SHAPE", 3: "QLORA_E
 EXPORTS = ("qlora_status_string", "qlora_abi_version", "qlora_nf4_levels", "qlora_dq_levels",
            "qlora_workspace_bytes", "qlora_quantize_nf4", "qlora_double_quant", "qlora_dequant",
            "qlora_linear_fwd", "qlora_linear_bwd", "qlora_device_error", "qlora_set_trace_events",
-           "qlora_launch_count")
+           "qlora_launch_count", "qlora_linear_fwd_noalloc")
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class QLoRAError(RuntimeError):
@@ -65,6 +67,8 @@ def load(path: str | None = None):
         lib.qlora_double_quant.argtypes = [P, I64, P, P, P, P]
         lib.qlora_dequant.argtypes = [P, P, P, I64, I64, P, P, P, P]
         lib.qlora_linear_fwd.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, P, I32, F32, P, P, P, SZ, P]
+        lib.qlora_linear_fwd_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, P, I32, F32, P, P, P]
+        lib.qlora_linear_fwd_noalloc.restype = I32
         lib.qlora_linear_bwd.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, P, P, P, I32, F32, P, P, P,
                                          P, SZ, P]
         lib.qlora_device_error.argtypes = [I32]
@@ -249,6 +253,28 @@ def linear_fwd(packed, q, scale2, X, A, B, alpha: float, N: int, K: int, nf4=Non
     _check(load().qlora_linear_fwd(_ptr(packed), _ptr(q), _ptr(scale2), tb.nf4, tb.t8, M, N, K, _ptr(X),
                                    _ptr(A), _ptr(B), r, float(alpha), _ptr(Y), _ptr(XA_out),
                                    _ptr(workspace), workspace.numel(), _stream()), "qlora_linear_fwd")
+    return Y
+
+
+def linear_fwd_noalloc(packed, q, scale2, X, A, B, alpha: float, N: int, K: int, nf4=None, t8=None,
+                       Y=None, XA_out=None):
+    """linear_fwd for callers that cannot allocate device memory: no workspace
+    argument; the library's fixed device scratch (NOALLOC_SCRATCH_BYTES) is
+    used instead. Y must be preallocated by such a caller (pass Y=...)."""
+    M = X.shape[0]
+    r = A.shape[1]
+    _req(X, "X", torch.bfloat16, (M, K))
+    _req(A, "A", torch.bfloat16, (K, r))
+    _req(B, "B", torch.bfloat16, (r, N))
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _req(Y, "Y", torch.bfloat16, (M, N))
+    if XA_out is not None:
+        _req(XA_out, "XA_out", torch.bfloat16, (M, r))
+    tb = _tables(nf4, t8)
+    _check(load().qlora_linear_fwd_noalloc(_ptr(packed), _ptr(q), _ptr(scale2), tb.nf4, tb.t8, M, N, K,
+                                           _ptr(X), _ptr(A), _ptr(B), r, float(alpha), _ptr(Y),
+                                           _ptr(XA_out), _stream()), "qlora_linear_fwd_noalloc")
     return Y
 
 

@@ -583,6 +583,50 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   return skinny(SK_DB, dY, N, M, xa, r, M, N, M, r, scl, dB, N, 0.0f, nullptr, 0, true, part, d.sms, cs);
 }
 
+}  // extern "C"
+
+// Scratch of qlora_linear_fwd_noalloc: a fixed array in device global memory,
+// one per GPU that loads the library, shared by every call on that GPU.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device with that device current (the host-side symbol is only a
+// stand-in and must never reach a kernel).
+qlora_status noalloc_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return QLORA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return QLORA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+qlora_status qlora_linear_fwd_noalloc(const uint8_t *packed, const uint8_t *q, const float *scale2,
+                                      const float nf4[16], const float t8[256], int64_t M, int64_t N, int64_t K,
+                                      const qlora_bf16 *X, const qlora_bf16 *A, const qlora_bf16 *B, int r,
+                                      float alpha, qlora_bf16 *Y, qlora_bf16 *XA_out, qlora_stream_t stream) {
+  const Shape s{M, N, K, r};
+  qlora_status st = check_linear(packed, q, scale2, nf4, t8, s, alpha);
+  if (st != QLORA_OK) return st;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != QLORA_OK) return st;
+  if (fwd_ws_bytes(s, d.sms) > QLORA_NOALLOC_SCRATCH_BYTES) return QLORA_ERR_WORKSPACE;
+  void *scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != QLORA_OK) return st;
+  return qlora_linear_fwd(packed, q, scale2, nf4, t8, M, N, K, X, A, B, r, alpha, Y, XA_out, scratch,
+                          QLORA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 void qlora_set_trace_events(void *start, void *stop) {
   t_trace_start = static_cast<cudaEvent_t>(start);
   t_trace_stop = static_cast<cudaEvent_t>(stop);

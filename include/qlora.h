@@ -188,6 +188,35 @@ QLORA_API qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q,
 QLORA_API uint32_t qlora_device_error(int clear);
 
 /*
+ * Forward without a caller workspace (the QLoRA pages have no counterpart:
+ * this is an integration convenience, not part of the method).
+ *
+ * Same arguments and result as qlora_linear_fwd, minus the workspace. It is
+ * for callers that cannot allocate device memory at all: code running as a
+ * plugin inside a host framework that owns every device allocation, or a
+ * latency-bound loop that must never enter the allocator. Its scratch is a
+ * static device array of QLORA_NOALLOC_SCRATCH_BYTES compiled into the
+ * library (each GPU that loads the library keeps it until the process
+ * exits); the call itself allocates nothing.
+ *   - A shape whose forward scratch (qlora_workspace_bytes' forward share)
+ *     exceeds QLORA_NOALLOC_SCRATCH_BYTES returns QLORA_ERR_WORKSPACE and
+ *     launches nothing.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the previous
+ *     call's contents (nothing in it needs to start at zero). Calls whose
+ *     kernels overlap on the GPU (different streams, no ordering) race on
+ *     it: order them.
+ */
+#define QLORA_NOALLOC_SCRATCH_BYTES (8u << 20)
+QLORA_API qlora_status qlora_linear_fwd_noalloc(const uint8_t *packed, const uint8_t *q,
+                                                const float *scale2, const float nf4[16],
+                                                const float t8[256], int64_t M, int64_t N, int64_t K,
+                                                const qlora_bf16 *X, const qlora_bf16 *A,
+                                                const qlora_bf16 *B, int r, float alpha, qlora_bf16 *Y,
+                                                qlora_bf16 *XA_out, qlora_stream_t stream);
+
+/*
  * Measurement instrumentation (no counterpart on the pages).
  *
  * qlora_set_trace_events: when both are non-NULL, the next qlora_linear_fwd

@@ -1,0 +1,70 @@
+"""GPU test of qlora_linear_fwd_noalloc, the forward for callers that cannot
+allocate device memory (a plugin inside a framework that owns every device
+allocation, or a loop that must never enter the allocator).
+
+The entry point takes no workspace: it runs the forward on the library's
+fixed device scratch array. Its output must match the ordinary
+qlora_linear_fwd (caller workspace) within the layer tolerance, on two calls
+in a row with different inputs (the scratch keeps the previous call's
+contents, so the second call checks that nothing leaks between calls), and a
+shape whose scratch would exceed the fixed size must be refused.
+
+Named test_zz_* so that pytest collects it last.
+"""
+import numpy as np
+import pytest
+import torch
+
+from bit_quantized_lora_blockwise_b200 import binding
+from bit_quantized_lora_blockwise_b200.inputs import normal_bf16, weight_bf16
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-2
+
+
+def _rel(a: torch.Tensor, b: torch.Tensor) -> float:
+    a64 = a.float().cpu().numpy().astype(np.float64)
+    b64 = b.float().cpu().numpy().astype(np.float64)
+    den = np.max(np.abs(b64))
+    return float(np.max(np.abs(a64 - b64)) / (den if den > 0 else 1.0))
+
+
+def _layer(M, N, K, r, seed):
+    W = weight_bf16(N, K, 0.02, seed, 0.001).cuda()
+    pk, am = binding.quantize_nf4(W)
+    q, s2 = binding.double_quant(am)
+    X = normal_bf16((M, K), 1.0, seed + 1).cuda()
+    A = normal_bf16((K, r), 0.01, seed + 2).cuda()
+    B = normal_bf16((r, N), 0.01, seed + 3).cuda()
+    return pk, q, s2, X, A, B
+
+
+@pytest.mark.parametrize("M,N,K,r", [(16, 1024, 1024, 8), (40, 256, 192, 16), (4, 2048, 2048, 64),
+                                     (2048, 4096, 1024, 64)])
+def test_noalloc_matches_workspace_forward_two_calls(M, N, K, r):
+    for call, seed in enumerate((11, 23)):
+        pk, q, s2, X, A, B = _layer(M, N, K, r, seed + M + N)
+        Y_ref = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        XA_ref = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+        binding.linear_fwd(pk, q, s2, X, A, B, 16.0, N, K, Y=Y_ref, XA_out=XA_ref)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        XA = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+        binding.linear_fwd_noalloc(pk, q, s2, X, A, B, 16.0, N, K, Y=Y, XA_out=XA)
+        torch.cuda.synchronize()
+        assert binding.device_error() == 0
+        assert _rel(Y, Y_ref) <= TOL, f"call {call}: Y"
+        assert _rel(XA, XA_ref) <= TOL, f"call {call}: XA"
+
+
+def test_noalloc_refuses_oversized_scratch():
+    M, N, K, r = 8192, 1024, 8192, 256
+    assert binding.workspace_bytes(M, N, K, r) > binding.NOALLOC_SCRATCH_BYTES
+    pk = torch.empty(N * K // 2, dtype=torch.uint8, device="cuda")
+    q = torch.empty(N * K // 64, dtype=torch.uint8, device="cuda")
+    s2 = torch.empty((N * K // 64 + 255) // 256, dtype=torch.float32, device="cuda")
+    X = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    A = torch.empty((K, r), dtype=torch.bfloat16, device="cuda")
+    B = torch.empty((r, N), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(binding.QLoRAError) as ei:
+        binding.linear_fwd_noalloc(pk, q, s2, X, A, B, 16.0, N, K)
+    assert ei.value.status == 7  # QLORA_ERR_WORKSPACE
