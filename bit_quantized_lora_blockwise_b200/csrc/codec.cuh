@@ -235,4 +235,32 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint2 *__restrict__ 
   }
 }
 
+// ------------------------------------------------------------------------
+// Decoded block constants for the GEMMs, block-major: cprime[kb * N + n] =
+// t8[q_b] * scale2[b / 256] (fp32 product), b = n * KB + kb. One thread per
+// (row n, 16 consecutive blocks); consecutive threads take consecutive rows
+// so every store instruction writes a contiguous run of one kb row.
+__global__ void __launch_bounds__(256) decode_constants_kernel(const uint8_t *__restrict__ q,
+                                                               const float *__restrict__ scale2,
+                                                               int64_t N, int64_t KB,
+                                                               float *__restrict__ cprime,
+                                                               const CodecTables tabs) {
+  __shared__ float s_t8[256];
+  s_t8[threadIdx.x] = tabs.t8[threadIdx.x];
+  __syncthreads();
+  const int64_t chunks = (KB + 15) / 16;
+  const int64_t total = N * chunks;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total; t += stride) {
+    const int64_t ch = t / N;
+    const int64_t n = t - ch * N;
+    const int64_t kb0 = ch * 16;
+    const int64_t kb1 = kb0 + 16 < KB ? kb0 + 16 : KB;
+    for (int64_t kb = kb0; kb < kb1; ++kb) {
+      const int64_t b = n * KB + kb;
+      cprime[kb * N + n] = __fmul_rn(s_t8[__ldg(q + b)], __ldg(scale2 + (b >> 8)));
+    }
+  }
+}
+
 }  // namespace qlora

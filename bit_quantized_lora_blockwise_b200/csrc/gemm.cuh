@@ -44,8 +44,7 @@ struct GemmArgs {
   CUtensorMap tm_pk;  // packed NF4 codes (dequant variants)
   CUtensorMap tm_a2;  // low-rank A2
   CUtensorMap tm_b2;  // low-rank B2
-  const uint8_t *q;       // 8-bit constant codes (dequant variants)
-  const float *scale2;    // second-level scales (dequant variants)
+  CUtensorMap tm_cp;  // decoded block constants c' [K/64][N] fp32 (dequant variants)
   void *out;              // EPI_BF16_T: bf16 out[col * out_ld + row]; EPI_F32: fp32 partials
   int64_t out_ld;
   int64_t w_kblocks;      // 64-blocks per weight row (K / 64)
@@ -57,39 +56,44 @@ struct GemmArgs {
   int w_rows;             // A_DEQ_K: rows of W (N)
   float out_scale;
   float nf4[16];
-  float t8[256];
 };
 
-template <int BN_, int ASRC_, int BSRC_, int L2_, int EPI_, int STAGES_, int NPW_>
+template <int BN_, int ASRC_, int BSRC_, int L2_, int EPI_, int SB_, int SA_, int SP_, int NPW_>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 64, BN = BN_;
   static constexpr int ASRC = ASRC_, BSRC = BSRC_, L2 = L2_, EPI = EPI_;
-  static constexpr int STAGES = STAGES_, NPW = NPW_;
+  static constexpr int SB = SB_, SA = SA_, SP = SP_, NPW = NPW_;
   static constexpr bool DEQ = ASRC_ >= A_DEQ_K;
   static constexpr bool A_MN = (ASRC_ == A_TMA_MN) || (ASRC_ == A_DEQ_MN);
   static constexpr bool B_MN = BSRC_ == B_TMA_MN;
   static constexpr int NGROUPS = NPW_ >= 4 ? NPW_ / 4 : 1;
-  static_assert(!DEQ || (NPW_ % 4 == 0 && NPW_ >= 4), "dequant needs whole producer groups");
+  static_assert(!DEQ || (NPW_ % 4 == 0 && NPW_ >= 4 && SP_ >= 2), "dequant needs producer groups and a P ring");
+  static_assert(DEQ || (SA_ == SB_ && SP_ == 0 && NPW_ == 0), "TMA-only A shares the B ring");
+  static_assert(DEQ || L2_ == L2_NONE, "low-rank steps only in the dequant variants");
   static_assert(BN_ % 16 == 0 && BN_ >= 16 && BN_ <= 256, "MMA N");
   static_assert(!B_MN || BN_ % 64 == 0, "MN-major B needs whole 64-wide chunks");
   static constexpr int A_BYTES = BM * BK * 2;  // 16 KB
   static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int P_BYTES = DEQ ? 4096 : 0;
-  static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_P = OFF_B + STAGES * B_BYTES;
-  static constexpr int OFF_BAR = OFF_P + STAGES * P_BYTES;
-  // barriers: tma_full[S], deq_full[S], empty[S], tmem_full[2], tmem_empty[2], drain
-  static constexpr int NBARS = 3 * STAGES + 5;
-  static constexpr int OFF_T8 = OFF_BAR + NBARS * 8;
-  static constexpr int OFF_MISC = OFF_T8 + 256 * 4;  // tmem base, abort flag
+  // P slot: packed codes of one 128 x 64 weight tile, then the 128 decoded
+  // block constants c' of its (row, block) pairs; both by TMA.
+  static constexpr int PK_BYTES = 4096;
+  static constexpr int P_CP = PK_BYTES;
+  static constexpr int P_BYTES = P_CP + 512;
+  static constexpr int OFF_B = 0;
+  static constexpr int OFF_A = OFF_B + SB * B_BYTES;
+  static constexpr int OFF_P = OFF_A + SA * A_BYTES;
+  static constexpr int OFF_BAR = OFF_P + SP * P_BYTES;
+  // b_full[SB] b_empty[SB] a_full[SA] a_empty[SA] p_full[SP] p_empty[SP]
+  // tmem_full[2] tmem_empty[2] drain
+  static constexpr int NBARS = 2 * SB + 2 * SA + 2 * SP + 5;
+  static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem base, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
-  static constexpr int WARPS = 6 + NPW_;
+  static constexpr int WARPS = DEQ ? 7 + NPW_ : 6;
   static constexpr int THREADS = WARPS * 32;
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64
                                         : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-  static constexpr uint32_t MAIN_TX = B_BYTES + (DEQ ? P_BYTES : A_BYTES);
+  static constexpr uint32_t MAIN_TX = B_BYTES + (DEQ ? 0 : A_BYTES);
   static constexpr uint32_t LORA_TX = A_BYTES + B_BYTES;
 };
 
@@ -130,21 +134,31 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
   const int lane = threadIdx.x & 31;
 
   const uint32_t bar0 = sbase + C::OFF_BAR;
-  auto tma_full = [&](int s) { return bar0 + 8u * s; };
-  auto deq_full = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (2 * C::STAGES + s); };
-  auto tmem_full = [&](int a) { return bar0 + 8u * (3 * C::STAGES + a); };
-  auto tmem_empty = [&](int a) { return bar0 + 8u * (3 * C::STAGES + 2 + a); };
-  const uint32_t drain_bar = bar0 + 8u * (3 * C::STAGES + 4);
-  float *s_t8 = reinterpret_cast<float *>(smem + C::OFF_T8);
+  auto b_full = [&](int s) { return bar0 + 8u * s; };
+  auto b_empty = [&](int s) { return bar0 + 8u * (C::SB + s); };
+  auto a_full = [&](int s) { return bar0 + 8u * (2 * C::SB + s); };
+  auto a_empty = [&](int s) { return bar0 + 8u * (2 * C::SB + C::SA + s); };
+  auto p_full = [&](int s) { return bar0 + 8u * (2 * C::SB + 2 * C::SA + s); };
+  auto p_empty = [&](int s) { return bar0 + 8u * (2 * C::SB + 2 * C::SA + C::SP + s); };
+  constexpr int TB = 2 * C::SB + 2 * C::SA + 2 * C::SP;
+  auto tmem_full = [&](int a) { return bar0 + 8u * (TB + a); };
+  auto tmem_empty = [&](int a) { return bar0 + 8u * (TB + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (TB + 4);
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
   volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(tma_full(s), 1);
-      mbar_init(deq_full(s), 4);
-      mbar_init(empty_bar(s), 1);
+    for (int s = 0; s < C::SB; ++s) {
+      mbar_init(b_full(s), 1);
+      mbar_init(b_empty(s), 1);
+    }
+    for (int s = 0; s < C::SA; ++s) {
+      mbar_init(a_full(s), 4);
+      mbar_init(a_empty(s), 1);
+    }
+    for (int s = 0; s < C::SP; ++s) {
+      mbar_init(p_full(s), 1);
+      mbar_init(p_empty(s), 4);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tmem_full(a), 1);
@@ -154,17 +168,17 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     *s_abort = 0;
     fence_barrier_init();
   }
-  if (C::DEQ) {
-    for (int i = threadIdx.x; i < 256; i += C::THREADS) s_t8[i] = args.t8[i];
-  }
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&args.tm_b);
     if (!C::DEQ) tma_prefetch_desc(&args.tm_a);
-    if (C::DEQ) tma_prefetch_desc(&args.tm_pk);
     if (C::L2 != L2_NONE) {
       tma_prefetch_desc(&args.tm_a2);
       tma_prefetch_desc(&args.tm_b2);
     }
+  }
+  if (C::DEQ && warp == 6 && lane == 0) {
+    tma_prefetch_desc(&args.tm_pk);
+    tma_prefetch_desc(&args.tm_cp);
   }
   if (warp == 5) {
     tmem_alloc(smem_u32(s_tmem), C::TMEM_COLS);
@@ -180,61 +194,59 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
   const int num_tiles = row_tiles * col_tiles * args.splits;
 
   if (warp == 4) {
-    // ------------------------------------------------------ TMA issue --
+    // ---------------------------------------- TMA: B ring (and A when TMA) --
     if (lane == 0) {
       uint32_t job = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && !*s_abort; tile += gridDim.x) {
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         const TileCoord t = tile_coord(args, tile, row_tiles, col_tiles, C::BN);
         const int njobs = t.nmain + t.nlora;
-        bool ok = true;
         for (int jj = 0; jj < njobs; ++jj, ++job) {
-          const int s = job % C::STAGES;
-          const uint32_t par = (job / C::STAGES) & 1u;
-          if (!mbar_wait(empty_bar(s), par ^ 1u, s_abort)) { ok = false; break; }
-          const uint32_t a_dst = sbase + C::OFF_A + s * C::A_BYTES;
-          const uint32_t b_dst = sbase + C::OFF_B + s * C::B_BYTES;
+          const int sb = job % C::SB;
+          if (!mbar_wait(b_empty(sb), ((job / C::SB) & 1u) ^ 1u, s_abort)) { ok = false; break; }
+          const uint32_t b_dst = sbase + C::OFF_B + sb * C::B_BYTES;
           if (jj < t.nmain) {
             const int kb = t.kb_begin + jj;
-            mbar_arrive_expect_tx(tma_full(s), C::MAIN_TX);
+            mbar_arrive_expect_tx(b_full(sb), C::MAIN_TX);
             if (C::BSRC == B_TMA_K) {
-              tma_load_2d(b_dst, &args.tm_b, tma_full(s), kb * 64, t.col0);
+              tma_load_2d(b_dst, &args.tm_b, b_full(sb), kb * 64, t.col0);
             } else {
 #pragma unroll
               for (int c = 0; c < C::BN / 64; ++c)
-                tma_load_2d(b_dst + c * 8192, &args.tm_b, tma_full(s), t.col0 + c * 64, kb * 64);
+                tma_load_2d(b_dst + c * 8192, &args.tm_b, b_full(sb), t.col0 + c * 64, kb * 64);
             }
-            if (C::ASRC == A_TMA_K) {
-              tma_load_2d(a_dst, &args.tm_a, tma_full(s), kb * 64, t.row0);
-            } else if (C::ASRC == A_TMA_MN) {
-              tma_load_2d(a_dst, &args.tm_a, tma_full(s), t.row0, kb * 64);
-              tma_load_2d(a_dst + 8192, &args.tm_a, tma_full(s), t.row0 + 64, kb * 64);
-            } else {
-              const uint32_t p_dst = sbase + C::OFF_P + s * C::P_BYTES;
-              if (C::ASRC == A_DEQ_K)
-                tma_load_2d(p_dst, &args.tm_pk, tma_full(s), kb * 32, t.row0);
-              else
-                tma_load_2d(p_dst, &args.tm_pk, tma_full(s), t.row0 / 2, kb * 64);
+            if (!C::DEQ) {  // A shares the B ring slot index
+              const uint32_t a_dst = sbase + C::OFF_A + sb * C::A_BYTES;
+              if (C::ASRC == A_TMA_K) {
+                tma_load_2d(a_dst, &args.tm_a, b_full(sb), kb * 64, t.row0);
+              } else {
+                tma_load_2d(a_dst, &args.tm_a, b_full(sb), t.row0, kb * 64);
+                tma_load_2d(a_dst + 8192, &args.tm_a, b_full(sb), t.row0 + 64, kb * 64);
+              }
             }
           } else {
+            // low-rank step: A2 into the A ring slot of this job, B2 into B
             const int lk = jj - t.nmain;
-            mbar_arrive_expect_tx(tma_full(s), C::LORA_TX);
-            tma_load_2d(b_dst, &args.tm_b2, tma_full(s), lk * 64, t.col0);
+            const int sa = job % C::SA;
+            if (!mbar_wait(a_empty(sa), ((job / C::SA) & 1u) ^ 1u, s_abort)) { ok = false; break; }
+            const uint32_t a_dst = sbase + C::OFF_A + sa * C::A_BYTES;
+            mbar_arrive_expect_tx(b_full(sb), C::LORA_TX);
+            tma_load_2d(b_dst, &args.tm_b2, b_full(sb), lk * 64, t.col0);
             if (C::L2 == L2_A_MN) {
-              tma_load_2d(a_dst, &args.tm_a2, tma_full(s), t.row0, lk * 64);
-              tma_load_2d(a_dst + 8192, &args.tm_a2, tma_full(s), t.row0 + 64, lk * 64);
+              tma_load_2d(a_dst, &args.tm_a2, b_full(sb), t.row0, lk * 64);
+              tma_load_2d(a_dst + 8192, &args.tm_a2, b_full(sb), t.row0 + 64, lk * 64);
             } else {
-              tma_load_2d(a_dst, &args.tm_a2, tma_full(s), lk * 64, t.row0);
+              tma_load_2d(a_dst, &args.tm_a2, b_full(sb), lk * 64, t.row0);
             }
           }
         }
-        if (!ok) break;
       }
-      // wait for this thread's own copies still in flight (bounded)
-      const uint32_t inflight = job < (uint32_t)C::STAGES ? job : (uint32_t)C::STAGES;
+      // wait (bounded) for this thread's copies still in flight
+      const uint32_t inflight = job < (uint32_t)C::SB ? job : (uint32_t)C::SB;
       for (uint32_t i = 0; i < inflight; ++i) {
         const uint32_t jb = job - 1 - i;
         const unsigned long long t0 = globaltimer_ns();
-        while (!mbar_try_wait(tma_full(jb % C::STAGES), (jb / C::STAGES) & 1u)) {
+        while (!mbar_try_wait(b_full(jb % C::SB), (jb / C::SB) & 1u)) {
           if (globaltimer_ns() - t0 > kWaitTimeoutNs) break;
         }
       }
@@ -244,26 +256,26 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     // ------------------------------------------------------ MMA issue --
     if (lane == 0) {
       uint32_t job = 0, iter = 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++iter) {
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++iter) {
         const TileCoord t = tile_coord(args, tile, row_tiles, col_tiles, C::BN);
         const int njobs = t.nmain + t.nlora;
         const int acc = iter & 1;
         if (!mbar_wait(tmem_empty(acc), ((iter >> 1) & 1u) ^ 1u, s_abort)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::BN;
-        bool ok = true;
         for (int jj = 0; jj < njobs; ++jj, ++job) {
-          const int s = job % C::STAGES;
-          const uint32_t par = (job / C::STAGES) & 1u;
-          if (!mbar_wait(tma_full(s), par, s_abort)) { ok = false; break; }
-          if (C::DEQ && !mbar_wait(deq_full(s), par, s_abort)) { ok = false; break; }
+          const int sb = job % C::SB;
+          const int sa = C::DEQ ? (int)(job % C::SA) : sb;
+          if (!mbar_wait(b_full(sb), (job / C::SB) & 1u, s_abort)) { ok = false; break; }
+          if (C::DEQ && !mbar_wait(a_full(sa), (job / C::SA) & 1u, s_abort)) { ok = false; break; }
           tc_fence_after();
           const bool main_job = jj < t.nmain;
           const bool a_mn = main_job ? C::A_MN : (C::L2 == L2_A_MN);
           const bool b_mn = main_job ? C::B_MN : false;
           const uint32_t idesc = make_idesc_bf16(128, C::BN, a_mn ? 1 : 0, b_mn ? 1 : 0);
-          const uint32_t a_addr = sbase + C::OFF_A + s * C::A_BYTES;
-          const uint32_t b_addr = sbase + C::OFF_B + s * C::B_BYTES;
+          const uint32_t a_addr = sbase + C::OFF_A + sa * C::A_BYTES;
+          const uint32_t b_addr = sbase + C::OFF_B + sb * C::B_BYTES;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = a_mn ? smem_desc_sw128(a_addr + kk * 2048, 8192, 1024)
@@ -272,7 +284,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
                                      : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
             tc_mma_ss(d_tmem, ad, bd, idesc, (jj > 0 || kk > 0) ? 1u : 0u);
           }
-          tc_commit(empty_bar(s));
+          tc_commit(b_empty(sb));
+          if (C::DEQ) tc_commit(a_empty(sa));
         }
         if (!ok) break;
         tc_commit(tmem_full(acc));
@@ -326,76 +339,93 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
       __syncwarp();
       if (lane == 0) mbar_arrive(tmem_empty(acc));
     }
-  } else if (C::DEQ) {
+  } else if constexpr (C::DEQ) {
+   if (warp == 6) {
+    // ------------------------------------------------ P ring: TMA issue --
+    // Runs up to SP main K blocks ahead of the producers, gated only by them:
+    // the packed codes of the 128 x 64 weight tile and its 128 decoded block
+    // constants (c' is block-major, so they are one contiguous 512-byte row
+    // for the forward and two 256-byte rows for the backward).
+    if (lane == 0) {
+      uint32_t mj = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const TileCoord t = tile_coord(args, tile, row_tiles, col_tiles, C::BN);
+        for (int jj = 0; jj < t.nmain; ++jj, ++mj) {
+          const int sp = mj % C::SP;
+          if (!mbar_wait(p_empty(sp), ((mj / C::SP) & 1u) ^ 1u, s_abort)) { ok = false; break; }
+          const int kb = t.kb_begin + jj;
+          const uint32_t p_dst = sbase + C::OFF_P + sp * C::P_BYTES;
+          mbar_arrive_expect_tx(p_full(sp), C::P_BYTES);
+          if (C::ASRC == A_DEQ_K) {
+            tma_load_2d(p_dst, &args.tm_pk, p_full(sp), kb * 32, t.row0);
+            tma_load_2d(p_dst + C::P_CP, &args.tm_cp, p_full(sp), t.row0, kb);
+          } else {
+            tma_load_2d(p_dst, &args.tm_pk, p_full(sp), t.row0 / 2, kb * 64);
+            tma_load_2d(p_dst + C::P_CP, &args.tm_cp, p_full(sp), kb * 64, t.row0 / 64);
+          }
+        }
+      }
+      // wait (bounded) for this thread's own copies still in flight
+      const uint32_t inflight = mj < (uint32_t)C::SP ? mj : (uint32_t)C::SP;
+      for (uint32_t i = 0; i < inflight; ++i) {
+        const uint32_t jb = mj - 1 - i;
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(p_full(jb % C::SP), (jb / C::SP) & 1u)) {
+          if (globaltimer_ns() - t0 > kWaitTimeoutNs) break;
+        }
+      }
+    }
+    __syncwarp();
+   } else {
     // ------------------------------------------------ dequant producers --
-    const int pw = warp - 6;
+    const int pw = warp - 7;
     const int group = pw >> 2;
-    const int p = (pw & 3) * 32 + lane;  // 0..127
+    const int p = (pw & 3) * 32 + lane;  // 0..127: the tile row this thread decodes
     float L[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) L[i] = args.nf4[i];
-    uint32_t job = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    const uint32_t p_off = (C::ASRC == A_DEQ_K) ? p * 32 : (p & 63) * 64 + (p >> 6) * 32;
+    const uint32_t a_off = (C::ASRC == A_DEQ_K) ? p * 128 : (p >> 6) * 8192 + (p & 63) * 128;
+    const uint32_t swz = p & 7;
+    uint32_t job = 0, mj = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const TileCoord t = tile_coord(args, tile, row_tiles, col_tiles, C::BN);
       const int njobs = t.nmain + t.nlora;
-      bool ok = true;
       for (int jj = 0; jj < njobs; ++jj, ++job) {
+        const bool main_job = jj < t.nmain;
+        const uint32_t my_mj = mj;
+        if (main_job) ++mj;
         if ((int)(job % C::NGROUPS) != group) continue;
-        const int s = job % C::STAGES;
-        const uint32_t par = (job / C::STAGES) & 1u;
-        if (jj < t.nmain) {
-          const int kb = t.kb_begin + jj;
-          int64_t n, kblk;
-          bool valid;
-          uint32_t p_off, a_off;
-          if (C::ASRC == A_DEQ_K) {
-            n = t.row0 + p;
-            kblk = kb;
-            valid = n < args.w_rows;
-            p_off = p * 32;
-            a_off = p * 128;
-          } else {
-            n = static_cast<int64_t>(kb) * 64 + (p & 63);
-            kblk = t.row0 / 64 + (p >> 6);
-            valid = kblk < args.w_kblocks;
-            p_off = (p & 63) * 64 + (p >> 6) * 32;
-            a_off = (p >> 6) * 8192 + (p & 63) * 128;
-          }
-          float cp = 0.0f;
-          if (valid) {
-            const int64_t b = n * args.w_kblocks + kblk;
-            cp = __fmul_rn(s_t8[__ldg(args.q + b)], __ldg(args.scale2 + (b >> 8)));
-          }
-          if (!warp_wait(empty_bar(s), par ^ 1u, s_abort)) { ok = false; break; }
-          if (!warp_wait(tma_full(s), par, s_abort)) { ok = false; break; }
-          uint8_t *a_slot = smem + C::OFF_A + s * C::A_BYTES;
-          const uint32_t swz = p & 7;
-          if (valid) {
-            const uint8_t *pk = smem + C::OFF_P + s * C::P_BYTES + p_off;
-            const uint4 w0 = *reinterpret_cast<const uint4 *>(pk);
-            const uint4 w1 = *reinterpret_cast<const uint4 *>(pk + 16);
-            const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-            const Nf4Planes P = make_planes(L, cp);
+        const int sa = job % C::SA;
+        if (!warp_wait(a_empty(sa), ((job / C::SA) & 1u) ^ 1u, s_abort)) { ok = false; break; }
+        if (main_job) {
+          const int sp = my_mj % C::SP;
+          if (!warp_wait(p_full(sp), (my_mj / C::SP) & 1u, s_abort)) { ok = false; break; }
+          const uint8_t *pslot = smem + C::OFF_P + sp * C::P_BYTES;
+          const float cp = reinterpret_cast<const float *>(pslot + C::PK_BYTES)[p];
+          const uint4 w0 = *reinterpret_cast<const uint4 *>(pslot + p_off);
+          const uint4 w1 = *reinterpret_cast<const uint4 *>(pslot + p_off + 16);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_empty(sp));  // packed tile and c' consumed
+          uint8_t *a_slot = smem + C::OFF_A + sa * C::A_BYTES;
+          // out-of-range rows decode with c' = 0 -> zeros
+          const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+          const Nf4Planes P = make_planes(L, cp);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              uint32_t o[4];
-              nf4_lookup8(P, words[c], o);
-              *reinterpret_cast<uint4 *>(a_slot + a_off + ((c ^ swz) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              *reinterpret_cast<uint4 *>(a_slot + a_off + (c << 4)) = make_uint4(0u, 0u, 0u, 0u);
+          for (int c = 0; c < 8; ++c) {
+            uint32_t o[4];
+            nf4_lookup8(P, words[c], o);
+            *reinterpret_cast<uint4 *>(a_slot + a_off + ((c ^ swz) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
           }
           fence_proxy_async_smem();
-        } else {
-          if (!warp_wait(empty_bar(s), par ^ 1u, s_abort)) { ok = false; break; }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(deq_full(s));
+        if (lane == 0) mbar_arrive(a_full(sa));
       }
-      if (!ok) break;
     }
+   }
   }
 
   tc_fence_before();

@@ -119,15 +119,20 @@ EncodeTiledFn encode_fn() {
 
 // 2-D row-major tensor [outer, inner] with row pitch `row_bytes`; box
 // {box_inner, box_outer}; out-of-range elements read as zero.
-bool make_map(CUtensorMap *map, const void *base, bool bf16, uint64_t inner, uint64_t outer,
+enum MapType { MAP_BF16, MAP_U8, MAP_F32 };
+
+bool make_map(CUtensorMap *map, const void *base, MapType type, uint64_t inner, uint64_t outer,
               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
+  const CUtensorMapDataType dt = type == MAP_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                 : type == MAP_U8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+  const CUresult r = fn(map, dt, 2,
                         const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -136,11 +141,11 @@ bool make_map(CUtensorMap *map, const void *base, bool bf16, uint64_t inner, uin
 
 // bf16 operand [outer rows, inner] read as K-major tiles (box {64, box_rows})
 bool map_kmajor(CUtensorMap *m, const void *p, int64_t inner, int64_t outer, uint32_t box_rows) {
-  return make_map(m, p, true, inner, outer, inner * 2, 64, box_rows, true);
+  return make_map(m, p, MAP_BF16, inner, outer, inner * 2, 64, box_rows, true);
 }
 // bf16 operand [outer rows, inner] read as MN-major 64x64 chunks
 bool map_mnmajor(CUtensorMap *m, const void *p, int64_t inner, int64_t outer) {
-  return make_map(m, p, true, inner, outer, inner * 2, 64, 64, true);
+  return make_map(m, p, MAP_BF16, inner, outer, inner * 2, 64, 64, true);
 }
 
 // ------------------------------------------------------- GEMM launcher --
@@ -175,6 +180,17 @@ qlora_status launch_reduce(const float *part, int splits, int rows, int cols, in
   return launched();
 }
 
+// Block constants c' = t8[q] * S, block-major [K/64][N] fp32 (GEMM operand
+// staging; one small pass per linear call).
+qlora_status launch_decode_constants(const uint8_t *q, const float *scale2, const float *t8, int64_t N,
+                                     int64_t KB, float *cprime, int sms, cudaStream_t stream) {
+  const int grid = grid_for(N * cdiv(KB, 16), 256, sms, 8);
+  decode_constants_kernel<<<grid, 256, 0, stream>>>(q, scale2, N, KB, cprime, make_tables(nullptr, t8));
+  return launched();
+}
+
+size_t cprime_bytes(int64_t N, int64_t K) { return align256(static_cast<size_t>(N) * (K / 64) * 4); }
+
 // ------------------------------------------------------- skinny GEMMs --
 // out[rows, r] (or its transpose) = scale * sum_k Aop[row, k] Bop[j, k],
 // with the K range split across CTAs into fp32 partials, then reduced.
@@ -203,7 +219,8 @@ SkinnyPlan plan_skinny(int64_t rows, int64_t kdim, int r, int sms) {
 
 template <int BN, int AS, int BS>
 qlora_status run_skinny_bn(const GemmArgs &a, int sms, cudaStream_t st) {
-  using C = GemmCfg<BN, AS, BS, L2_NONE, EPI_F32, (BN == 256 ? 4 : 6), 0>;
+  constexpr int S = BN == 256 ? 4 : 6;
+  using C = GemmCfg<BN, AS, BS, L2_NONE, EPI_F32, S, S, 0, 0>;
   return launch_gemm<C>(a, sms, st);
 }
 
@@ -284,8 +301,10 @@ FusedPlan plan_fused(int64_t M, int64_t rows, int64_t kblocks, int sms) {
 
 template <int BN, int AS, int L2>
 qlora_status run_fused_bn(const GemmArgs &a, int sms, cudaStream_t st) {
-  if (a.splits > 1) return launch_gemm<GemmCfg<BN, AS, B_TMA_K, L2, EPI_F32, (BN > 64 ? 4 : 8), 8>>(a, sms, st);
-  return launch_gemm<GemmCfg<BN, AS, B_TMA_K, L2, EPI_BF16_T, (BN > 64 ? 4 : 8), 8>>(a, sms, st);
+  // rings: activation tiles (SB), dequantized weight tiles (SA), packed codes + constants (SP)
+  constexpr int SB = BN > 64 ? 4 : 8, SA = BN > 64 ? 3 : 4, SP = 8;
+  if (a.splits > 1) return launch_gemm<GemmCfg<BN, AS, B_TMA_K, L2, EPI_F32, SB, SA, SP, 8>>(a, sms, st);
+  return launch_gemm<GemmCfg<BN, AS, B_TMA_K, L2, EPI_BF16_T, SB, SA, SP, 8>>(a, sms, st);
 }
 
 // Layer sizes shared by forward and backward.
@@ -298,7 +317,7 @@ size_t fwd_ws_bytes(const Shape &s, int sms) {
   const size_t xas = align256(static_cast<size_t>(s.M) * s.r * 2);
   const SkinnyPlan xa = plan_skinny(s.M, s.K, s.r, sms);
   const FusedPlan fp = plan_fused(s.M, s.N, s.K / 64, sms);
-  return xas + (xa.part_bytes > fp.part_bytes ? xa.part_bytes : fp.part_bytes);
+  return xas + cprime_bytes(s.N, s.K) + (xa.part_bytes > fp.part_bytes ? xa.part_bytes : fp.part_bytes);
 }
 
 size_t bwd_ws_bytes(const Shape &s, int sms) {
@@ -308,7 +327,7 @@ size_t bwd_ws_bytes(const Shape &s, int sms) {
   part = std::max(part, plan_skinny(s.N, s.M, s.r, sms).part_bytes);         // dB
   part = std::max(part, plan_skinny(s.M, s.K, s.r, sms).part_bytes);         // XA recompute
   part = std::max(part, plan_fused(s.M, s.K, s.N / 64, sms).part_bytes);     // dX split-K
-  return 2 * mr + part;
+  return 2 * mr + cprime_bytes(s.N, s.K) + part;
 }
 
 void trace_begin(cudaStream_t s) {
@@ -460,7 +479,8 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   qlora_bf16 *xas = reinterpret_cast<qlora_bf16 *>(ws);
-  float *part = reinterpret_cast<float *>(ws + align256(static_cast<size_t>(M) * r * 2));
+  float *cprime = reinterpret_cast<float *>(ws + align256(static_cast<size_t>(M) * r * 2));
+  float *part = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(cprime) + cprime_bytes(N, K));
 
   // 1) XA = X A (split-K partials) -> XA_out = bf16(XA), xas = bf16(s XA)
   if (XA_out != nullptr)
@@ -469,16 +489,19 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
     st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, scl, xas, r, 0.0f, nullptr, 0, false, part, d.sms, cs);
   if (st != QLORA_OK) return st;
 
-  // 2) Y^T[n, m] = W'[n, :] . X[m, :] + B^T[n, :] . xas[m, :]
+  // 2) block constants c' for the GEMM producers
+  st = launch_decode_constants(q, scale2, t8, N, K / 64, cprime, d.sms, cs);
+  if (st != QLORA_OK) return st;
+
+  // 3) Y^T[n, m] = W'[n, :] . X[m, :] + B^T[n, :] . xas[m, :]
   const FusedPlan fp = plan_fused(M, N, K / 64, d.sms);
   GemmArgs a;
   std::memset(&a, 0, sizeof a);
   if (!map_kmajor(&a.tm_b, X, K, M, fp.bn) ||
-      !make_map(&a.tm_pk, packed, false, K / 2, N, K / 2, 32, 128, false) ||
+      !make_map(&a.tm_pk, packed, MAP_U8, K / 2, N, K / 2, 32, 128, false) ||
+      !make_map(&a.tm_cp, cprime, MAP_F32, N, K / 64, N * 4, 128, 1, false) ||
       !map_mnmajor(&a.tm_a2, B, N, r) || !map_kmajor(&a.tm_b2, xas, r, M, fp.bn))
     return QLORA_ERR_CUDA;
-  a.q = q;
-  a.scale2 = scale2;
   a.w_kblocks = K / 64;
   a.w_rows = static_cast<int>(N);
   a.rows = static_cast<int>(N);
@@ -488,7 +511,6 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   a.lora_kblocks = static_cast<int>(cdiv(r, 64));
   a.out_scale = 1.0f;
   std::memcpy(a.nf4, nf4, sizeof a.nf4);
-  std::memcpy(a.t8, t8, sizeof a.t8);
   if (fp.splits == 1) {
     a.out = Y;
     a.out_ld = N;
@@ -526,22 +548,26 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   const size_t mr = align256(static_cast<size_t>(M) * r * 2);
   qlora_bf16 *gs = reinterpret_cast<qlora_bf16 *>(ws);
   qlora_bf16 *xa_ws = reinterpret_cast<qlora_bf16 *>(ws + mr);
-  float *part = reinterpret_cast<float *>(ws + 2 * mr);
+  float *cprime = reinterpret_cast<float *>(ws + 2 * mr);
+  float *part = reinterpret_cast<float *>(ws + 2 * mr + cprime_bytes(N, K));
 
   // 1) Gs = bf16(s * dY B^T)
   st = skinny(SK_G, dY, N, M, B, N, r, M, N, r, scl, gs, r, 0.0f, nullptr, 0, false, part, d.sms, cs);
   if (st != QLORA_OK) return st;
 
-  // 2) dX^T[k, m] = W'^T[k, :] . dY[m, :] + A[k, :] . Gs[m, :]
+  // 2) block constants c' for the GEMM producers
+  st = launch_decode_constants(q, scale2, t8, N, K / 64, cprime, d.sms, cs);
+  if (st != QLORA_OK) return st;
+
+  // 3) dX^T[k, m] = W'^T[k, :] . dY[m, :] + A[k, :] . Gs[m, :]
   const FusedPlan fp = plan_fused(M, K, N / 64, d.sms);
   GemmArgs a;
   std::memset(&a, 0, sizeof a);
   if (!map_kmajor(&a.tm_b, dY, N, M, fp.bn) ||
-      !make_map(&a.tm_pk, packed, false, K / 2, N, K / 2, 64, 64, false) || !map_kmajor(&a.tm_a2, A, r, K, 128) ||
-      !map_kmajor(&a.tm_b2, gs, r, M, fp.bn))
+      !make_map(&a.tm_pk, packed, MAP_U8, K / 2, N, K / 2, 64, 64, false) ||
+      !make_map(&a.tm_cp, cprime, MAP_F32, N, K / 64, N * 4, 64, 2, false) ||
+      !map_kmajor(&a.tm_a2, A, r, K, 128) || !map_kmajor(&a.tm_b2, gs, r, M, fp.bn))
     return QLORA_ERR_CUDA;
-  a.q = q;
-  a.scale2 = scale2;
   a.w_kblocks = K / 64;
   a.w_rows = static_cast<int>(N);
   a.rows = static_cast<int>(K);
@@ -551,7 +577,6 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   a.lora_kblocks = static_cast<int>(cdiv(r, 64));
   a.out_scale = 1.0f;
   std::memcpy(a.nf4, nf4, sizeof a.nf4);
-  std::memcpy(a.t8, t8, sizeof a.t8);
   if (fp.splits == 1) {
     a.out = dX;
     a.out_ld = K;
@@ -569,11 +594,11 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
     if (st != QLORA_OK) return st;
   }
 
-  // 3) dA = X^T Gs   ([K, r])
+  // 4) dA = X^T Gs   ([K, r])
   st = skinny(SK_DA, X, K, M, gs, r, M, K, M, r, 1.0f, dA, r, 0.0f, nullptr, 0, false, part, d.sms, cs);
   if (st != QLORA_OK) return st;
 
-  // 4) XA (saved or recomputed), then dB = s XA^T dY   ([r, N], from dB^T[n, j])
+  // 5) XA (saved or recomputed), then dB = s XA^T dY   ([r, N], from dB^T[n, j])
   const qlora_bf16 *xa = XA;
   if (xa == nullptr) {
     st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, 1.0f, xa_ws, r, 0.0f, nullptr, 0, false, part, d.sms, cs);
