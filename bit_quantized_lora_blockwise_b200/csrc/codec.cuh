@@ -239,15 +239,20 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint2 *__restrict__ 
 // Decoded block constants for the GEMMs, block-major: cprime[kb * N + n] =
 // t8[q_b] * scale2[b / 256] (fp32 product), b = n * KB + kb. One thread per
 // (row n, 16 consecutive blocks); consecutive threads take consecutive rows
-// so every store instruction writes a contiguous run of one kb row.
+// so every store instruction writes a contiguous run of one kb row. The
+// launch also zeroes `ncounters` split-K tile counters.
 __global__ void __launch_bounds__(256) decode_constants_kernel(const uint8_t *__restrict__ q,
                                                                const float *__restrict__ scale2,
                                                                int64_t N, int64_t KB,
                                                                float *__restrict__ cprime,
-                                                               const CodecTables tabs) {
+                                                               unsigned int *__restrict__ counters,
+                                                               int64_t ncounters, const CodecTables tabs) {
   __shared__ float s_t8[256];
   s_t8[threadIdx.x] = tabs.t8[threadIdx.x];
   __syncthreads();
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < ncounters;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    counters[i] = 0u;
   const int64_t chunks = (KB + 15) / 16;
   const int64_t total = N * chunks;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;

@@ -36,7 +36,6 @@ namespace qlora {
 enum : int { A_TMA_K = 0, A_TMA_MN = 1, A_DEQ_K = 2, A_DEQ_MN = 3 };
 enum : int { B_TMA_K = 0, B_TMA_MN = 1 };
 enum : int { L2_NONE = 0, L2_A_MN = 1, L2_A_K = 2 };  // A2 major-ness (B2 is K-major)
-enum : int { EPI_BF16_T = 0, EPI_F32 = 1 };
 
 struct GemmArgs {
   CUtensorMap tm_a;   // A operand (TMA variants)
@@ -45,23 +44,32 @@ struct GemmArgs {
   CUtensorMap tm_a2;  // low-rank A2
   CUtensorMap tm_b2;  // low-rank B2
   CUtensorMap tm_cp;  // decoded block constants c' [K/64][N] fp32 (dequant variants)
-  void *out;              // EPI_BF16_T: bf16 out[col * out_ld + row]; EPI_F32: fp32 partials
+  // Output: bf16 out[row * out_ld + col] (transpose = 0) or
+  // out[col * out_ld + row] (transpose = 1), times out_scale; optionally a
+  // second copy out2 (same layout, out2_ld) times out2_scale.
+  void *out;
+  void *out2;
   int64_t out_ld;
+  int64_t out2_ld;
+  float *part;             // fp32 split-K partials [splits][rows_pad][cols_pad] (splits > 1)
+  unsigned int *counters;  // one per output tile; zero on entry, left zero (splits > 1)
   int64_t w_kblocks;      // 64-blocks per weight row (K / 64)
   int rows;               // extent of the 128-row MMA dimension
   int cols;               // extent of the BN-column MMA dimension
   int kblocks;            // 64-deep K blocks of the main product
-  int splits;             // split-K count (fp32 partials when > 1 or EPI_F32)
+  int splits;             // split-K count (> 1: partials reduced by the last CTA of a tile)
   int lora_kblocks;       // 64-deep K blocks of the low-rank product (last split only)
   int w_rows;             // A_DEQ_K: rows of W (N)
   float out_scale;
+  float out2_scale;
+  int transpose;
   float nf4[16];
 };
 
-template <int BN_, int ASRC_, int BSRC_, int L2_, int EPI_, int SB_, int SA_, int SP_, int NPW_>
+template <int BN_, int ASRC_, int BSRC_, int L2_, int SB_, int SA_, int SP_, int NPW_>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 64, BN = BN_;
-  static constexpr int ASRC = ASRC_, BSRC = BSRC_, L2 = L2_, EPI = EPI_;
+  static constexpr int ASRC = ASRC_, BSRC = BSRC_, L2 = L2_;
   static constexpr int SB = SB_, SA = SA_, SP = SP_, NPW = NPW_;
   static constexpr bool DEQ = ASRC_ >= A_DEQ_K;
   static constexpr bool A_MN = (ASRC_ == A_TMA_MN) || (ASRC_ == A_DEQ_MN);
@@ -86,7 +94,7 @@ struct GemmCfg {
   // b_full[SB] b_empty[SB] a_full[SA] a_empty[SA] p_full[SP] p_empty[SP]
   // tmem_full[2] tmem_empty[2] drain
   static constexpr int NBARS = 2 * SB + 2 * SA + 2 * SP + 5;
-  static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem base, abort flag
+  static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem base, abort flag, last-CTA flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr int WARPS = DEQ ? 7 + NPW_ : 6;
   static constexpr int THREADS = WARPS * 32;
@@ -98,7 +106,7 @@ struct GemmCfg {
 };
 
 struct TileCoord {
-  int row0, col0, split, kb_begin, nmain, nlora;
+  int row0, col0, split, rc, kb_begin, nmain, nlora;  // rc: (row tile, col tile) index
 };
 
 __device__ __forceinline__ TileCoord tile_coord(const GemmArgs &a, int tile, int row_tiles,
@@ -107,6 +115,7 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs &a, int tile, int
   const int per_split = row_tiles * col_tiles;
   t.split = tile / per_split;
   const int rem = tile - t.split * per_split;
+  t.rc = rem;
   const int rt = rem / col_tiles;
   const int ct = rem - rt * col_tiles;
   t.row0 = rt * 128;
@@ -300,44 +309,108 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     __syncwarp();
   } else if (warp < 4) {
     // ------------------------------------------------------- epilogue --
+    // splits == 1: TMEM -> bf16 output directly. splits > 1: TMEM -> fp32
+    // partial in global memory; the last of the tile's splits to arrive
+    // (atomic counter) sums the partials in split order (deterministic) and
+    // writes the bf16 output.
+    volatile int *s_last = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
+    const int64_t rows_pad = static_cast<int64_t>(row_tiles) * 128;
+    const int64_t cols_pad = static_cast<int64_t>(col_tiles) * C::BN;
     uint32_t iter = 0;
     const int qrow = warp * 32 + lane;  // TMEM lane of this thread
+    auto store_out = [&](int row, int col_base, const float (&v)[32]) {
+      if (row >= args.rows) return;
+      const int ncol = args.cols - col_base < 32 ? args.cols - col_base : 32;
+      for (int o = 0; o < 2; ++o) {
+        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(o ? args.out2 : args.out);
+        if (dst == nullptr) continue;
+        const float sc = o ? args.out2_scale : args.out_scale;
+        const int64_t ld = o ? args.out2_ld : args.out_ld;
+        if (args.transpose) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < ncol) dst[static_cast<int64_t>(col_base + j) * ld + row] = __float2bfloat16_rn(v[j] * sc);
+        } else if (ncol == 32) {
+          uint32_t w[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(v[2 * j] * sc, v[2 * j + 1] * sc);
+          uint4 *d4 = reinterpret_cast<uint4 *>(dst + static_cast<int64_t>(row) * ld + col_base);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) d4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < ncol) dst[static_cast<int64_t>(row) * ld + col_base + j] = __float2bfloat16_rn(v[j] * sc);
+        }
+      }
+    };
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++iter) {
       const TileCoord t = tile_coord(args, tile, row_tiles, col_tiles, C::BN);
       const int acc = iter & 1;
       if (!warp_wait(tmem_full(acc), (iter >> 1) & 1u, s_abort)) break;
       tc_fence_after();
       const int row = t.row0 + qrow;
+      const uint32_t tcol = tmem_base + ((uint32_t)(warp * 32) << 16) + acc * C::BN;
+      if (args.splits == 1) {
+#pragma unroll 1
+        for (int ch = 0; ch < C::BN / 32; ++ch) {
+          uint32_t u[32];
+          tmem_ld_32x32b_x32(tcol + ch * 32, u);
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(u[j]);
+          store_out(row, t.col0 + ch * 32, v);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tmem_empty(acc));
+        continue;
+      }
+      float *prow = args.part + (static_cast<int64_t>(t.split) * rows_pad + row) * cols_pad + t.col0;
 #pragma unroll 1
       for (int ch = 0; ch < C::BN / 32; ++ch) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(warp * 32) << 16) + acc * C::BN + ch * 32, v);
-        const int col_base = t.col0 + ch * 32;
-        if (C::EPI == EPI_BF16_T) {
-          __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(args.out);
-          if (row < args.rows) {
+        uint32_t u[32];
+        tmem_ld_32x32b_x32(tcol + ch * 32, u);
+        float4 *o = reinterpret_cast<float4 *>(prow + ch * 32);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int col = col_base + j;
-              if (col < args.cols)
-                o[static_cast<int64_t>(col) * args.out_ld + row] =
-                    __float2bfloat16_rn(__uint_as_float(v[j]) * args.out_scale);
-            }
-          }
-        } else {
-          const int64_t rows_pad = static_cast<int64_t>(row_tiles) * 128;
-          const int64_t cols_pad = static_cast<int64_t>(col_tiles) * C::BN;
-          float4 *o = reinterpret_cast<float4 *>(reinterpret_cast<float *>(args.out) +
-                                                 (t.split * rows_pad + row) * cols_pad + col_base);
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            o[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                               __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-        }
+        for (int j = 0; j < 8; ++j)
+          o[j] = make_float4(__uint_as_float(u[4 * j]), __uint_as_float(u[4 * j + 1]),
+                             __uint_as_float(u[4 * j + 2]), __uint_as_float(u[4 * j + 3]));
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tmem_empty(acc));
+      if (lane == 0) mbar_arrive(tmem_empty(acc));  // accumulator free: partial is in memory
+      __threadfence();
+      named_bar_sync(1, 128);
+      if (warp == 0 && lane == 0) {
+        const unsigned int prev = atomicAdd(args.counters + t.rc, 1u);
+        const int last = prev == static_cast<unsigned int>(args.splits - 1);
+        if (last) args.counters[t.rc] = 0u;  // every split has arrived: reset for the next use
+        *s_last = last;
+      }
+      named_bar_sync(1, 128);
+      if (*s_last) {
+        __threadfence();
+#pragma unroll 1
+        for (int ch = 0; ch < C::BN / 32; ++ch) {
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+          for (int sp = 0; sp < args.splits; ++sp) {
+            const float4 *src = reinterpret_cast<const float4 *>(
+                args.part + (static_cast<int64_t>(sp) * rows_pad + row) * cols_pad + t.col0 + ch * 32);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float4 x = __ldcg(src + j);
+              v[4 * j] += x.x;
+              v[4 * j + 1] += x.y;
+              v[4 * j + 2] += x.z;
+              v[4 * j + 3] += x.w;
+            }
+          }
+          store_out(row, t.col0 + ch * 32, v);
+        }
+      }
     }
   } else if constexpr (C::DEQ) {
    if (warp == 6) {
@@ -433,39 +506,6 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
   if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
-  }
-}
-
-// ------------------------------------------------------------------------
-// Deterministic split-K reduction of fp32 partials [splits][rows_pad][cols_pad]:
-//   v = sum over splits in order; out[...] = bf16(v * scale) (and out2 with
-//   scale2 when given), row-major [rows, cols] with leading dim ld, or
-//   transposed ([cols, rows]) when `transpose`.
-__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restrict__ part, int splits,
-                                                            int rows, int cols, int64_t rows_pad,
-                                                            int64_t cols_pad, float scale,
-                                                            __nv_bfloat16 *__restrict__ out, int64_t ld,
-                                                            float scale2, __nv_bfloat16 *__restrict__ out2,
-                                                            int64_t ld2, int transpose) {
-  const int64_t total = static_cast<int64_t>(rows) * cols;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
-    int64_t r, c;
-    if (transpose) {  // consecutive threads -> consecutive rows (contiguous output)
-      c = i / rows;
-      r = i - c * rows;
-    } else {
-      r = i / cols;
-      c = i - r * cols;
-    }
-    float v = 0.0f;
-    for (int s = 0; s < splits; ++s) v += part[(s * rows_pad + r) * cols_pad + c];
-    const int64_t o = transpose ? c * ld + r : r * ld + c;
-    out[o] = __float2bfloat16_rn(v * scale);
-    if (out2 != nullptr) {
-      const int64_t o2 = transpose ? c * ld2 + r : r * ld2 + c;
-      out2[o2] = __float2bfloat16_rn(v * scale2);
-    }
   }
 }
 

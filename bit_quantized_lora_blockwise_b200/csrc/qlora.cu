@@ -168,32 +168,36 @@ qlora_status launch_gemm(const GemmArgs &args, int sms, cudaStream_t stream) {
   return launched();
 }
 
-qlora_status launch_reduce(const float *part, int splits, int rows, int cols, int64_t rows_pad,
-                           int64_t cols_pad, float scale, void *out, int64_t ld, float scale2, void *out2,
-                           int64_t ld2, bool transpose, int sms, cudaStream_t stream) {
-  const int64_t total = static_cast<int64_t>(rows) * cols;
-  const int grid = grid_for(total, 256, sms, 8);
-  splitk_reduce_kernel<<<grid, 256, 0, stream>>>(part, splits, rows, cols, rows_pad, cols_pad, scale,
-                                                 reinterpret_cast<__nv_bfloat16 *>(out), ld, scale2,
-                                                 reinterpret_cast<__nv_bfloat16 *>(out2), ld2,
-                                                 transpose ? 1 : 0);
-  return launched();
-}
-
 // Block constants c' = t8[q] * S, block-major [K/64][N] fp32 (GEMM operand
-// staging; one small pass per linear call).
+// staging; one small pass per linear call). The same launch zeroes the
+// split-K tile counters the call's GEMMs use (each GEMM leaves them zero).
 qlora_status launch_decode_constants(const uint8_t *q, const float *scale2, const float *t8, int64_t N,
-                                     int64_t KB, float *cprime, int sms, cudaStream_t stream) {
+                                     int64_t KB, float *cprime, unsigned int *counters, int64_t ncounters,
+                                     int sms, cudaStream_t stream) {
   const int grid = grid_for(N * cdiv(KB, 16), 256, sms, 8);
-  decode_constants_kernel<<<grid, 256, 0, stream>>>(q, scale2, N, KB, cprime, make_tables(nullptr, t8));
+  decode_constants_kernel<<<grid, 256, 0, stream>>>(q, scale2, N, KB, cprime, counters, ncounters,
+                                                    make_tables(nullptr, t8));
   return launched();
 }
 
 size_t cprime_bytes(int64_t N, int64_t K) { return align256(static_cast<size_t>(N) * (K / 64) * 4); }
 
+// Layer sizes shared by forward and backward.
+struct Shape {
+  int64_t M, N, K;
+  int r;
+};
+
+// One counter per output tile of any GEMM of the call (tiles are at least
+// 128 x 32).
+int64_t counters_needed(const Shape &s) {
+  const int64_t rows = std::max(std::max(cdiv(s.M, 128), cdiv(s.N, 128)), cdiv(s.K, 128));
+  return rows * std::max<int64_t>(1, cdiv(s.M, 32));
+}
+
 // ------------------------------------------------------- skinny GEMMs --
 // out[rows, r] (or its transpose) = scale * sum_k Aop[row, k] Bop[j, k],
-// with the K range split across CTAs into fp32 partials, then reduced.
+// the K range split across CTAs; the last CTA of a tile reduces.
 enum SkinnyKind { SK_XA, SK_G, SK_DA, SK_DB };
 
 int rank_tile(int r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
@@ -209,19 +213,18 @@ SkinnyPlan plan_skinny(int64_t rows, int64_t kdim, int r, int sms) {
   p.kblocks = static_cast<int>(cdiv(kdim, 64));
   p.bn = rank_tile(r);
   const int row_tiles = static_cast<int>(cdiv(rows, 128));
-  int splits = static_cast<int>(cdiv(sms, row_tiles));
+  int splits = sms / row_tiles;  // one wave
   if (splits > p.kblocks) splits = p.kblocks;
   if (splits < 1) splits = 1;
   p.splits = splits;
-  p.part_bytes = align256(static_cast<size_t>(splits) * row_tiles * 128 * p.bn * 4);
+  p.part_bytes = splits > 1 ? align256(static_cast<size_t>(splits) * row_tiles * 128 * p.bn * 4) : 0;
   return p;
 }
 
 template <int BN, int AS, int BS>
 qlora_status run_skinny_bn(const GemmArgs &a, int sms, cudaStream_t st) {
   constexpr int S = BN == 256 ? 4 : 6;
-  using C = GemmCfg<BN, AS, BS, L2_NONE, EPI_F32, S, S, 0, 0>;
-  return launch_gemm<C>(a, sms, st);
+  return launch_gemm<GemmCfg<BN, AS, BS, L2_NONE, S, S, 0, 0>>(a, sms, st);
 }
 
 template <int AS, int BS>
@@ -235,10 +238,19 @@ qlora_status run_skinny(const GemmArgs &a, int bn, int sms, cudaStream_t st) {
 //       SK_G    Aop = dY [M,N] (K-major),  Bop = B  [r,N] (K-major),  rows = M, kdim = N
 //       SK_DA   Aop = X^T (MN-major),      Bop = Gs [M,r] (MN-major), rows = K, kdim = M
 //       SK_DB   Aop = dY^T (MN-major),     Bop = XA [M,r] (MN-major), rows = N, kdim = M
+struct OutSpec {
+  void *out;
+  int64_t ld;
+  float scale;
+  void *out2;
+  int64_t ld2;
+  float scale2;
+  bool transpose;
+};
+
 qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a_outer, const void *bop,
-                    int64_t b_inner, int64_t b_outer, int64_t rows, int64_t kdim, int r, float scale,
-                    void *out, int64_t ld, float scale2, void *out2, int64_t ld2, bool transpose,
-                    float *part, int sms, cudaStream_t st) {
+                    int64_t b_inner, int64_t b_outer, int64_t rows, int64_t kdim, int r, const OutSpec &o,
+                    float *part, unsigned int *counters, int sms, cudaStream_t st) {
   const SkinnyPlan p = plan_skinny(rows, kdim, r, sms);
   GemmArgs a;
   std::memset(&a, 0, sizeof a);
@@ -257,23 +269,25 @@ qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a
       break;
   }
   if (!ok) return QLORA_ERR_CUDA;
-  a.out = part;
+  a.out = o.out;
+  a.out_ld = o.ld;
+  a.out_scale = o.scale;
+  a.out2 = o.out2;
+  a.out2_ld = o.ld2;
+  a.out2_scale = o.scale2;
+  a.transpose = o.transpose ? 1 : 0;
+  a.part = part;
+  a.counters = counters;
   a.rows = p.rows;
   a.cols = r;
   a.kblocks = p.kblocks;
   a.splits = p.splits;
   a.lora_kblocks = 0;
-  a.out_scale = 1.0f;
-  qlora_status s;
   switch (kind) {
-    case SK_XA: s = run_skinny<A_TMA_K, B_TMA_MN>(a, p.bn, sms, st); break;
-    case SK_G: s = run_skinny<A_TMA_K, B_TMA_K>(a, p.bn, sms, st); break;
-    default: s = run_skinny<A_TMA_MN, B_TMA_MN>(a, p.bn, sms, st); break;
+    case SK_XA: return run_skinny<A_TMA_K, B_TMA_MN>(a, p.bn, sms, st);
+    case SK_G: return run_skinny<A_TMA_K, B_TMA_K>(a, p.bn, sms, st);
+    default: return run_skinny<A_TMA_MN, B_TMA_MN>(a, p.bn, sms, st);
   }
-  if (s != QLORA_OK) return s;
-  const int64_t rows_pad = cdiv(rows, 128) * 128;
-  return launch_reduce(part, p.splits, static_cast<int>(rows), r, rows_pad, p.bn, scale, out, ld, scale2,
-                       out2, ld2, transpose, sms, st);
 }
 
 // -------------------------------------------------------- fused GEMMs --
@@ -303,32 +317,38 @@ template <int BN, int AS, int L2>
 qlora_status run_fused_bn(const GemmArgs &a, int sms, cudaStream_t st) {
   // rings: activation tiles (SB), dequantized weight tiles (SA), packed codes + constants (SP)
   constexpr int SB = BN > 64 ? 4 : 8, SA = BN > 64 ? 3 : 4, SP = 8;
-  if (a.splits > 1) return launch_gemm<GemmCfg<BN, AS, B_TMA_K, L2, EPI_F32, SB, SA, SP, 8>>(a, sms, st);
-  return launch_gemm<GemmCfg<BN, AS, B_TMA_K, L2, EPI_BF16_T, SB, SA, SP, 8>>(a, sms, st);
+  return launch_gemm<GemmCfg<BN, AS, B_TMA_K, L2, SB, SA, SP, 8>>(a, sms, st);
 }
 
-// Layer sizes shared by forward and backward.
-struct Shape {
-  int64_t M, N, K;
-  int r;
+// Workspace carve-up: [tile counters][bf16 M x r][bf16 M x r (backward)][c'][fp32 partials]
+struct WsLayout {
+  size_t counters, mr, cprime, part, total;
+  int64_t ncounters;
 };
 
-size_t fwd_ws_bytes(const Shape &s, int sms) {
-  const size_t xas = align256(static_cast<size_t>(s.M) * s.r * 2);
-  const SkinnyPlan xa = plan_skinny(s.M, s.K, s.r, sms);
-  const FusedPlan fp = plan_fused(s.M, s.N, s.K / 64, sms);
-  return xas + cprime_bytes(s.N, s.K) + (xa.part_bytes > fp.part_bytes ? xa.part_bytes : fp.part_bytes);
+WsLayout ws_layout(const Shape &s, int sms, bool backward) {
+  WsLayout w;
+  w.ncounters = counters_needed(s);
+  w.counters = align256(static_cast<size_t>(w.ncounters) * 4);
+  w.mr = align256(static_cast<size_t>(s.M) * s.r * 2);
+  w.cprime = cprime_bytes(s.N, s.K);
+  if (!backward) {
+    w.part = std::max(plan_skinny(s.M, s.K, s.r, sms).part_bytes, plan_fused(s.M, s.N, s.K / 64, sms).part_bytes);
+    w.total = w.counters + w.mr + w.cprime + w.part;
+  } else {
+    size_t part = plan_skinny(s.M, s.N, s.r, sms).part_bytes;               // G
+    part = std::max(part, plan_skinny(s.K, s.M, s.r, sms).part_bytes);       // dA
+    part = std::max(part, plan_skinny(s.N, s.M, s.r, sms).part_bytes);       // dB
+    part = std::max(part, plan_skinny(s.M, s.K, s.r, sms).part_bytes);       // XA recompute
+    part = std::max(part, plan_fused(s.M, s.K, s.N / 64, sms).part_bytes);   // dX split-K
+    w.part = part;
+    w.total = w.counters + 2 * w.mr + w.cprime + w.part;
+  }
+  return w;
 }
 
-size_t bwd_ws_bytes(const Shape &s, int sms) {
-  const size_t mr = align256(static_cast<size_t>(s.M) * s.r * 2);
-  size_t part = plan_skinny(s.M, s.N, s.r, sms).part_bytes;                 // G
-  part = std::max(part, plan_skinny(s.K, s.M, s.r, sms).part_bytes);         // dA
-  part = std::max(part, plan_skinny(s.N, s.M, s.r, sms).part_bytes);         // dB
-  part = std::max(part, plan_skinny(s.M, s.K, s.r, sms).part_bytes);         // XA recompute
-  part = std::max(part, plan_fused(s.M, s.K, s.N / 64, sms).part_bytes);     // dX split-K
-  return 2 * mr + cprime_bytes(s.N, s.K) + part;
-}
+size_t fwd_ws_bytes(const Shape &s, int sms) { return ws_layout(s, sms, false).total; }
+size_t bwd_ws_bytes(const Shape &s, int sms) { return ws_layout(s, sms, true).total; }
 
 void trace_begin(cudaStream_t s) {
   if (t_trace_start && t_trace_stop) cudaEventRecord(t_trace_start, s);
@@ -477,21 +497,23 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const float scl = alpha / static_cast<float>(r);
 
+  const WsLayout w = ws_layout(s, d.sms, false);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  qlora_bf16 *xas = reinterpret_cast<qlora_bf16 *>(ws);
-  float *cprime = reinterpret_cast<float *>(ws + align256(static_cast<size_t>(M) * r * 2));
-  float *part = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(cprime) + cprime_bytes(N, K));
+  unsigned int *counters = reinterpret_cast<unsigned int *>(ws);
+  qlora_bf16 *xas = reinterpret_cast<qlora_bf16 *>(ws + w.counters);
+  float *cprime = reinterpret_cast<float *>(ws + w.counters + w.mr);
+  float *part = reinterpret_cast<float *>(ws + w.counters + w.mr + w.cprime);
 
-  // 1) XA = X A (split-K partials) -> XA_out = bf16(XA), xas = bf16(s XA)
-  if (XA_out != nullptr)
-    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, 1.0f, XA_out, r, scl, xas, r, false, part, d.sms, cs);
-  else
-    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, scl, xas, r, 0.0f, nullptr, 0, false, part, d.sms, cs);
+  // 1) block constants c' for the GEMM producers (also zeroes the tile counters)
+  st = launch_decode_constants(q, scale2, t8, N, K / 64, cprime, counters, w.ncounters, d.sms, cs);
   if (st != QLORA_OK) return st;
 
-  // 2) block constants c' for the GEMM producers
-  st = launch_decode_constants(q, scale2, t8, N, K / 64, cprime, d.sms, cs);
-  if (st != QLORA_OK) return st;
+  // 2) XA = X A -> XA_out = bf16(XA) (if wanted), xas = bf16(s XA)
+  {
+    OutSpec o{xas, r, scl, XA_out, r, 1.0f, false};
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, part, counters, d.sms, cs);
+    if (st != QLORA_OK) return st;
+  }
 
   // 3) Y^T[n, m] = W'[n, :] . X[m, :] + B^T[n, :] . xas[m, :]
   const FusedPlan fp = plan_fused(M, N, K / 64, d.sms);
@@ -509,21 +531,18 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   a.kblocks = static_cast<int>(K / 64);
   a.splits = fp.splits;
   a.lora_kblocks = static_cast<int>(cdiv(r, 64));
+  a.out = Y;
+  a.out_ld = N;
   a.out_scale = 1.0f;
+  a.transpose = 1;
+  a.part = part;
+  a.counters = counters;
   std::memcpy(a.nf4, nf4, sizeof a.nf4);
-  if (fp.splits == 1) {
-    a.out = Y;
-    a.out_ld = N;
-  } else {
-    a.out = part;
-  }
   trace_begin(cs);
   st = fp.bn == 32 ? run_fused_bn<32, A_DEQ_K, L2_A_MN>(a, d.sms, cs)
                    : run_fused_bn<256, A_DEQ_K, L2_A_MN>(a, d.sms, cs);
   trace_end(cs);
-  if (st != QLORA_OK || fp.splits == 1) return st;
-  return launch_reduce(part, fp.splits, static_cast<int>(N), static_cast<int>(M), cdiv(N, 128) * 128,
-                       cdiv(M, fp.bn) * fp.bn, 1.0f, Y, N, 0.0f, nullptr, 0, true, d.sms, cs);
+  return st;
 }
 
 qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const float *scale2, const float nf4[16],
@@ -544,20 +563,24 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const float scl = alpha / static_cast<float>(r);
 
+  const WsLayout w = ws_layout(s, d.sms, true);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  const size_t mr = align256(static_cast<size_t>(M) * r * 2);
-  qlora_bf16 *gs = reinterpret_cast<qlora_bf16 *>(ws);
-  qlora_bf16 *xa_ws = reinterpret_cast<qlora_bf16 *>(ws + mr);
-  float *cprime = reinterpret_cast<float *>(ws + 2 * mr);
-  float *part = reinterpret_cast<float *>(ws + 2 * mr + cprime_bytes(N, K));
+  unsigned int *counters = reinterpret_cast<unsigned int *>(ws);
+  qlora_bf16 *gs = reinterpret_cast<qlora_bf16 *>(ws + w.counters);
+  qlora_bf16 *xa_ws = reinterpret_cast<qlora_bf16 *>(ws + w.counters + w.mr);
+  float *cprime = reinterpret_cast<float *>(ws + w.counters + 2 * w.mr);
+  float *part = reinterpret_cast<float *>(ws + w.counters + 2 * w.mr + w.cprime);
 
-  // 1) Gs = bf16(s * dY B^T)
-  st = skinny(SK_G, dY, N, M, B, N, r, M, N, r, scl, gs, r, 0.0f, nullptr, 0, false, part, d.sms, cs);
+  // 1) block constants c' (also zeroes the tile counters)
+  st = launch_decode_constants(q, scale2, t8, N, K / 64, cprime, counters, w.ncounters, d.sms, cs);
   if (st != QLORA_OK) return st;
 
-  // 2) block constants c' for the GEMM producers
-  st = launch_decode_constants(q, scale2, t8, N, K / 64, cprime, d.sms, cs);
-  if (st != QLORA_OK) return st;
+  // 2) Gs = bf16(s * dY B^T)
+  {
+    OutSpec o{gs, r, scl, nullptr, 0, 0.0f, false};
+    st = skinny(SK_G, dY, N, M, B, N, r, M, N, r, o, part, counters, d.sms, cs);
+    if (st != QLORA_OK) return st;
+  }
 
   // 3) dX^T[k, m] = W'^T[k, :] . dY[m, :] + A[k, :] . Gs[m, :]
   const FusedPlan fp = plan_fused(M, K, N / 64, d.sms);
@@ -575,37 +598,36 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   a.kblocks = static_cast<int>(N / 64);
   a.splits = fp.splits;
   a.lora_kblocks = static_cast<int>(cdiv(r, 64));
+  a.out = dX;
+  a.out_ld = K;
   a.out_scale = 1.0f;
+  a.transpose = 1;
+  a.part = part;
+  a.counters = counters;
   std::memcpy(a.nf4, nf4, sizeof a.nf4);
-  if (fp.splits == 1) {
-    a.out = dX;
-    a.out_ld = K;
-  } else {
-    a.out = part;
-  }
   trace_begin(cs);
   st = fp.bn == 32 ? run_fused_bn<32, A_DEQ_MN, L2_A_K>(a, d.sms, cs)
                    : run_fused_bn<256, A_DEQ_MN, L2_A_K>(a, d.sms, cs);
   trace_end(cs);
   if (st != QLORA_OK) return st;
-  if (fp.splits > 1) {
-    st = launch_reduce(part, fp.splits, static_cast<int>(K), static_cast<int>(M), cdiv(K, 128) * 128,
-                       cdiv(M, fp.bn) * fp.bn, 1.0f, dX, K, 0.0f, nullptr, 0, true, d.sms, cs);
-    if (st != QLORA_OK) return st;
-  }
 
   // 4) dA = X^T Gs   ([K, r])
-  st = skinny(SK_DA, X, K, M, gs, r, M, K, M, r, 1.0f, dA, r, 0.0f, nullptr, 0, false, part, d.sms, cs);
-  if (st != QLORA_OK) return st;
+  {
+    OutSpec o{dA, r, 1.0f, nullptr, 0, 0.0f, false};
+    st = skinny(SK_DA, X, K, M, gs, r, M, K, M, r, o, part, counters, d.sms, cs);
+    if (st != QLORA_OK) return st;
+  }
 
   // 5) XA (saved or recomputed), then dB = s XA^T dY   ([r, N], from dB^T[n, j])
   const qlora_bf16 *xa = XA;
   if (xa == nullptr) {
-    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, 1.0f, xa_ws, r, 0.0f, nullptr, 0, false, part, d.sms, cs);
+    OutSpec o{xa_ws, r, 1.0f, nullptr, 0, 0.0f, false};
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, part, counters, d.sms, cs);
     if (st != QLORA_OK) return st;
     xa = xa_ws;
   }
-  return skinny(SK_DB, dY, N, M, xa, r, M, N, M, r, scl, dB, N, 0.0f, nullptr, 0, true, part, d.sms, cs);
+  OutSpec o{dB, N, scl, nullptr, 0, 0.0f, true};
+  return skinny(SK_DB, dY, N, M, xa, r, M, N, M, r, o, part, counters, d.sms, cs);
 }
 
 }  // extern "C"
