@@ -48,60 +48,103 @@ __device__ __forceinline__ float div_by_recip(float w, float c, float r) {
   return __fmaf_rn(e, r, q0);
 }
 
+// Bucketed encode. y = RN(16 x + 16 + 1.5 * 2^23) rounds 16 x + 16 to an
+// integer (the ulp at that magnitude is 1) and is monotone in x, so the
+// bucket j = bits(y) - bits(1.5 * 2^23) in [0, 32] is an interval of x
+// values (|x| <= 1). The host builds, for each bucket, the code of its first
+// x (cand) and the one midpoint that falls strictly inside it (thr; 2.0
+// when none), after checking that no bucket holds two; then
+// code(x) = cand[j] + (x > thr[j]) exactly. Tables whose midpoints are
+// closer than a bucket width (1/16) use the binary search instead.
+struct BucketTable {
+  float thr[33];
+  unsigned int cand[33];
+};
+constexpr float kBucketMagic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ uint32_t nf4_code_bucket(float x, const float2 *bk) {
+  const float y = __fmaf_rn(x, 16.0f, 16.0f + kBucketMagic);
+  const uint32_t j = min(__float_as_uint(y) - __float_as_uint(kBucketMagic), 32u);  // |x| <= 1 keeps j <= 32
+  const float2 e = bk[j];
+  return __float_as_uint(e.y) + (x > e.x ? 1u : 0u);
+}
+
+// Encode of one 64-block slice: 8 weights (one 16-byte word) -> 8 nibbles.
+template <bool BUCKET>
+__device__ __forceinline__ uint32_t encode8(const float (&f)[8], float c, const float *s_mid, float mid7,
+                                            const float2 *s_bk) {
+  auto code = [&](float x) -> uint32_t {
+    return BUCKET ? nf4_code_bucket(x, s_bk) : nf4_code(x, s_mid, mid7);
+  };
+  uint32_t word = 0;
+  if (c == 0.0f) {
+    word = code(0.0f) * 0x11111111u;
+  } else if (c >= 0x1p-125f && c <= 0x1p125f) {
+    const float r = __frcp_rn(c);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) word |= code(div_by_recip(f[i], c, r)) << (4 * i);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) word |= code(__fdiv_rn(f[i], c)) << (4 * i);
+  }
+  return word;
+}
+
 // One 64-weight block per 8 lanes; each lane encodes 8 consecutive weights
-// (one 16-byte load) into one 32-bit word of 8 nibbles.
+// (one 16-byte load) into one 32-bit word of 8 nibbles. A warp takes 8
+// blocks per iteration (two independent 16-byte loads per lane in flight).
+template <bool BUCKET>
 __global__ void __launch_bounds__(256) quantize_nf4_kernel(const uint4 *__restrict__ W,
                                                            int64_t nblocks,
                                                            uint32_t *__restrict__ packed,
                                                            float *__restrict__ absmax,
-                                                           const CodecTables tabs) {
+                                                           const CodecTables tabs, const BucketTable bt) {
   __shared__ float s_mid[16];
+  __shared__ float2 s_bk[33];
   if (threadIdx.x < 15)
     s_mid[threadIdx.x] = __fmul_rn(__fadd_rn(tabs.nf4[threadIdx.x], tabs.nf4[threadIdx.x + 1]), 0.5f);
+  if (threadIdx.x < 33) s_bk[threadIdx.x] = make_float2(bt.thr[threadIdx.x], __uint_as_float(bt.cand[threadIdx.x]));
   __syncthreads();
+  grid_dep_wait();
+  grid_dep_launch();
   const float mid7 = s_mid[7];
   const uint32_t sub = threadIdx.x & 7u;
   const uint32_t lane = threadIdx.x & 31u;
   const int64_t nwords = nblocks * 8;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x * 2;
   // The loop runs per warp (base is warp-uniform) so the shuffles below
   // always see all 32 lanes; lanes past the end compute on zeros.
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31u);
+  for (int64_t base = (static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31u)) * 2;
        base < nwords; base += stride) {
-    const int64_t t = base + lane;
-    const bool valid = t < nwords;
-    const int64_t b = t >> 3;
-    const uint4 v = valid ? __ldg(&W[t]) : make_uint4(0u, 0u, 0u, 0u);
-    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-    float f[8];
+    int64_t t[2];
+    uint4 v[2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      f[2 * i] = __uint_as_float(wd[i] << 16);
-      f[2 * i + 1] = __uint_as_float(wd[i] & 0xFFFF0000u);
+    for (int h = 0; h < 2; ++h) {
+      t[h] = base + 32 * h + lane;
+      v[h] = t[h] < nwords ? __ldg(&W[t[h]]) : make_uint4(0u, 0u, 0u, 0u);
     }
-    float m = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
-    // each 8-lane group (one 64-block) reduces independently
-    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
-    const float c = m;
-    uint32_t word = 0;
-    if (c == 0.0f) {
-      const uint32_t z = nf4_code(0.0f, s_mid, mid7);
-      word = z * 0x11111111u;
-    } else if (c >= 0x1p-125f && c <= 0x1p125f) {
-      const float r = __frcp_rn(c);
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t wd[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
+      float f[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) word |= nf4_code(div_by_recip(f[i], c, r), s_mid, mid7) << (4 * i);
-    } else {
+      for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(wd[i] << 16);
+        f[2 * i + 1] = __uint_as_float(wd[i] & 0xFFFF0000u);
+      }
+      float m = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) word |= nf4_code(__fdiv_rn(f[i], c), s_mid, mid7) << (4 * i);
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+      // each 8-lane group (one 64-block) reduces independently
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+      const uint32_t word = encode8<BUCKET>(f, m, s_mid, mid7, s_bk);
+      if (t[h] < nwords) {
+        packed[t[h]] = word;
+        if (sub == 0) absmax[t[h] >> 3] = m;
+      }
     }
-    if (!valid) continue;
-    packed[t] = word;
-    if (sub == 0) absmax[b] = c;
   }
 }
 
@@ -117,6 +160,8 @@ __global__ void __launch_bounds__(256) double_quant_kernel(const float *__restri
   if (threadIdx.x < 255)
     s_mid[threadIdx.x] = __fmul_rn(__fadd_rn(tabs.t8[threadIdx.x], tabs.t8[threadIdx.x + 1]), 0.5f);
   __syncthreads();
+  grid_dep_wait();
+  grid_dep_launch();
   const int lane = threadIdx.x & 31;
   const int64_t ng = (nb + 255) / 256;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -207,39 +252,62 @@ __device__ __forceinline__ void nf4_lookup8(const Nf4Planes &P, uint32_t w, uint
   }
 }
 
-// Standalone dequantization: one lane per 16 consecutive weights
-// (a quarter of a 64-block): 8 packed bytes in, 32 bytes of bf16 out.
-__global__ void __launch_bounds__(256) dequant_kernel(const uint2 *__restrict__ packed,
+// Standalone dequantization: one lane per 64-block (its bf16 table built
+// once), 32 consecutive blocks per warp. Each lane writes its 128 output
+// bytes into a padded shared-memory row, and the warp then stores the 4 KB
+// with fully coalesced 16-byte stores.
+__global__ void __launch_bounds__(256) dequant_kernel(const uint4 *__restrict__ packed,
                                                       const uint8_t *__restrict__ q,
                                                       const float *__restrict__ scale2,
-                                                      int64_t nquarters, uint4 *__restrict__ out,
+                                                      int64_t nblocks, uint4 *__restrict__ out,
                                                       const CodecTables tabs) {
   __shared__ float s_t8[256];
+  __shared__ uint4 s_stage[8][32 * 9];  // per warp: 32 rows of 128 B, padded to 144 B
   s_t8[threadIdx.x] = tabs.t8[threadIdx.x];
   __syncthreads();
+  grid_dep_wait();
+  grid_dep_launch();
   float L[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) L[i] = tabs.nf4[i];
-  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < nquarters;
-       t += nthreads) {
-    const int64_t b = t >> 2;
-    const uint2 pk = __ldg(&packed[t]);
-    const float cp = __fmul_rn(s_t8[__ldg(&q[b])], __ldg(&scale2[b >> 8]));
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  uint4 *stage = s_stage[wid];
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * 8;
+  for (int64_t b0 = (static_cast<int64_t>(blockIdx.x) * 8 + wid) * 32; b0 < nblocks; b0 += nwarps * 32) {
+    const int64_t b = b0 + lane;
+    const bool valid = b < nblocks;
+    uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
+    float cp = 0.0f;
+    if (valid) {
+      w0 = __ldg(&packed[2 * b]);
+      w1 = __ldg(&packed[2 * b + 1]);
+      cp = __fmul_rn(s_t8[__ldg(&q[b])], __ldg(&scale2[b >> 8]));
+    }
     const Nf4Planes P = make_planes(L, cp);
-    uint32_t o0[4], o1[4];
-    nf4_lookup8(P, pk.x, o0);
-    nf4_lookup8(P, pk.y, o1);
-    out[2 * t] = make_uint4(o0[0], o0[1], o0[2], o0[3]);
-    out[2 * t + 1] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+    const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      uint32_t o[4];
+      nf4_lookup8(P, words[c], o);
+      stage[lane * 9 + c] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    __syncwarp();
+    const int64_t nvalid = nblocks - b0 < 32 ? nblocks - b0 : 32;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int idx = i * 32 + lane;  // 16-byte chunk of the warp's 4 KB
+      const int row = idx >> 3, ch = idx & 7;
+      if (row < nvalid) out[b0 * 8 + idx] = stage[row * 9 + ch];
+    }
+    __syncwarp();
   }
 }
 
 // ------------------------------------------------------------------------
 // Decoded block constants for the GEMMs, block-major: cprime[kb * N + n] =
 // t8[q_b] * scale2[b / 256] (fp32 product), b = n * KB + kb. One thread per
-// (row n, 16 consecutive blocks); consecutive threads take consecutive rows
-// so every store instruction writes a contiguous run of one kb row. The
+// constant; consecutive threads take consecutive rows n of one kb, so the
+// stores are coalesced (the 8-bit codes are small and L2-resident). The
 // launch also zeroes `ncounters` split-K tile counters.
 __global__ void __launch_bounds__(256) decode_constants_kernel(const uint8_t *__restrict__ q,
                                                                const float *__restrict__ scale2,
@@ -250,21 +318,17 @@ __global__ void __launch_bounds__(256) decode_constants_kernel(const uint8_t *__
   __shared__ float s_t8[256];
   s_t8[threadIdx.x] = tabs.t8[threadIdx.x];
   __syncthreads();
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < ncounters;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    counters[i] = 0u;
-  const int64_t chunks = (KB + 15) / 16;
-  const int64_t total = N * chunks;
+  grid_dep_wait();
+  grid_dep_launch();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total; t += stride) {
-    const int64_t ch = t / N;
-    const int64_t n = t - ch * N;
-    const int64_t kb0 = ch * 16;
-    const int64_t kb1 = kb0 + 16 < KB ? kb0 + 16 : KB;
-    for (int64_t kb = kb0; kb < kb1; ++kb) {
-      const int64_t b = n * KB + kb;
-      cprime[kb * N + n] = __fmul_rn(s_t8[__ldg(q + b)], __ldg(scale2 + (b >> 8)));
-    }
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (int64_t i = first; i < ncounters; i += stride) counters[i] = 0u;
+  const int64_t total = N * KB;
+  for (int64_t t = first; t < total; t += stride) {
+    const int64_t kb = t / N;
+    const int64_t n = t - kb * N;
+    const int64_t b = n * KB + kb;
+    cprime[t] = __fmul_rn(s_t8[__ldg(q + b)], __ldg(scale2 + (b >> 8)));
   }
 }
 

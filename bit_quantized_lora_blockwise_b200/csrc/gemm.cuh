@@ -127,12 +127,6 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs &a, int tile, int
   return t;
 }
 
-// Warp-collective bounded wait: every lane waits (each acquires), and the
-// warp gives up together if any lane gave up.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
-  const bool ok = mbar_wait(bar, parity, abort_flag);
-  return __all_sync(0xFFFFFFFFu, ok);
-}
 
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_constant__ GemmArgs args) {
@@ -197,6 +191,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
+  // everything above overlaps the previous kernel's tail; its outputs are
+  // read only below
+  grid_dep_wait();
+  grid_dep_launch();
 
   const int row_tiles = (args.rows + 127) / 128;
   const int col_tiles = (args.cols + C::BN - 1) / C::BN;
@@ -347,7 +345,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++iter) {
       const TileCoord t = tile_coord(args, tile, row_tiles, col_tiles, C::BN);
       const int acc = iter & 1;
-      if (!warp_wait(tmem_full(acc), (iter >> 1) & 1u, s_abort)) break;
+      if (!warp_wait_all(tmem_full(acc), (iter >> 1) & 1u, s_abort)) break;
       tc_fence_after();
       const int row = t.row0 + qrow;
       const uint32_t tcol = tmem_base + ((uint32_t)(warp * 32) << 16) + acc * C::BN;
@@ -472,10 +470,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
         if (main_job) ++mj;
         if ((int)(job % C::NGROUPS) != group) continue;
         const int sa = job % C::SA;
-        if (!warp_wait(a_empty(sa), ((job / C::SA) & 1u) ^ 1u, s_abort)) { ok = false; break; }
+        if (!warp_wait_all(a_empty(sa), ((job / C::SA) & 1u) ^ 1u, s_abort)) { ok = false; break; }
         if (main_job) {
           const int sp = my_mj % C::SP;
-          if (!warp_wait(p_full(sp), (my_mj / C::SP) & 1u, s_abort)) { ok = false; break; }
+          if (!warp_wait_all(p_full(sp), (my_mj / C::SP) & 1u, s_abort)) { ok = false; break; }
           const uint8_t *pslot = smem + C::OFF_P + sp * C::P_BYTES;
           const float cp = reinterpret_cast<const float *>(pslot + C::PK_BYTES)[p];
           const uint4 w0 = *reinterpret_cast<const uint4 *>(pslot + p_off);

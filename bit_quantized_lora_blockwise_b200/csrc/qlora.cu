@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <utility>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -15,6 +16,7 @@
 #include "qlora.h"
 #include "codec.cuh"
 #include "gemm.cuh"
+#include "skinny.cuh"
 #include "ptx.cuh"
 
 using namespace qlora;
@@ -39,11 +41,6 @@ std::atomic<uint64_t> g_launches{0};
 thread_local cudaEvent_t t_trace_start = nullptr;
 thread_local cudaEvent_t t_trace_stop = nullptr;
 
-// Every kernel launch goes through here: counts it and maps a launch error.
-qlora_status launched() {
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
-}
 
 qlora_status device_info(DeviceInfo *out) {
   int dev = 0;
@@ -90,6 +87,58 @@ CodecTables make_tables(const float *nf4, const float *t8) {
   if (nf4) std::memcpy(t.nf4, nf4, sizeof t.nf4);
   if (t8) std::memcpy(t.t8, t8, sizeof t.t8);
   return t;
+}
+
+// Bucket table of the exact bucketed encode (see BucketTable): false when
+// two midpoints fall inside one bucket (the binary search is used then).
+// Host float arithmetic here is IEEE binary32 with the same operation order
+// as the device (sum then halve; one fused multiply-add for the bucket).
+bool build_buckets(const float *L, BucketTable *bt) {
+  auto bucket = [](float x) {  // same arithmetic as nf4_code_bucket (|x| <= 1)
+    const float y = std::fmaf(x, 16.0f, 16.0f + kBucketMagic);
+    uint32_t a, b;
+    std::memcpy(&a, &y, 4);
+    std::memcpy(&b, &kBucketMagic, 4);
+    return static_cast<int>(a - b);
+  };
+  int jm[15], jp[15], inside[33] = {0};
+  for (int j = 0; j < 33; ++j) bt->thr[j] = 2.0f;
+  for (int i = 0; i < 15; ++i) {
+    const float m = (L[i] + L[i + 1]) * 0.5f;
+    jm[i] = bucket(m);
+    jp[i] = bucket(std::nextafter(m, 2.0f));
+    if (jm[i] == jp[i]) {
+      if (inside[jm[i]]++) return false;
+      bt->thr[jm[i]] = m;
+    }
+  }
+  for (int j = 0; j < 33; ++j) {
+    unsigned int c = 0;
+    for (int i = 0; i < 15; ++i) c += (jp[i] < j || (jp[i] == j && jm[i] < j)) ? 1u : 0u;
+    bt->cand[j] = c;
+  }
+  return true;
+}
+
+// Every kernel is launched with programmatic stream serialization: it may
+// start (prologue only) while the previous kernel in the stream finishes,
+// and waits for it (griddepcontrol.wait) before touching its outputs.
+template <typename... KArgs, typename... Args>
+qlora_status launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t stream,
+                        Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 int grid_for(int64_t work_items, int per_cta, int sms, int waves) {
@@ -164,8 +213,7 @@ qlora_status launch_gemm(const GemmArgs &args, int sms, cudaStream_t stream) {
   const int col_tiles = (args.cols + C::BN - 1) / C::BN;
   const int tiles = row_tiles * col_tiles * args.splits;
   const int grid = tiles < sms ? tiles : sms;
-  qgemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(args);
-  return launched();
+  return launch_pdl(qgemm_kernel<C>, grid, C::THREADS, C::SMEM_BYTES, stream, args);
 }
 
 // Block constants c' = t8[q] * S, block-major [K/64][N] fp32 (GEMM operand
@@ -174,10 +222,9 @@ qlora_status launch_gemm(const GemmArgs &args, int sms, cudaStream_t stream) {
 qlora_status launch_decode_constants(const uint8_t *q, const float *scale2, const float *t8, int64_t N,
                                      int64_t KB, float *cprime, unsigned int *counters, int64_t ncounters,
                                      int sms, cudaStream_t stream) {
-  const int grid = grid_for(N * cdiv(KB, 16), 256, sms, 8);
-  decode_constants_kernel<<<grid, 256, 0, stream>>>(q, scale2, N, KB, cprime, counters, ncounters,
-                                                    make_tables(nullptr, t8));
-  return launched();
+  const int grid = grid_for(N * KB, 256, sms, 8);
+  return launch_pdl(decode_constants_kernel, grid, 256, 0, stream, q, scale2, N, KB, cprime, counters,
+                    ncounters, make_tables(nullptr, t8));
 }
 
 size_t cprime_bytes(int64_t N, int64_t K) { return align256(static_cast<size_t>(N) * (K / 64) * 4); }
@@ -204,34 +251,59 @@ int rank_tile(int r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
 
 struct SkinnyPlan {
   int rows, kblocks, splits, bn;
-  size_t part_bytes;
+  size_t part_bytes;  // none: the split-K partials are reduced in shared memory
 };
 
+// Split K over a cluster of 1, 2, 4 or 8 CTAs per 128-row tile, one wave.
 SkinnyPlan plan_skinny(int64_t rows, int64_t kdim, int r, int sms) {
   SkinnyPlan p;
   p.rows = static_cast<int>(rows);
   p.kblocks = static_cast<int>(cdiv(kdim, 64));
   p.bn = rank_tile(r);
   const int row_tiles = static_cast<int>(cdiv(rows, 128));
-  int splits = sms / row_tiles;  // one wave
-  if (splits > p.kblocks) splits = p.kblocks;
-  if (splits < 1) splits = 1;
+  int splits = 1;
+  while (splits < 8 && 2 * splits * row_tiles <= sms && 2 * splits <= p.kblocks) splits *= 2;
   p.splits = splits;
-  p.part_bytes = splits > 1 ? align256(static_cast<size_t>(splits) * row_tiles * 128 * p.bn * 4) : 0;
+  p.part_bytes = 0;
   return p;
 }
 
-template <int BN, int AS, int BS>
-qlora_status run_skinny_bn(const GemmArgs &a, int sms, cudaStream_t st) {
-  constexpr int S = BN == 256 ? 4 : 6;
-  return launch_gemm<GemmCfg<BN, AS, BS, L2_NONE, S, S, 0, 0>>(a, sms, st);
+template <int BN, bool AMN, bool BMN>
+qlora_status run_skinny_bn(const SkinnyArgs &a, int row_tiles, cudaStream_t st) {
+  constexpr int S = BN == 64 ? 8 : (BN == 128 ? 6 : 4);
+  using C = SkinnyCfg<BN, AMN, BMN, S>;
+  static std::once_flag once[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(once[dev], [&] {
+    attr_err = cudaFuncSetAttribute(skinny_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return QLORA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(row_tiles * a.splits);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = a.splits;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.splits > 1 ? 2 : 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, skinny_kernel<C>, a);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
-template <int AS, int BS>
-qlora_status run_skinny(const GemmArgs &a, int bn, int sms, cudaStream_t st) {
-  if (bn == 64) return run_skinny_bn<64, AS, BS>(a, sms, st);
-  if (bn == 128) return run_skinny_bn<128, AS, BS>(a, sms, st);
-  return run_skinny_bn<256, AS, BS>(a, sms, st);
+template <bool AMN, bool BMN>
+qlora_status run_skinny(const SkinnyArgs &a, int bn, int row_tiles, cudaStream_t st) {
+  if (bn == 64) return run_skinny_bn<64, AMN, BMN>(a, row_tiles, st);
+  if (bn == 128) return run_skinny_bn<128, AMN, BMN>(a, row_tiles, st);
+  return run_skinny_bn<256, AMN, BMN>(a, row_tiles, st);
 }
 
 // kind: SK_XA   Aop = X [M,K] (K-major),   Bop = A  [K,r] (MN-major), rows = M, kdim = K
@@ -250,9 +322,9 @@ struct OutSpec {
 
 qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a_outer, const void *bop,
                     int64_t b_inner, int64_t b_outer, int64_t rows, int64_t kdim, int r, const OutSpec &o,
-                    float *part, unsigned int *counters, int sms, cudaStream_t st) {
+                    int sms, cudaStream_t st) {
   const SkinnyPlan p = plan_skinny(rows, kdim, r, sms);
-  GemmArgs a;
+  SkinnyArgs a;
   std::memset(&a, 0, sizeof a);
   bool ok = true;
   switch (kind) {
@@ -276,17 +348,15 @@ qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a
   a.out2_ld = o.ld2;
   a.out2_scale = o.scale2;
   a.transpose = o.transpose ? 1 : 0;
-  a.part = part;
-  a.counters = counters;
   a.rows = p.rows;
   a.cols = r;
   a.kblocks = p.kblocks;
   a.splits = p.splits;
-  a.lora_kblocks = 0;
+  const int row_tiles = static_cast<int>(cdiv(rows, 128));
   switch (kind) {
-    case SK_XA: return run_skinny<A_TMA_K, B_TMA_MN>(a, p.bn, sms, st);
-    case SK_G: return run_skinny<A_TMA_K, B_TMA_K>(a, p.bn, sms, st);
-    default: return run_skinny<A_TMA_MN, B_TMA_MN>(a, p.bn, sms, st);
+    case SK_XA: return run_skinny<false, true>(a, p.bn, row_tiles, st);
+    case SK_G: return run_skinny<false, false>(a, p.bn, row_tiles, st);
+    default: return run_skinny<true, true>(a, p.bn, row_tiles, st);
   }
 }
 
@@ -439,11 +509,12 @@ qlora_status qlora_quantize_nf4(const qlora_bf16 *W, int64_t N, int64_t K, const
   DeviceInfo d;
   if ((st = device_info(&d)) != QLORA_OK) return st;
   const int64_t nblocks = N * (K / 64);
-  const int grid = grid_for(nblocks * 8, 256, d.sms, 16);
-  quantize_nf4_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const uint4 *>(W), nblocks, reinterpret_cast<uint32_t *>(packed), absmax,
-      make_tables(nf4, nullptr));
-  return launched();
+  const int grid = grid_for(nblocks * 8, 512, d.sms, 8);
+  BucketTable bt;
+  const bool bucketed = build_buckets(nf4, &bt);
+  return launch_pdl(bucketed ? quantize_nf4_kernel<true> : quantize_nf4_kernel<false>, grid, 256, 0,
+                    static_cast<cudaStream_t>(stream), reinterpret_cast<const uint4 *>(W), nblocks,
+                    reinterpret_cast<uint32_t *>(packed), absmax, make_tables(nf4, nullptr), bt);
 }
 
 qlora_status qlora_double_quant(const float *absmax, int64_t nb, const float t8[256], uint8_t *q, float *scale2,
@@ -457,9 +528,8 @@ qlora_status qlora_double_quant(const float *absmax, int64_t nb, const float t8[
   if ((st = device_info(&d)) != QLORA_OK) return st;
   const int64_t ng = cdiv(nb, 256);
   const int grid = grid_for(ng, 8, d.sms, 16);
-  double_quant_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(absmax, nb, q, scale2,
-                                                                            make_tables(nullptr, t8));
-  return launched();
+  return launch_pdl(double_quant_kernel, grid, 256, 0, static_cast<cudaStream_t>(stream), absmax, nb, q, scale2,
+                    make_tables(nullptr, t8));
 }
 
 qlora_status qlora_dequant(const uint8_t *packed, const uint8_t *q, const float *scale2, int64_t N, int64_t K,
@@ -471,12 +541,11 @@ qlora_status qlora_dequant(const uint8_t *packed, const uint8_t *q, const float 
   if (st != QLORA_OK) return st;
   DeviceInfo d;
   if ((st = device_info(&d)) != QLORA_OK) return st;
-  const int64_t quarters = N * K / 16;
-  const int grid = grid_for(quarters, 256, d.sms, 16);
-  dequant_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const uint2 *>(packed), q, scale2, quarters, reinterpret_cast<uint4 *>(W_out),
-      make_tables(nf4, t8));
-  return launched();
+  const int64_t nblocks = N * K / 64;
+  const int grid = grid_for(nblocks, 256, d.sms, 4);
+  return launch_pdl(dequant_kernel, grid, 256, 0, static_cast<cudaStream_t>(stream),
+                    reinterpret_cast<const uint4 *>(packed), q, scale2, nblocks, reinterpret_cast<uint4 *>(W_out),
+                    make_tables(nf4, t8));
 }
 
 qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const float *scale2, const float nf4[16],
@@ -511,7 +580,7 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   // 2) XA = X A -> XA_out = bf16(XA) (if wanted), xas = bf16(s XA)
   {
     OutSpec o{xas, r, scl, XA_out, r, 1.0f, false};
-    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, part, counters, d.sms, cs);
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs);
     if (st != QLORA_OK) return st;
   }
 
@@ -578,7 +647,7 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   // 2) Gs = bf16(s * dY B^T)
   {
     OutSpec o{gs, r, scl, nullptr, 0, 0.0f, false};
-    st = skinny(SK_G, dY, N, M, B, N, r, M, N, r, o, part, counters, d.sms, cs);
+    st = skinny(SK_G, dY, N, M, B, N, r, M, N, r, o, d.sms, cs);
     if (st != QLORA_OK) return st;
   }
 
@@ -614,7 +683,7 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   // 4) dA = X^T Gs   ([K, r])
   {
     OutSpec o{dA, r, 1.0f, nullptr, 0, 0.0f, false};
-    st = skinny(SK_DA, X, K, M, gs, r, M, K, M, r, o, part, counters, d.sms, cs);
+    st = skinny(SK_DA, X, K, M, gs, r, M, K, M, r, o, d.sms, cs);
     if (st != QLORA_OK) return st;
   }
 
@@ -622,12 +691,12 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   const qlora_bf16 *xa = XA;
   if (xa == nullptr) {
     OutSpec o{xa_ws, r, 1.0f, nullptr, 0, 0.0f, false};
-    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, part, counters, d.sms, cs);
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs);
     if (st != QLORA_OK) return st;
     xa = xa_ws;
   }
   OutSpec o{dB, N, scl, nullptr, 0, 0.0f, true};
-  return skinny(SK_DB, dY, N, M, xa, r, M, N, M, r, o, part, counters, d.sms, cs);
+  return skinny(SK_DB, dY, N, M, xa, r, M, N, M, r, o, d.sms, cs);
 }
 
 }  // extern "C"
