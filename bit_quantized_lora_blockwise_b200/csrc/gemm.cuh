@@ -95,7 +95,7 @@ struct GemmCfg {
   // tmem_full[2] tmem_empty[2] drain
   static constexpr int NBARS = 2 * SB + 2 * SA + 2 * SP + 5;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem base, abort flag, last-CTA flag
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int WARPS = DEQ ? 7 + NPW_ : 6;
   static constexpr int THREADS = WARPS * 32;
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64
@@ -130,8 +130,8 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs &a, int tile, int
 
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_constant__ GemmArgs args) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = smem_raw;  // 1024-byte aligned: the 128-byte swizzle atoms need it
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;

@@ -254,15 +254,20 @@ struct SkinnyPlan {
   size_t part_bytes;  // none: the split-K partials are reduced in shared memory
 };
 
-// Split K over a cluster of 1, 2, 4 or 8 CTAs per 128-row tile, one wave.
+// Split K over a cluster of 1, 2 or 4 CTAs per 128-row tile, in one wave.
+// (One CTA per SM; measured on B200: at most 15 eight-CTA clusters, 33
+// four-CTA clusters and 74 two-CTA clusters are co-resident, so clusters of 8
+// would spill into a second wave.)
 SkinnyPlan plan_skinny(int64_t rows, int64_t kdim, int r, int sms) {
   SkinnyPlan p;
   p.rows = static_cast<int>(rows);
   p.kblocks = static_cast<int>(cdiv(kdim, 64));
   p.bn = rank_tile(r);
   const int row_tiles = static_cast<int>(cdiv(rows, 128));
+  const int max_clusters4 = (sms * 33) / 148, max_clusters2 = (sms * 74) / 148;
   int splits = 1;
-  while (splits < 8 && 2 * splits * row_tiles <= sms && 2 * splits <= p.kblocks) splits *= 2;
+  if (row_tiles <= max_clusters4 && 4 <= p.kblocks) splits = 4;
+  else if (row_tiles <= max_clusters2 && 2 <= p.kblocks) splits = 2;
   p.splits = splits;
   p.part_bytes = 0;
   return p;

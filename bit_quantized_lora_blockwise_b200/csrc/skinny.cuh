@@ -48,7 +48,7 @@ struct SkinnyCfg {
   static constexpr int OFF_BAR = OFF_B + STAGES_ * B_BYTES;
   static constexpr int NBARS = 2 * STAGES_ + 2;  // full[S], empty[S], tmem_full, drain
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int THREADS = 256;
   static constexpr uint32_t TMEM_COLS = BN_ <= 64 ? 64 : (BN_ <= 128 ? 128 : 256);
   static constexpr int PART_LD = BN_ + 4;  // fp32 per partial row (16-byte pad against bank conflicts)
@@ -59,8 +59,8 @@ struct SkinnyCfg {
 
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_constant__ SkinnyArgs args) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = smem_raw;  // 1024-byte aligned: the 128-byte swizzle atoms need it
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
