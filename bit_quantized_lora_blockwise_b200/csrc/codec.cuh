@@ -70,9 +70,36 @@ __device__ __forceinline__ uint32_t nf4_code_bucket(float x, const float2 *bk) {
 }
 
 // Encode of one 64-block slice: 8 weights (one 16-byte word) -> 8 nibbles.
+// The bucketed path runs the division and the bucket map on fp32 pairs
+// (f32x2 FMA/MUL: two IEEE round-to-nearest lanes per instruction) and packs
+// nibbles with one multiply-add each.
 template <bool BUCKET>
 __device__ __forceinline__ uint32_t encode8(const float (&f)[8], float c, const float *s_mid, float mid7,
                                             const float2 *s_bk) {
+  if (BUCKET && c >= 0x1p-125f && c <= 0x1p125f) {
+    const float r = __frcp_rn(c);
+    const unsigned long long R = f2_pack(r, r), NC = f2_pack(-c, -c);
+    const unsigned long long S16 = f2_pack(16.0f, 16.0f);
+    const unsigned long long OFF = f2_pack(16.0f + kBucketMagic, 16.0f + kBucketMagic);
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 3; i >= 0; --i) {  // pairs (6,7), (4,5), ... so the word fills from the top nibble
+      const unsigned long long W = f2_pack(f[2 * i], f[2 * i + 1]);
+      const unsigned long long Q0 = f2_mul(W, R);       // RN(w r)
+      const unsigned long long E = f2_fma(Q0, NC, W);   // w - q0 c, exact
+      const unsigned long long X = f2_fma(E, R, Q0);    // RN(q0 + e r) = RN(w / c)
+      const unsigned long long Y = f2_fma(X, S16, OFF);  // bucket map
+      float x0, x1, y0, y1;
+      f2_unpack(X, x0, x1);
+      f2_unpack(Y, y0, y1);
+      const uint32_t j1 = min(__float_as_uint(y1) - __float_as_uint(kBucketMagic), 32u);
+      const uint32_t j0 = min(__float_as_uint(y0) - __float_as_uint(kBucketMagic), 32u);
+      const float2 e1 = s_bk[j1], e0 = s_bk[j0];
+      word = word * 16u + __float_as_uint(e1.y) + (x1 > e1.x ? 1u : 0u);
+      word = word * 16u + __float_as_uint(e0.y) + (x0 > e0.x ? 1u : 0u);
+    }
+    return word;
+  }
   auto code = [&](float x) -> uint32_t {
     return BUCKET ? nf4_code_bucket(x, s_bk) : nf4_code(x, s_mid, mid7);
   };

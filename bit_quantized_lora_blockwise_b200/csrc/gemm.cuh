@@ -79,6 +79,7 @@ struct GemmCfg {
   static_assert(DEQ || (SA_ == SB_ && SP_ == 0 && NPW_ == 0), "TMA-only A shares the B ring");
   static_assert(DEQ || L2_ == L2_NONE, "low-rank steps only in the dequant variants");
   static_assert(BN_ % 16 == 0 && BN_ >= 16 && BN_ <= 256, "MMA N");
+  static constexpr int NCHUNK = (BN_ + 31) / 32;  // epilogue chunks of 32 columns (last may hold 16)
   static_assert(!B_MN || BN_ % 64 == 0, "MN-major B needs whole 64-wide chunks");
   static constexpr int A_BYTES = BM * BK * 2;  // 16 KB
   static constexpr int B_BYTES = BN * BK * 2;
@@ -100,6 +101,7 @@ struct GemmCfg {
   static constexpr int THREADS = WARPS * 32;
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64
                                         : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
+  static constexpr uint32_t ACC_STRIDE = TMEM_COLS / 2;  // column offset of accumulator 1
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
   static constexpr uint32_t MAIN_TX = B_BYTES + (DEQ ? 0 : A_BYTES);
   static constexpr uint32_t LORA_TX = A_BYTES + B_BYTES;
@@ -270,7 +272,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
         const int acc = iter & 1;
         if (!mbar_wait(tmem_empty(acc), ((iter >> 1) & 1u) ^ 1u, s_abort)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * C::BN;
+        const uint32_t d_tmem = tmem_base + acc * C::ACC_STRIDE;
         for (int jj = 0; jj < njobs; ++jj, ++job) {
           const int sb = job % C::SB;
           const int sa = C::DEQ ? (int)(job % C::SA) : sb;
@@ -313,12 +315,30 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     // writes the bf16 output.
     volatile int *s_last = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
     const int64_t rows_pad = static_cast<int64_t>(row_tiles) * 128;
-    const int64_t cols_pad = static_cast<int64_t>(col_tiles) * C::BN;
+    // partial rows are padded to whole 32-column chunks per tile
+    const int64_t cols_pad = static_cast<int64_t>(col_tiles) * C::NCHUNK * 32;
     uint32_t iter = 0;
     const int qrow = warp * 32 + lane;  // TMEM lane of this thread
-    auto store_out = [&](int row, int col_base, const float (&v)[32]) {
+    // chunk ch of the accumulator row (32 columns; a 16-column tail is zero-padded)
+    auto load_chunk = [&](uint32_t tcol, int ch, uint32_t (&u)[32]) {
+      if (C::BN % 32 == 16 && ch == C::NCHUNK - 1) {
+        uint32_t h[16];
+        tmem_ld_32x32b_x16(tcol + ch * 32, h);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          u[j] = h[j];
+          u[16 + j] = 0u;
+        }
+      } else {
+        tmem_ld_32x32b_x32(tcol + ch * 32, u);
+      }
+    };
+    // col_end: first column past this tile (a 240-wide tile's last chunk
+    // must not spill into the next tile)
+    auto store_out = [&](int row, int col_base, int col_end, const float (&v)[32]) {
       if (row >= args.rows) return;
-      const int ncol = args.cols - col_base < 32 ? args.cols - col_base : 32;
+      const int lim = col_end < args.cols ? col_end : args.cols;
+      const int ncol = lim - col_base < 32 ? lim - col_base : 32;
       for (int o = 0; o < 2; ++o) {
         __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(o ? args.out2 : args.out);
         if (dst == nullptr) continue;
@@ -348,27 +368,28 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
       if (!warp_wait_all(tmem_full(acc), (iter >> 1) & 1u, s_abort)) break;
       tc_fence_after();
       const int row = t.row0 + qrow;
-      const uint32_t tcol = tmem_base + ((uint32_t)(warp * 32) << 16) + acc * C::BN;
+      const uint32_t tcol = tmem_base + ((uint32_t)(warp * 32) << 16) + acc * C::ACC_STRIDE;
       if (args.splits == 1) {
 #pragma unroll 1
-        for (int ch = 0; ch < C::BN / 32; ++ch) {
+        for (int ch = 0; ch < C::NCHUNK; ++ch) {
           uint32_t u[32];
-          tmem_ld_32x32b_x32(tcol + ch * 32, u);
+          load_chunk(tcol, ch, u);
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(u[j]);
-          store_out(row, t.col0 + ch * 32, v);
+          store_out(row, t.col0 + ch * 32, t.col0 + C::BN, v);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(tmem_empty(acc));
         continue;
       }
-      float *prow = args.part + (static_cast<int64_t>(t.split) * rows_pad + row) * cols_pad + t.col0;
+      float *prow = args.part + (static_cast<int64_t>(t.split) * rows_pad + row) * cols_pad +
+                    (t.col0 / C::BN) * (C::NCHUNK * 32);
 #pragma unroll 1
-      for (int ch = 0; ch < C::BN / 32; ++ch) {
+      for (int ch = 0; ch < C::NCHUNK; ++ch) {
         uint32_t u[32];
-        tmem_ld_32x32b_x32(tcol + ch * 32, u);
+        load_chunk(tcol, ch, u);
         float4 *o = reinterpret_cast<float4 *>(prow + ch * 32);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
@@ -390,13 +411,14 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
       if (*s_last) {
         __threadfence();
 #pragma unroll 1
-        for (int ch = 0; ch < C::BN / 32; ++ch) {
+        for (int ch = 0; ch < C::NCHUNK; ++ch) {
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = 0.0f;
           for (int sp = 0; sp < args.splits; ++sp) {
             const float4 *src = reinterpret_cast<const float4 *>(
-                args.part + (static_cast<int64_t>(sp) * rows_pad + row) * cols_pad + t.col0 + ch * 32);
+                args.part + (static_cast<int64_t>(sp) * rows_pad + row) * cols_pad +
+                (t.col0 / C::BN) * (C::NCHUNK * 32) + ch * 32);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               const float4 x = __ldcg(src + j);
@@ -406,7 +428,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
               v[4 * j + 3] += x.w;
             }
           }
-          store_out(row, t.col0 + ch * 32, v);
+          store_out(row, t.col0 + ch * 32, t.col0 + C::BN, v);
         }
       }
     }

@@ -72,6 +72,8 @@ class Layer:
     (520, 384, 256, 16),     # three row tiles, K = 256
     (64, 128, 128, 128),     # rank 128
     (40, 256, 192, 256),     # rank 256 (four low-rank K blocks)
+    (2048, 4096, 512, 16),   # forward on 240-token tiles, 9 column tiles, no split
+    (2048, 512, 4096, 16),   # backward on 240-token tiles, no split
 ])
 def test_fwd_bwd_parity(M, N, K, r):
     L = Layer(M, N, K, r, seed=M * 7 + N + K + r)
