@@ -77,17 +77,23 @@ struct GemmCfg {
   static constexpr int NGROUPS = NPW_ >= 4 ? NPW_ / 4 : 1;
   static_assert(!DEQ || (NPW_ % 4 == 0 && NPW_ >= 4 && SP_ >= 2), "dequant needs producer groups and a P ring");
   static_assert(DEQ || (SA_ == SB_ && SP_ == 0 && NPW_ == 0), "TMA-only A shares the B ring");
+  // (a 16-warp, 3-slot configuration timed out on B200: keep a slot per
+  // producer group and one spare)
+  static_assert(!DEQ || SA_ > NPW_ / 4, "dequantized-tile ring needs more slots than producer groups");
   static_assert(DEQ || L2_ == L2_NONE, "low-rank steps only in the dequant variants");
   static_assert(BN_ % 16 == 0 && BN_ >= 16 && BN_ <= 256, "MMA N");
   static constexpr int NCHUNK = (BN_ + 31) / 32;  // epilogue chunks of 32 columns (last may hold 16)
   static_assert(!B_MN || BN_ % 64 == 0, "MN-major B needs whole 64-wide chunks");
   static constexpr int A_BYTES = BM * BK * 2;  // 16 KB
   static constexpr int B_BYTES = BN * BK * 2;
-  // P slot: packed codes of one 128 x 64 weight tile, then the 128 decoded
-  // block constants c' of its (row, block) pairs; both by TMA.
-  static constexpr int PK_BYTES = 4096;
+  // P slot: the packed codes of KSUP consecutive 64-deep K blocks of the
+  // 128-row weight tile (128 contiguous bytes per weight row: forward;
+  // 64 bytes of 4 x 64 rows: backward), then their 4 x 128 decoded block
+  // constants c'; both by TMA, shared by KSUP consecutive MMA jobs.
+  static constexpr int KSUP = 4;
+  static constexpr int PK_BYTES = 4096 * KSUP;
   static constexpr int P_CP = PK_BYTES;
-  static constexpr int P_BYTES = P_CP + 512;
+  static constexpr int P_BYTES = P_CP + 512 * KSUP;
   static constexpr int OFF_B = 0;
   static constexpr int OFF_A = OFF_B + SB * B_BYTES;
   static constexpr int OFF_P = OFF_A + SA * A_BYTES;
@@ -95,8 +101,9 @@ struct GemmCfg {
   // b_full[SB] b_empty[SB] a_full[SA] a_empty[SA] p_full[SP] p_empty[SP]
   // tmem_full[2] tmem_empty[2] drain
   static constexpr int NBARS = 2 * SB + 2 * SA + 2 * SP + 5;
-  static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem base, abort flag, last-CTA flag
-  static constexpr int SMEM_BYTES = OFF_MISC + 16;
+  // misc: tmem base, abort flag, last-CTA flag (16 B), then the 16 NF4 levels
+  static constexpr int OFF_MISC = ((OFF_BAR + NBARS * 8) + 15) & ~15;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 64;
   static constexpr int WARPS = DEQ ? 7 + NPW_ : 6;
   static constexpr int THREADS = WARPS * 32;
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64
@@ -163,7 +170,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     }
     for (int s = 0; s < C::SP; ++s) {
       mbar_init(p_full(s), 1);
-      mbar_init(p_empty(s), 4);
+      mbar_init(p_empty(s), 4 * C::KSUP);  // 4 warps per sub-job
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tmem_full(a), 1);
@@ -173,6 +180,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     *s_abort = 0;
     fence_barrier_init();
   }
+  if (threadIdx.x < 16) reinterpret_cast<float *>(smem + C::OFF_MISC + 16)[threadIdx.x] = args.nf4[threadIdx.x];
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&args.tm_b);
     if (!C::DEQ) tma_prefetch_desc(&args.tm_a);
@@ -263,7 +271,16 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     __syncwarp();
   } else if (warp == 5) {
     // ------------------------------------------------------ MMA issue --
+    // One thread issues every MMA of the CTA, so this loop is kept lean: the
+    // fixed bits of both descriptor layouts and both instruction descriptors
+    // are formed once, and each MMA only adds its K offset to the start
+    // address field.
     if (lane == 0) {
+      constexpr uint64_t DK = smem_desc_const(16, 1024);    // K-major, 128B swizzle
+      constexpr uint64_t DM = smem_desc_const(8192, 1024);  // MN-major, 128B swizzle
+      constexpr uint32_t ID_MAIN = make_idesc_bf16(128, C::BN, C::A_MN ? 1 : 0, C::B_MN ? 1 : 0);
+      constexpr uint32_t ID_LORA = make_idesc_bf16(128, C::BN, C::L2 == L2_A_MN ? 1 : 0, 0);
+      const uint32_t a_base = sbase + C::OFF_A, b_base = sbase + C::OFF_B;
       uint32_t job = 0, iter = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++iter) {
@@ -273,28 +290,31 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
         if (!mbar_wait(tmem_empty(acc), ((iter >> 1) & 1u) ^ 1u, s_abort)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::ACC_STRIDE;
+        int sb = job % C::SB, sa = C::DEQ ? (int)(job % C::SA) : sb;
+        uint32_t pb = (job / C::SB) & 1u, pa = (job / C::SA) & 1u;
         for (int jj = 0; jj < njobs; ++jj, ++job) {
-          const int sb = job % C::SB;
-          const int sa = C::DEQ ? (int)(job % C::SA) : sb;
-          if (!mbar_wait(b_full(sb), (job / C::SB) & 1u, s_abort)) { ok = false; break; }
-          if (C::DEQ && !mbar_wait(a_full(sa), (job / C::SA) & 1u, s_abort)) { ok = false; break; }
+          if (!mbar_try_wait(b_full(sb), pb) && !mbar_wait(b_full(sb), pb, s_abort)) { ok = false; break; }
+          if (C::DEQ && !mbar_try_wait(a_full(sa), pa) && !mbar_wait(a_full(sa), pa, s_abort)) { ok = false; break; }
           tc_fence_after();
           const bool main_job = jj < t.nmain;
           const bool a_mn = main_job ? C::A_MN : (C::L2 == L2_A_MN);
-          const bool b_mn = main_job ? C::B_MN : false;
-          const uint32_t idesc = make_idesc_bf16(128, C::BN, a_mn ? 1 : 0, b_mn ? 1 : 0);
-          const uint32_t a_addr = sbase + C::OFF_A + sa * C::A_BYTES;
-          const uint32_t b_addr = sbase + C::OFF_B + sb * C::B_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = a_mn ? smem_desc_sw128(a_addr + kk * 2048, 8192, 1024)
-                                     : smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-            const uint64_t bd = b_mn ? smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
-                                     : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-            tc_mma_ss(d_tmem, ad, bd, idesc, (jj > 0 || kk > 0) ? 1u : 0u);
-          }
+          const bool b_mn = main_job && C::B_MN;
+          const uint64_t ad = (a_mn ? DM : DK) | (((a_base + sa * C::A_BYTES) >> 4) & 0x3FFFu);
+          const uint64_t bd = (b_mn ? DM : DK) | (((b_base + sb * C::B_BYTES) >> 4) & 0x3FFFu);
+          const uint32_t astep = a_mn ? 2048u >> 4 : 32u >> 4, bstep = b_mn ? 2048u >> 4 : 32u >> 4;
+          const uint32_t idesc = main_job ? ID_MAIN : ID_LORA;
+          tc_mma_ss(d_tmem, ad, bd, idesc, jj > 0 ? 1u : 0u);
+          tc_mma_ss(d_tmem, ad + astep, bd + bstep, idesc, 1u);
+          tc_mma_ss(d_tmem, ad + 2 * astep, bd + 2 * bstep, idesc, 1u);
+          tc_mma_ss(d_tmem, ad + 3 * astep, bd + 3 * bstep, idesc, 1u);
           tc_commit(b_empty(sb));
           if (C::DEQ) tc_commit(a_empty(sa));
+          if (++sb == C::SB) { sb = 0; pb ^= 1u; }
+          if (C::DEQ) {
+            if (++sa == C::SA) { sa = 0; pa ^= 1u; }
+          } else {
+            sa = sb;
+          }
         }
         if (!ok) break;
         tc_commit(tmem_full(acc));
@@ -440,29 +460,29 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     // constants (c' is block-major, so they are one contiguous 512-byte row
     // for the forward and two 256-byte rows for the backward).
     if (lane == 0) {
-      uint32_t mj = 0;
+      uint32_t ms = 0;  // superjob counter (KSUP main jobs each, per tile)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         const TileCoord t = tile_coord(args, tile, row_tiles, col_tiles, C::BN);
-        for (int jj = 0; jj < t.nmain; ++jj, ++mj) {
-          const int sp = mj % C::SP;
-          if (!mbar_wait(p_empty(sp), ((mj / C::SP) & 1u) ^ 1u, s_abort)) { ok = false; break; }
-          const int kb = t.kb_begin + jj;
+        for (int u = 0; u * C::KSUP < t.nmain; ++u, ++ms) {
+          const int sp = ms % C::SP;
+          if (!mbar_wait(p_empty(sp), ((ms / C::SP) & 1u) ^ 1u, s_abort)) { ok = false; break; }
+          const int kb0 = t.kb_begin + u * C::KSUP;
           const uint32_t p_dst = sbase + C::OFF_P + sp * C::P_BYTES;
           mbar_arrive_expect_tx(p_full(sp), C::P_BYTES);
           if (C::ASRC == A_DEQ_K) {
-            tma_load_2d(p_dst, &args.tm_pk, p_full(sp), kb * 32, t.row0);
-            tma_load_2d(p_dst + C::P_CP, &args.tm_cp, p_full(sp), t.row0, kb);
+            tma_load_2d(p_dst, &args.tm_pk, p_full(sp), kb0 * 32, t.row0);
+            tma_load_2d(p_dst + C::P_CP, &args.tm_cp, p_full(sp), t.row0, kb0);
           } else {
-            tma_load_2d(p_dst, &args.tm_pk, p_full(sp), t.row0 / 2, kb * 64);
-            tma_load_2d(p_dst + C::P_CP, &args.tm_cp, p_full(sp), kb * 64, t.row0 / 64);
+            tma_load_2d(p_dst, &args.tm_pk, p_full(sp), t.row0 / 2, kb0 * 64);
+            tma_load_2d(p_dst + C::P_CP, &args.tm_cp, p_full(sp), kb0 * 64, t.row0 / 64);
           }
         }
       }
       // wait (bounded) for this thread's own copies still in flight
-      const uint32_t inflight = mj < (uint32_t)C::SP ? mj : (uint32_t)C::SP;
+      const uint32_t inflight = ms < (uint32_t)C::SP ? ms : (uint32_t)C::SP;
       for (uint32_t i = 0; i < inflight; ++i) {
-        const uint32_t jb = mj - 1 - i;
+        const uint32_t jb = ms - 1 - i;
         const unsigned long long t0 = globaltimer_ns();
         while (!mbar_try_wait(p_full(jb % C::SP), (jb / C::SP) & 1u)) {
           if (globaltimer_ns() - t0 > kWaitTimeoutNs) break;
@@ -475,36 +495,55 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     const int pw = warp - 7;
     const int group = pw >> 2;
     const int p = (pw & 3) * 32 + lane;  // 0..127: the tile row this thread decodes
-    float L[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) L[i] = args.nf4[i];
-    const uint32_t p_off = (C::ASRC == A_DEQ_K) ? p * 32 : (p & 63) * 64 + (p >> 6) * 32;
     const uint32_t a_off = (C::ASRC == A_DEQ_K) ? p * 128 : (p >> 6) * 8192 + (p & 63) * 128;
     const uint32_t swz = p & 7;
-    uint32_t job = 0, mj = 0;
+    uint32_t job = 0, ms = 0;  // ms: superjob counter at the start of the tile
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const TileCoord t = tile_coord(args, tile, row_tiles, col_tiles, C::BN);
       const int njobs = t.nmain + t.nlora;
+      const int nsup = (t.nmain + C::KSUP - 1) / C::KSUP;
       for (int jj = 0; jj < njobs; ++jj, ++job) {
         const bool main_job = jj < t.nmain;
-        const uint32_t my_mj = mj;
-        if (main_job) ++mj;
         if ((int)(job % C::NGROUPS) != group) continue;
         const int sa = job % C::SA;
         if (!warp_wait_all(a_empty(sa), ((job / C::SA) & 1u) ^ 1u, s_abort)) { ok = false; break; }
         if (main_job) {
-          const int sp = my_mj % C::SP;
-          if (!warp_wait_all(p_full(sp), (my_mj / C::SP) & 1u, s_abort)) { ok = false; break; }
+          const uint32_t my_ms = ms + jj / C::KSUP;
+          const int sub = jj % C::KSUP;
+          const int sp = my_ms % C::SP;
+          if (!warp_wait_all(p_full(sp), (my_ms / C::SP) & 1u, s_abort)) { ok = false; break; }
           const uint8_t *pslot = smem + C::OFF_P + sp * C::P_BYTES;
-          const float cp = reinterpret_cast<const float *>(pslot + C::PK_BYTES)[p];
+          uint32_t p_off, c_idx;
+          if (C::ASRC == A_DEQ_K) {  // [128 rows][KSUP x 32 B], c' [KSUP][128]
+            p_off = p * (32 * C::KSUP) + sub * 32;
+            c_idx = sub * 128 + p;
+          } else {  // [KSUP x 64 rows][2 x 32 B], c' [2][KSUP x 64]
+            p_off = (sub * 64 + (p & 63)) * 64 + (p >> 6) * 32;
+            c_idx = (p >> 6) * (64 * C::KSUP) + sub * 64 + (p & 63);
+          }
+          const float cp = reinterpret_cast<const float *>(pslot + C::P_CP)[c_idx];
           const uint4 w0 = *reinterpret_cast<const uint4 *>(pslot + p_off);
           const uint4 w1 = *reinterpret_cast<const uint4 *>(pslot + p_off + 16);
           __syncwarp();
-          if (lane == 0) mbar_arrive(p_empty(sp));  // packed tile and c' consumed
+          if (lane == 0) {  // this sub-job's share of the slot is consumed
+            // a short last superjob releases the missing sub-jobs' shares too
+            const int nsub = t.nmain - (jj / C::KSUP) * C::KSUP;
+            const int extra = (jj == t.nmain - 1 && nsub < C::KSUP) ? C::KSUP - nsub : 0;
+            for (int e = 0; e <= extra; ++e) mbar_arrive(p_empty(sp));
+          }
           uint8_t *a_slot = smem + C::OFF_A + sa * C::A_BYTES;
           // out-of-range rows decode with c' = 0 -> zeros
           const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+          float L[16];  // NF4 levels, re-read each job (shared-memory broadcast) to spare registers
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 l4 = reinterpret_cast<const float4 *>(smem + C::OFF_MISC + 16)[i];
+            L[4 * i] = l4.x;
+            L[4 * i + 1] = l4.y;
+            L[4 * i + 2] = l4.z;
+            L[4 * i + 3] = l4.w;
+          }
           const Nf4Planes P = make_planes(L, cp);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -517,6 +556,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
         __syncwarp();
         if (lane == 0) mbar_arrive(a_full(sa));
       }
+      ms += nsup;
     }
    }
   }

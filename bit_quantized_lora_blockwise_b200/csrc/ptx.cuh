@@ -247,6 +247,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo,
   return d;
 }
 
+// The address-independent bits of a 128B-swizzle descriptor (OR in the
+// start address >> 4 to complete it).
+__host__ __device__ constexpr uint64_t smem_desc_const(uint32_t lbo, uint32_t sbo) {
+  return (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) | (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) |
+         (1ull << 46) | (2ull << 61);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B, fp32 accumulator.
 __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, int a_mn_major,
                                                       int b_mn_major) {

@@ -254,10 +254,10 @@ struct SkinnyPlan {
   size_t part_bytes;  // none: the split-K partials are reduced in shared memory
 };
 
-// Split K over a cluster of 1, 2 or 4 CTAs per 128-row tile, in one wave.
+// Split K over a cluster of 1, 2, 4 or 8 CTAs per 128-row tile, in one wave.
 // (One CTA per SM; measured on B200: at most 15 eight-CTA clusters, 33
-// four-CTA clusters and 74 two-CTA clusters are co-resident, so clusters of 8
-// would spill into a second wave.)
+// four-CTA clusters and 74 two-CTA clusters are co-resident; clusters of 8
+// only for a few row tiles, e.g. the few-token X A.)
 SkinnyPlan plan_skinny(int64_t rows, int64_t kdim, int r, int sms) {
   SkinnyPlan p;
   p.rows = static_cast<int>(rows);
@@ -265,8 +265,10 @@ SkinnyPlan plan_skinny(int64_t rows, int64_t kdim, int r, int sms) {
   p.bn = rank_tile(r);
   const int row_tiles = static_cast<int>(cdiv(rows, 128));
   const int max_clusters4 = (sms * 33) / 148, max_clusters2 = (sms * 74) / 148;
+  const int max_clusters8 = (sms * 15) / 148;
   int splits = 1;
-  if (row_tiles <= max_clusters4 && 4 <= p.kblocks) splits = 4;
+  if (row_tiles <= max_clusters8 && row_tiles * 8 <= sms / 2 && 8 <= p.kblocks) splits = 8;
+  else if (row_tiles <= max_clusters4 && 4 <= p.kblocks) splits = 4;
   else if (row_tiles <= max_clusters2 && 2 <= p.kblocks) splits = 2;
   p.splits = splits;
   p.part_bytes = 0;
@@ -400,9 +402,12 @@ FusedPlan plan_fused(int64_t M, int64_t rows, int64_t kblocks, int sms) {
 
 template <int BN, int AS, int L2>
 qlora_status run_fused_bn(const GemmArgs &a, int sms, cudaStream_t st) {
-  // rings: activation tiles (SB), dequantized weight tiles (SA), packed codes + constants (SP)
-  constexpr int SB = BN > 64 ? 4 : 8, SA = BN > 64 ? 3 : 4, SP = 8;
-  return launch_gemm<GemmCfg<BN, AS, B_TMA_K, L2, SB, SA, SP, 8>>(a, sms, st);
+  // rings: activation tiles (SB), dequantized weight tiles (SA), packed codes + constants (SP);
+  // a few tokens leave the tensor core idle, so that variant runs 12 dequant warps
+  // (P slots hold 4 K blocks each; the few-token variant streams the packed
+  // weight from DRAM, so its P ring is deeper)
+  constexpr int SB = BN > 64 ? 4 : 8, SA = BN > 64 ? 3 : 6, SP = BN > 64 ? 2 : 4, NPW = BN > 64 ? 8 : 12;
+  return launch_gemm<GemmCfg<BN, AS, B_TMA_K, L2, SB, SA, SP, NPW>>(a, sms, st);
 }
 
 // Workspace carve-up: [tile counters][bf16 M x r][bf16 M x r (backward)][c'][fp32 partials]
@@ -604,8 +609,8 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   GemmArgs a;
   std::memset(&a, 0, sizeof a);
   if (!map_kmajor(&a.tm_b, X, K, M, fp.bn) ||
-      !make_map(&a.tm_pk, packed, MAP_U8, K / 2, N, K / 2, 32, 128, false) ||
-      !make_map(&a.tm_cp, cprime, MAP_F32, N, K / 64, N * 4, 128, 1, false) ||
+      !make_map(&a.tm_pk, packed, MAP_U8, K / 2, N, K / 2, 128, 128, false) ||
+      !make_map(&a.tm_cp, cprime, MAP_F32, N, K / 64, N * 4, 128, 4, false) ||
       !map_mnmajor(&a.tm_a2, B, N, r) || !map_kmajor(&a.tm_b2, xas, r, M, fp.bn))
     return QLORA_ERR_CUDA;
   a.w_kblocks = K / 64;
@@ -672,8 +677,8 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   GemmArgs a;
   std::memset(&a, 0, sizeof a);
   if (!map_kmajor(&a.tm_b, dY, N, M, fp.bn) ||
-      !make_map(&a.tm_pk, packed, MAP_U8, K / 2, N, K / 2, 64, 64, false) ||
-      !make_map(&a.tm_cp, cprime, MAP_F32, N, K / 64, N * 4, 64, 2, false) ||
+      !make_map(&a.tm_pk, packed, MAP_U8, K / 2, N, K / 2, 64, 256, false) ||
+      !make_map(&a.tm_cp, cprime, MAP_F32, N, K / 64, N * 4, 256, 2, false) ||
       !map_kmajor(&a.tm_a2, A, r, K, 128) || !map_kmajor(&a.tm_b2, gs, r, M, fp.bn))
     return QLORA_ERR_CUDA;
   a.w_kblocks = K / 64;
