@@ -9,13 +9,15 @@ alpha = 16, W ~ N(0, 0.02) with 0.1 % outliers at +-10 sigma; synthetic
 seeded inputs, generated on the device before timing.
 
 One step = for every linear: qlora_quantize_nf4, qlora_double_quant,
-qlora_dequant, qlora_linear_fwd (saving XA), qlora_linear_bwd — every row of
-the hot path once. Under torchrun each rank runs its own batch (weak
+qlora_dequant, qlora_linear_fwd (saving XA), qlora_linear_bwd, and a
+few-token qlora_linear_fwd (the first 16 tokens: the memory-bound small-M
+path) — every row of the hot path once. Under torchrun each rank runs its own batch (weak
 scaling, data parallel over tokens) and the adapter gradients dA, dB of
 every linear are summed across ranks with one NCCL all-reduce per step.
 
-`value` = fwd+bwd algorithmic FLOPs of all ranks / step time (max over
-ranks), sum over linears of 4MNK + 6Mr(N+K). The codec phases are reported
+`value` = algorithmic FLOPs of all ranks / step time (max over ranks), sum
+over linears of 4MNK + 6Mr(N+K) for the fwd+bwd plus 2mNK + 2mr(N+K) for
+the m = 16 token forward. The codec phases are reported
 in GB/s beside it. The reference arm (--impl reference) times the CPU
 oracle on a bounded sample of the same workload.
 """
@@ -41,6 +43,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 KERNEL_SOURCES = ["bit_quantized_lora_blockwise_b200/csrc/gemm.cuh",
                   "bit_quantized_lora_blockwise_b200/csrc/skinny.cuh",
                   "bit_quantized_lora_blockwise_b200/csrc/codec.cuh",
+                  "bit_quantized_lora_blockwise_b200/csrc/smallm.cuh",
                   "bit_quantized_lora_blockwise_b200/csrc/ptx.cuh"]
 
 
@@ -221,6 +224,9 @@ def run_reference(args, rank):
 
 
 # ------------------------------------------------------------------ native --
+SMALL_M = 16  # tokens of the few-token forward in each step
+
+
 class LinearState:
     def __init__(self, wl, li, M, device):
         import torch
@@ -243,9 +249,22 @@ class LinearState:
         self.dA = torch.empty((K, r), dtype=torch.bfloat16, **e)
         self.dB = torch.empty((r, N), dtype=torch.bfloat16, **e)
         self.ws_bytes = binding.workspace_bytes(M, N, K, r)
+        self.Xs = self.X[:SMALL_M].contiguous()
+        self.Ys = torch.empty((SMALL_M, N), dtype=torch.bfloat16, **e)
+        self.XAs = torch.empty((SMALL_M, r), dtype=torch.bfloat16, **e)
+
+    def smallm_flops(self):
+        return 2 * SMALL_M * self.N * self.K + 2 * SMALL_M * self.r * (self.N + self.K)
 
     def flops(self):
-        return linear_flops(self.M, self.N, self.K, self.r)
+        return linear_flops(self.M, self.N, self.K, self.r) + self.smallm_flops()
+
+    def smallm_bytes(self):
+        """Bytes the few-token forward must move: the packed weight with its
+        block constants, X, A, B, and the outputs Y, XA."""
+        N, K, r, m = self.N, self.K, self.r, SMALL_M
+        nb = N * K // 64
+        return N * K // 2 + nb + ((nb + 255) // 256) * 4 + 2 * (m * K + K * r + r * N + m * N + m * r)
 
     def codec_bytes(self):
         n = self.N * self.K
@@ -284,7 +303,7 @@ def run_native(args, rank, world, local_rank):
     # per step, per linear: events around the codec calls and the fused GEMMs
     def make_events():
         return [{k: (ev(), ev()) for k in ("quantize", "double_quant", "dequant", "fwd_gemm", "bwd_gemm",
-                                            "fwd_call", "bwd_call")}
+                                            "fwd_call", "bwd_call", "smallm_fwd")}
                 for _ in range(nl)]
 
     def step(evs=None, trace=None):
@@ -304,6 +323,8 @@ def run_native(args, rank, world, local_rank):
                 binding.linear_bwd(L.packed, L.q, L.scale2, L.X, L.dY, L.A, L.B, L.alpha, L.N, L.K, XA=L.XA,
                                    dX=L.dX, dA=L.dA, dB=L.dB, workspace=ws)
                 binding.set_trace_events(None, None)
+                binding.linear_fwd(L.packed, L.q, L.scale2, L.Xs, L.A, L.B, L.alpha, L.N, L.K, Y=L.Ys,
+                                   XA_out=L.XAs, workspace=ws)
                 continue
             if e: e["quantize"][0].record()
             binding.quantize_nf4(L.W, packed=L.packed, absmax=L.absmax)
@@ -317,7 +338,10 @@ def run_native(args, rank, world, local_rank):
             if e: e["fwd_call"][1].record(); binding.set_trace_events(*e["bwd_gemm"]); e["bwd_call"][0].record()
             binding.linear_bwd(L.packed, L.q, L.scale2, L.X, L.dY, L.A, L.B, L.alpha, L.N, L.K, XA=L.XA,
                                dX=L.dX, dA=L.dA, dB=L.dB, workspace=ws)
-            if e: e["bwd_call"][1].record(); binding.set_trace_events(None, None)
+            if e: e["bwd_call"][1].record(); binding.set_trace_events(None, None); e["smallm_fwd"][0].record()
+            binding.linear_fwd(L.packed, L.q, L.scale2, L.Xs, L.A, L.B, L.alpha, L.N, L.K, Y=L.Ys,
+                               XA_out=L.XAs, workspace=ws)
+            if e: e["smallm_fwd"][1].record()
         if world > 1:
             # data parallel over tokens: sum the adapter gradients of all ranks
             allreduce_adapter_grads([t for L in layers for t in (L.dA, L.dB)])
@@ -369,7 +393,7 @@ def run_native(args, rank, world, local_rank):
 
     # per-phase device times (mean over the timed steps)
     phase = {k: [] for k in ("quantize", "double_quant", "dequant", "fwd_gemm", "bwd_gemm", "fwd_call",
-                             "bwd_call")}
+                             "bwd_call", "smallm_fwd")}
     for evs in evs_steps:
         for k in phase:
             phase[k].append(sum(evs[i][k][0].elapsed_time(evs[i][k][1]) for i in range(nl)))
@@ -387,6 +411,13 @@ def run_native(args, rank, world, local_rank):
     for k in ("fwd_gemm", "bwd_gemm"):
         tf = gemm_flops[k] / (phase_ms[k] * 1e-3) / 1e12
         phases[k] = {"ms": round(phase_ms[k], 4), "TFLOP/s": round(tf, 1), "frac_tensor": round(tf / tc, 3)}
+    # few-token forward: a whole qlora_linear_fwd call (X A product + weight stream)
+    sm_bytes = sum(L.smallm_bytes() for L in layers)
+    sm_gbs = sm_bytes / (phase_ms["smallm_fwd"] * 1e-3) / 1e9
+    phases["smallm_fwd"] = {"ms": round(phase_ms["smallm_fwd"], 4), "tokens": SMALL_M, "GB/s": round(sm_gbs, 1),
+                            "frac_hbm": round(sm_gbs / hbm, 3),
+                            "TFLOP/s": round(sum(L.smallm_flops() for L in layers) /
+                                             (phase_ms["smallm_fwd"] * 1e-3) / 1e12, 2)}
     # whole qlora_linear_fwd / _bwd calls (fused GEMM + constants pass + adapter GEMMs)
     for k in ("fwd_call", "bwd_call"):
         phases[k] = {"ms": round(phase_ms[k], 4), "outside_fused_gemm_ms":
@@ -452,7 +483,8 @@ def run_native(args, rank, world, local_rank):
                            "M": M, "r": wl.r, "alpha": wl.alpha, "per_rank_tokens": M,
                            "parallelism": f"dp{world}",
                            "l2": "inputs larger than L2 (405 MB of bf16 weights + 320 MB of activations per step)",
-                           "step": "per linear: quantize_nf4, double_quant, dequant, linear_fwd, linear_bwd"},
+                           "step": "per linear: quantize_nf4, double_quant, dequant, linear_fwd, linear_bwd, "
+                                   f"linear_fwd on the first {SMALL_M} tokens"},
                 "phases": phases, "roofline": roofline, "gpu_launches": launches,
                 "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "device_error": err}
         print(json.dumps(line), flush=True)

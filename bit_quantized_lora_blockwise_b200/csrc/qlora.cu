@@ -17,6 +17,7 @@
 #include "codec.cuh"
 #include "gemm.cuh"
 #include "skinny.cuh"
+#include "smallm.cuh"
 #include "ptx.cuh"
 
 using namespace qlora;
@@ -197,6 +198,21 @@ bool map_mnmajor(CUtensorMap *m, const void *p, int64_t inner, int64_t outer) {
   return make_map(m, p, MAP_BF16, inner, outer, inner * 2, 64, 64, true);
 }
 
+// X [M, K] bf16 viewed as {64, K/64, M} (k within a block, block, token):
+// box {64, 4, tokens} = four quantization blocks of K for every token row.
+bool map_x_blocks(CUtensorMap *map, const void *X, int64_t M, int64_t K, uint32_t tokens) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(K / 64), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[3] = {64, 4, tokens};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(X), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------- GEMM launcher --
 template <class C>
 qlora_status launch_gemm(const GemmArgs &args, int sms, cudaStream_t stream) {
@@ -329,7 +345,7 @@ struct OutSpec {
 
 qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a_outer, const void *bop,
                     int64_t b_inner, int64_t b_outer, int64_t rows, int64_t kdim, int r, const OutSpec &o,
-                    int sms, cudaStream_t st) {
+                    int sms, cudaStream_t st, unsigned int *zero_words = nullptr, int nzero = 0) {
   const SkinnyPlan p = plan_skinny(rows, kdim, r, sms);
   SkinnyArgs a;
   std::memset(&a, 0, sizeof a);
@@ -359,6 +375,8 @@ qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a
   a.cols = r;
   a.kblocks = p.kblocks;
   a.splits = p.splits;
+  a.zero_words = zero_words;
+  a.nzero = nzero;
   const int row_tiles = static_cast<int>(cdiv(rows, 128));
   switch (kind) {
     case SK_XA: return run_skinny<false, true>(a, p.bn, row_tiles, st);
@@ -410,6 +428,56 @@ qlora_status run_fused_bn(const GemmArgs &a, int sms, cudaStream_t st) {
   return launch_gemm<GemmCfg<BN, AS, B_TMA_K, L2, SB, SA, SP, NPW>>(a, sms, st);
 }
 
+// ---------------------------------------------------- few-token forward --
+// Used for M <= 16 tokens: bands of 256 rows x chunks of 256 K split evenly
+// over a persistent grid of one CTA per SM. The X A kernel launched just
+// before it (and overlapping it) holds `busy_sms` SMs; leaving those out
+// keeps every CTA of the stream starting at once.
+constexpr int kSmallmMaxTokens = 16;
+
+struct SmallmPlan {
+  int nt, grid, units, kc, bands;
+  size_t part_bytes;
+};
+
+SmallmPlan plan_smallm(int64_t M, int64_t N, int64_t K, int sms, int busy_sms) {
+  SmallmPlan p;
+  p.nt = static_cast<int>(cdiv(M, 8));
+  p.bands = static_cast<int>(cdiv(N, SmallmCfg<1>::BAND));
+  p.kc = static_cast<int>(cdiv(K, 256));
+  p.units = p.bands * p.kc;
+  const int avail = std::max(1, sms - busy_sms);
+  p.grid = std::min(p.units, avail);
+  // one partial slot per CTA: its piece of the band an earlier CTA started
+  p.part_bytes = align256(static_cast<size_t>(p.grid) * SmallmCfg<1>::WARPS * p.nt * 32 * 16);
+  return p;
+}
+
+int skinny_ctas(int64_t rows, int64_t kdim, int r, int sms) {
+  const SkinnyPlan sp = plan_skinny(rows, kdim, r, sms);
+  return static_cast<int>(cdiv(rows, 128)) * sp.splits;
+}
+
+template <int NT, bool V8>
+qlora_status run_smallm_nt(const SmallmArgs &a, int grid, cudaStream_t st) {
+  using C = SmallmCfg<NT>;
+  static std::once_flag once[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(once[dev], [&] {
+    attr_err = cudaFuncSetAttribute(smallm_kernel<NT, V8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return QLORA_ERR_CUDA;
+  return launch_pdl(smallm_kernel<NT, V8>, grid, C::THREADS, C::SMEM_BYTES, st, a);
+}
+
+qlora_status run_smallm(const SmallmArgs &a, const SmallmPlan &p, bool v8, cudaStream_t st) {
+  if (p.nt == 1) return v8 ? run_smallm_nt<1, true>(a, p.grid, st) : run_smallm_nt<1, false>(a, p.grid, st);
+  return v8 ? run_smallm_nt<2, true>(a, p.grid, st) : run_smallm_nt<2, false>(a, p.grid, st);
+}
+
 // Workspace carve-up: [tile counters][bf16 M x r][bf16 M x r (backward)][c'][fp32 partials]
 struct WsLayout {
   size_t counters, mr, cprime, part, total;
@@ -424,6 +492,7 @@ WsLayout ws_layout(const Shape &s, int sms, bool backward) {
   w.cprime = cprime_bytes(s.N, s.K);
   if (!backward) {
     w.part = std::max(plan_skinny(s.M, s.K, s.r, sms).part_bytes, plan_fused(s.M, s.N, s.K / 64, sms).part_bytes);
+    if (s.M <= kSmallmMaxTokens) w.part = std::max(w.part, plan_smallm(s.M, s.N, s.K, sms, 0).part_bytes);
     w.total = w.counters + w.mr + w.cprime + w.part;
   } else {
     size_t part = plan_skinny(s.M, s.N, s.r, sms).part_bytes;               // G
@@ -592,6 +661,38 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   qlora_bf16 *xas = reinterpret_cast<qlora_bf16 *>(ws + w.counters);
   float *cprime = reinterpret_cast<float *>(ws + w.counters + w.mr);
   float *part = reinterpret_cast<float *>(ws + w.counters + w.mr + w.cprime);
+
+  if (M <= kSmallmMaxTokens) {
+    // Few tokens: XA (which also zeroes the band counters), then one pass over
+    // the packed weight that dequantizes in registers.
+    const SmallmPlan sp = plan_smallm(M, N, K, d.sms, skinny_ctas(M, K, r, d.sms));
+    OutSpec o{xas, r, scl, XA_out, r, 1.0f, false};
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs, counters, sp.bands);
+    if (st != QLORA_OK) return st;
+    SmallmArgs a;
+    std::memset(&a, 0, sizeof a);
+    if (!map_x_blocks(&a.tm_x, X, M, K, static_cast<uint32_t>(8 * sp.nt))) return QLORA_ERR_CUDA;
+    a.packed = packed;
+    a.q = q;
+    a.scale2 = scale2;
+    a.B = reinterpret_cast<const __nv_bfloat16 *>(B);
+    a.xas = reinterpret_cast<const __nv_bfloat16 *>(xas);
+    a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
+    a.part = part;
+    a.counters = counters;
+    a.N = N;
+    a.K = K;
+    a.M = static_cast<int>(M);
+    a.r = r;
+    a.kc = sp.kc;
+    a.units = sp.units;
+    a.tabs = make_tables(nf4, t8);
+    const bool v8 = (reinterpret_cast<uintptr_t>(packed) & 31u) == 0;
+    trace_begin(cs);
+    st = run_smallm(a, sp, v8, cs);
+    trace_end(cs);
+    return st;
+  }
 
   // 1) block constants c' for the GEMM producers (also zeroes the tile counters)
   st = launch_decode_constants(q, scale2, t8, N, K / 64, cprime, counters, w.ncounters, d.sms, cs);

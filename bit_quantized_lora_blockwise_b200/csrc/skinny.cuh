@@ -34,6 +34,8 @@ struct SkinnyArgs {
   int cols;     // r
   int kblocks;  // 64-deep K blocks in total
   int splits;   // CTAs per cluster (1, 2, 4 or 8), each taking a K range
+  unsigned int *zero_words;  // optional: words CTA 0 sets to zero (tile counters of the next kernel)
+  int nzero;
 };
 
 template <int BN_, bool A_MN_, bool B_MN_, int STAGES_>
@@ -104,6 +106,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_cons
   const uint32_t tmem_base = *s_tmem;
   grid_dep_wait();
   grid_dep_launch();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < args.nzero; i += blockDim.x) args.zero_words[i] = 0u;
 
   if (warp == 0) {
     if (lane == 0) {

@@ -147,3 +147,38 @@ def test_small_m_split_k(M):
     dX, dA, dB = L.bwd(XA)
     dXo, dAo, dBo = L.oracle_bwd()
     assert _rel(dX, dXo) <= TOL and _rel(dA, dAo) <= TOL and _rel(dB, dBo) <= TOL
+
+
+@pytest.mark.parametrize("M,N,K,r", [
+    (16, 4096, 4096, 64),   # bands shared by two CTAs (stream-K pieces)
+    (1, 8192, 2048, 64),    # one token
+    (7, 2112, 1600, 16),    # half band at the end of N, one-block K chunk at the end of K
+    (12, 1024, 8192, 8),    # long K: many chunks per band
+])
+def test_few_token_forward_stream_k(M, N, K, r):
+    """Few tokens: the forward streams the packed weight once, dequantizing
+    in registers; bands split across CTAs are summed in a fixed order, so two
+    calls give the same bits."""
+    L = Layer(M, N, K, r, seed=300 + M + N + K, w_std=0.015, outl=0.001)
+    Y, XA = L.fwd()
+    Y2, XA2 = L.fwd()
+    torch.cuda.synchronize()
+    assert binding.device_error() == 0
+    Yo, XAo = L.oracle_fwd()
+    assert _rel(Y, Yo) <= TOL
+    assert _rel(XA, XAo) <= TOL
+    assert torch.equal(Y, Y2) and torch.equal(XA, XA2)
+
+
+def test_few_token_one_hot_rows_pin_register_dequant():
+    """B = 0 and one-hot rows of X: each forward row is exactly a column of
+    W', which pins the in-register dequantization of the few-token path."""
+    M, N, K, r = 16, 2112, 1600, 8
+    L = Layer(M, N, K, r, seed=77, outl=0.001, zero_B=True)
+    ks = (np.arange(M) * 97 + 13) % K
+    X = torch.zeros((M, K), dtype=torch.bfloat16)
+    X[np.arange(M), ks] = 1.0
+    L.X = X
+    Y, _ = L.fwd()
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_bits(Y), L.Wq_bits[:, ks].T)
