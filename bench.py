@@ -292,7 +292,8 @@ def run_native(args, rank, world, local_rank):
     keep = [n for n in args.linears.split(",") if n]
     layers = [LinearState(wl, i, M, dev) for i in range(len(wl.linears))
               if not keep or wl.linears[i].name in keep]
-    ws = torch.empty(max(l.ws_bytes for l in layers), dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(max(l.ws_bytes, binding.workspace_bytes(SMALL_M, l.N, l.K, l.r)) for l in layers),
+                     dtype=torch.uint8, device=dev)
     nl = len(layers)
 
     def ev():

@@ -140,18 +140,24 @@ __global__ void __launch_bounds__(256) quantize_nf4_kernel(const uint4 *__restri
   const int64_t nwords = nblocks * 8;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x * 2;
   // The loop runs per warp (base is warp-uniform) so the shuffles below
-  // always see all 32 lanes; lanes past the end compute on zeros.
-  for (int64_t base = (static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31u)) * 2;
-       base < nwords; base += stride) {
-    int64_t t[2];
-    uint4 v[2];
+  // always see all 32 lanes; lanes past the end compute on zeros. The next
+  // iteration's two 16-byte loads are issued before this one is encoded.
+  int64_t base = (static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31u)) * 2;
+  uint4 vn[2];
+  auto load = [&](int64_t b, uint4 (&v)[2]) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      t[h] = base + 32 * h + lane;
-      v[h] = t[h] < nwords ? __ldg(&W[t[h]]) : make_uint4(0u, 0u, 0u, 0u);
+      const int64_t t = b + 32 * h + lane;
+      v[h] = t < nwords ? __ldg(&W[t]) : make_uint4(0u, 0u, 0u, 0u);
     }
+  };
+  if (base < nwords) load(base, vn);
+  for (; base < nwords; base += stride) {
+    uint4 v[2] = {vn[0], vn[1]};
+    if (base + stride < nwords) load(base + stride, vn);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
+      const int64_t t = base + 32 * h + lane;
       const uint32_t wd[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
       float f[8];
 #pragma unroll
@@ -167,9 +173,9 @@ __global__ void __launch_bounds__(256) quantize_nf4_kernel(const uint4 *__restri
       m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
       m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
       const uint32_t word = encode8<BUCKET>(f, m, s_mid, mid7, s_bk);
-      if (t[h] < nwords) {
-        packed[t[h]] = word;
-        if (sub == 0) absmax[t[h] >> 3] = m;
+      if (t < nwords) {
+        packed[t] = word;
+        if (sub == 0) absmax[t >> 3] = m;
       }
     }
   }
@@ -300,16 +306,29 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint4 *__restrict__ 
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   uint4 *stage = s_stage[wid];
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * 8;
-  for (int64_t b0 = (static_cast<int64_t>(blockIdx.x) * 8 + wid) * 32; b0 < nblocks; b0 += nwarps * 32) {
-    const int64_t b = b0 + lane;
-    const bool valid = b < nblocks;
-    uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
-    float cp = 0.0f;
-    if (valid) {
-      w0 = __ldg(&packed[2 * b]);
-      w1 = __ldg(&packed[2 * b + 1]);
-      cp = __fmul_rn(s_t8[__ldg(&q[b])], __ldg(&scale2[b >> 8]));
+  // this lane's block of the next iteration is loaded before the current one
+  // is decoded
+  uint4 n0 = make_uint4(0u, 0u, 0u, 0u), n1 = n0;
+  uint32_t nq = 0u;
+  float ns = 0.0f;
+  auto load = [&](int64_t b) {
+    if (b < nblocks) {
+      n0 = __ldg(&packed[2 * b]);
+      n1 = __ldg(&packed[2 * b + 1]);
+      nq = __ldg(&q[b]);
+      ns = __ldg(&scale2[b >> 8]);
+    } else {
+      n0 = n1 = make_uint4(0u, 0u, 0u, 0u);
+      nq = 0u;
+      ns = 0.0f;
     }
+  };
+  int64_t b0 = (static_cast<int64_t>(blockIdx.x) * 8 + wid) * 32;
+  if (b0 < nblocks) load(b0 + lane);
+  for (; b0 < nblocks; b0 += nwarps * 32) {
+    const uint4 w0 = n0, w1 = n1;
+    const float cp = __fmul_rn(s_t8[nq], ns);
+    if (b0 + nwarps * 32 < nblocks) load(b0 + nwarps * 32 + lane);
     const Nf4Planes P = make_planes(L, cp);
     const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll

@@ -191,6 +191,11 @@ __device__ __forceinline__ uint4 ld_stream_16B(const void *p) {
   return v;
 }
 
+// Bring a global line into L2 ahead of its use (no register, no wait).
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // 16-byte shared-memory load.
 __device__ __forceinline__ uint4 lds_16B(uint32_t addr) {
   uint4 v;

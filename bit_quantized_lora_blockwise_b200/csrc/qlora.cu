@@ -142,6 +142,23 @@ qlora_status launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t sm
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// CTAs of `kernel` (block threads, static shared memory only) resident per
+// SM, asked of the runtime once per kernel and device.
+template <auto Kernel>
+int resident_per_sm(int block) {
+  static std::once_flag once[kMaxDevices];
+  static int cached[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::call_once(once[dev], [&] {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kernel, block, 0) != cudaSuccess || n < 1) n = 1;
+    cached[dev] = n;
+    cudaGetLastError();
+  });
+  return cached[dev];
+}
+
 int grid_for(int64_t work_items, int per_cta, int sms, int waves) {
   const int64_t want = cdiv(work_items, per_cta);
   const int64_t cap = static_cast<int64_t>(sms) * waves;
@@ -265,44 +282,80 @@ enum SkinnyKind { SK_XA, SK_G, SK_DA, SK_DB };
 
 int rank_tile(int r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
 
-struct SkinnyPlan {
-  int rows, kblocks, splits, bn;
-  size_t part_bytes;  // none: the split-K partials are reduced in shared memory
+// Ring depth per rank tile: 4 stages of 24 KB (r <= 64) or 3 of 32 KB
+// (r <= 128) keep two CTAs on an SM; r <= 256 uses 4 stages of 48 KB.
+constexpr int skinny_stages(int bn) { return bn == 64 ? 4 : (bn == 128 ? 3 : 4); }
+
+// One skinny-GEMM variant: its shared-memory opt-in and how many clusters
+// of 2, 4 and 8 CTAs can be resident at once (asked of the runtime once per
+// device).
+template <int BN, bool AMN, bool BMN>
+struct SkinnyVariant {
+  using C = SkinnyCfg<BN, AMN, BMN, skinny_stages(BN)>;
+  static qlora_status prepare(int (&max_clusters)[4]) {
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t err[kMaxDevices];
+    static int cached[kMaxDevices][4];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::call_once(once[dev], [&] {
+      err[dev] = cudaFuncSetAttribute(skinny_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+      cached[dev][0] = 0;
+      for (int l = 1; l <= 3; ++l) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(1u << l);
+        cfg.blockDim = dim3(C::THREADS);
+        cfg.dynamicSmemBytes = C::SMEM_BYTES;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = 1u << l;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (err[dev] != cudaSuccess ||
+            cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void *>(skinny_kernel<C>), &cfg) !=
+                cudaSuccess)
+          n = 0;
+        cached[dev][l] = n;
+      }
+      cudaGetLastError();  // an unsupported cluster size only means "not that one"
+    });
+    for (int l = 0; l < 4; ++l) max_clusters[l] = cached[dev][l];
+    return err[dev] == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  }
 };
 
-// Split K over a cluster of 1, 2, 4 or 8 CTAs per 128-row tile, in one wave.
-// (One CTA per SM; measured on B200: at most 15 eight-CTA clusters, 33
-// four-CTA clusters and 74 two-CTA clusters are co-resident; clusters of 8
-// only for a few row tiles, e.g. the few-token X A.)
-SkinnyPlan plan_skinny(int64_t rows, int64_t kdim, int r, int sms) {
-  SkinnyPlan p;
-  p.rows = static_cast<int>(rows);
-  p.kblocks = static_cast<int>(cdiv(kdim, 64));
-  p.bn = rank_tile(r);
+struct SkinnyPlan {
+  int rows, kblocks, splits, bn;
+};
+
+// Split K over a cluster of 2, 4 or 8 CTAs per 128-row tile: the largest
+// split whose clusters for all row tiles are resident at once (one wave),
+// else one CTA per tile.
+template <bool AMN, bool BMN>
+qlora_status plan_skinny_v(int64_t rows, int64_t kdim, int r, SkinnyPlan *p) {
+  p->rows = static_cast<int>(rows);
+  p->kblocks = static_cast<int>(cdiv(kdim, 64));
+  p->bn = rank_tile(r);
+  int maxc[4];
+  const qlora_status st = p->bn == 64    ? SkinnyVariant<64, AMN, BMN>::prepare(maxc)
+                          : p->bn == 128 ? SkinnyVariant<128, AMN, BMN>::prepare(maxc)
+                                         : SkinnyVariant<256, AMN, BMN>::prepare(maxc);
   const int row_tiles = static_cast<int>(cdiv(rows, 128));
-  const int max_clusters4 = (sms * 33) / 148, max_clusters2 = (sms * 74) / 148;
-  const int max_clusters8 = (sms * 15) / 148;
-  int splits = 1;
-  if (row_tiles <= max_clusters8 && row_tiles * 8 <= sms / 2 && 8 <= p.kblocks) splits = 8;
-  else if (row_tiles <= max_clusters4 && 4 <= p.kblocks) splits = 4;
-  else if (row_tiles <= max_clusters2 && 2 <= p.kblocks) splits = 2;
-  p.splits = splits;
-  p.part_bytes = 0;
-  return p;
+  p->splits = 1;
+  for (int l = 3; l >= 1; --l)
+    if ((1 << l) <= p->kblocks && row_tiles <= maxc[l]) {
+      p->splits = 1 << l;
+      break;
+    }
+  return st;
 }
 
 template <int BN, bool AMN, bool BMN>
 qlora_status run_skinny_bn(const SkinnyArgs &a, int row_tiles, cudaStream_t st) {
-  constexpr int S = BN == 64 ? 8 : (BN == 128 ? 6 : 4);
-  using C = SkinnyCfg<BN, AMN, BMN, S>;
-  static std::once_flag once[kMaxDevices];
-  int dev = 0;
-  cudaGetDevice(&dev);
-  cudaError_t attr_err = cudaSuccess;
-  std::call_once(once[dev], [&] {
-    attr_err = cudaFuncSetAttribute(skinny_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-  });
-  if (attr_err != cudaSuccess) return QLORA_ERR_CUDA;
+  using C = typename SkinnyVariant<BN, AMN, BMN>::C;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(row_tiles * a.splits);
   cfg.blockDim = dim3(C::THREADS);
@@ -345,8 +398,14 @@ struct OutSpec {
 
 qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a_outer, const void *bop,
                     int64_t b_inner, int64_t b_outer, int64_t rows, int64_t kdim, int r, const OutSpec &o,
-                    int sms, cudaStream_t st, unsigned int *zero_words = nullptr, int nzero = 0) {
-  const SkinnyPlan p = plan_skinny(rows, kdim, r, sms);
+                    int sms, cudaStream_t st, unsigned int *zero_words = nullptr, int nzero = 0,
+                    bool early = false) {
+  (void)sms;
+  SkinnyPlan p;
+  qlora_status pst = kind == SK_XA  ? plan_skinny_v<false, true>(rows, kdim, r, &p)
+                     : kind == SK_G ? plan_skinny_v<false, false>(rows, kdim, r, &p)
+                                    : plan_skinny_v<true, true>(rows, kdim, r, &p);
+  if (pst != QLORA_OK) return pst;
   SkinnyArgs a;
   std::memset(&a, 0, sizeof a);
   bool ok = true;
@@ -377,6 +436,7 @@ qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a
   a.splits = p.splits;
   a.zero_words = zero_words;
   a.nzero = nzero;
+  a.early = early ? 1 : 0;
   const int row_tiles = static_cast<int>(cdiv(rows, 128));
   switch (kind) {
     case SK_XA: return run_skinny<false, true>(a, p.bn, row_tiles, st);
@@ -453,9 +513,10 @@ SmallmPlan plan_smallm(int64_t M, int64_t N, int64_t K, int sms, int busy_sms) {
   return p;
 }
 
-int skinny_ctas(int64_t rows, int64_t kdim, int r, int sms) {
-  const SkinnyPlan sp = plan_skinny(rows, kdim, r, sms);
-  return static_cast<int>(cdiv(rows, 128)) * sp.splits;
+int skinny_ctas(int64_t rows, int64_t kdim, int r) {
+  SkinnyPlan p;
+  if (plan_skinny_v<false, true>(rows, kdim, r, &p) != QLORA_OK) return 8;
+  return static_cast<int>(cdiv(rows, 128)) * p.splits;
 }
 
 template <int NT, bool V8>
@@ -491,15 +552,12 @@ WsLayout ws_layout(const Shape &s, int sms, bool backward) {
   w.mr = align256(static_cast<size_t>(s.M) * s.r * 2);
   w.cprime = cprime_bytes(s.N, s.K);
   if (!backward) {
-    w.part = std::max(plan_skinny(s.M, s.K, s.r, sms).part_bytes, plan_fused(s.M, s.N, s.K / 64, sms).part_bytes);
-    if (s.M <= kSmallmMaxTokens) w.part = std::max(w.part, plan_smallm(s.M, s.N, s.K, sms, 0).part_bytes);
+    w.part = s.M <= kSmallmMaxTokens ? plan_smallm(s.M, s.N, s.K, sms, 0).part_bytes
+                                     : plan_fused(s.M, s.N, s.K / 64, sms).part_bytes;
     w.total = w.counters + w.mr + w.cprime + w.part;
   } else {
-    size_t part = plan_skinny(s.M, s.N, s.r, sms).part_bytes;               // G
-    part = std::max(part, plan_skinny(s.K, s.M, s.r, sms).part_bytes);       // dA
-    part = std::max(part, plan_skinny(s.N, s.M, s.r, sms).part_bytes);       // dB
-    part = std::max(part, plan_skinny(s.M, s.K, s.r, sms).part_bytes);       // XA recompute
-    part = std::max(part, plan_fused(s.M, s.K, s.N / 64, sms).part_bytes);   // dX split-K
+    // the skinny GEMMs reduce their split-K partials in shared memory
+    const size_t part = plan_fused(s.M, s.K, s.N / 64, sms).part_bytes;   // dX split-K
     w.part = part;
     w.total = w.counters + 2 * w.mr + w.cprime + w.part;
   }
@@ -598,10 +656,14 @@ qlora_status qlora_quantize_nf4(const qlora_bf16 *W, int64_t N, int64_t K, const
   DeviceInfo d;
   if ((st = device_info(&d)) != QLORA_OK) return st;
   const int64_t nblocks = N * (K / 64);
-  const int grid = grid_for(nblocks * 8, 512, d.sms, 8);
   BucketTable bt;
   const bool bucketed = build_buckets(nf4, &bt);
-  return launch_pdl(bucketed ? quantize_nf4_kernel<true> : quantize_nf4_kernel<false>, grid, 256, 0,
+  auto kernel = bucketed ? quantize_nf4_kernel<true> : quantize_nf4_kernel<false>;
+  // one resident wave (a grid-stride loop covers the rest)
+  const int grid = grid_for(nblocks * 8, 512, d.sms,
+                            bucketed ? resident_per_sm<quantize_nf4_kernel<true>>(256)
+                                     : resident_per_sm<quantize_nf4_kernel<false>>(256));
+  return launch_pdl(kernel, grid, 256, 0,
                     static_cast<cudaStream_t>(stream), reinterpret_cast<const uint4 *>(W), nblocks,
                     reinterpret_cast<uint32_t *>(packed), absmax, make_tables(nf4, nullptr), bt);
 }
@@ -631,7 +693,7 @@ qlora_status qlora_dequant(const uint8_t *packed, const uint8_t *q, const float 
   DeviceInfo d;
   if ((st = device_info(&d)) != QLORA_OK) return st;
   const int64_t nblocks = N * K / 64;
-  const int grid = grid_for(nblocks, 256, d.sms, 4);
+  const int grid = grid_for(nblocks, 256, d.sms, resident_per_sm<dequant_kernel>(256));
   return launch_pdl(dequant_kernel, grid, 256, 0, static_cast<cudaStream_t>(stream),
                     reinterpret_cast<const uint4 *>(packed), q, scale2, nblocks, reinterpret_cast<uint4 *>(W_out),
                     make_tables(nf4, t8));
@@ -665,7 +727,7 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   if (M <= kSmallmMaxTokens) {
     // Few tokens: XA (which also zeroes the band counters), then one pass over
     // the packed weight that dequantizes in registers.
-    const SmallmPlan sp = plan_smallm(M, N, K, d.sms, skinny_ctas(M, K, r, d.sms));
+    const SmallmPlan sp = plan_smallm(M, N, K, d.sms, skinny_ctas(M, K, r));
     OutSpec o{xas, r, scl, XA_out, r, 1.0f, false};
     st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs, counters, sp.bands);
     if (st != QLORA_OK) return st;
@@ -701,7 +763,8 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   // 2) XA = X A -> XA_out = bf16(XA) (if wanted), xas = bf16(s XA)
   {
     OutSpec o{xas, r, scl, XA_out, r, 1.0f, false};
-    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs);
+    // X and A are inputs: the constants pass just before writes neither
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs, nullptr, 0, true);
     if (st != QLORA_OK) return st;
   }
 
@@ -769,7 +832,7 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   // 2) Gs = bf16(s * dY B^T)
   {
     OutSpec o{gs, r, scl, nullptr, 0, 0.0f, false};
-    st = skinny(SK_G, dY, N, M, B, N, r, M, N, r, o, d.sms, cs);
+    st = skinny(SK_G, dY, N, M, B, N, r, M, N, r, o, d.sms, cs, nullptr, 0, true);
     if (st != QLORA_OK) return st;
   }
 
@@ -806,7 +869,8 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   // 4) dA = X^T Gs   ([K, r])
   {
     OutSpec o{dA, r, 1.0f, nullptr, 0, 0.0f, false};
-    st = skinny(SK_DA, X, K, M, gs, r, M, K, M, r, o, d.sms, cs);
+    // Gs was written two kernels back (complete once the dX GEMM started)
+    st = skinny(SK_DA, X, K, M, gs, r, M, K, M, r, o, d.sms, cs, nullptr, 0, true);
     if (st != QLORA_OK) return st;
   }
 
@@ -814,12 +878,13 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   const qlora_bf16 *xa = XA;
   if (xa == nullptr) {
     OutSpec o{xa_ws, r, 1.0f, nullptr, 0, 0.0f, false};
-    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs);
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs, nullptr, 0, true);
     if (st != QLORA_OK) return st;
     xa = xa_ws;
   }
   OutSpec o{dB, N, scl, nullptr, 0, 0.0f, true};
-  return skinny(SK_DB, dY, N, M, xa, r, M, N, M, r, o, d.sms, cs);
+  // a recomputed XA is written by the kernel just before: wait for it first
+  return skinny(SK_DB, dY, N, M, xa, r, M, N, M, r, o, d.sms, cs, nullptr, 0, XA != nullptr);
 }
 
 }  // extern "C"

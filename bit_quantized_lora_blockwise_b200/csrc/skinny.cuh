@@ -36,6 +36,8 @@ struct SkinnyArgs {
   int splits;   // CTAs per cluster (1, 2, 4 or 8), each taking a K range
   unsigned int *zero_words;  // optional: words CTA 0 sets to zero (tile counters of the next kernel)
   int nzero;
+  int early;  // 1: neither operand is written by the kernel just before this one in the stream, so the
+              // first ring stages may be loaded before waiting for that kernel (programmatic launch)
 };
 
 template <int BN_, bool A_MN_, bool B_MN_, int STAGES_>
@@ -104,6 +106,30 @@ __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
+  // producer state: stages issued so far (the first ring's worth may go out
+  // ahead of the wait for the previous kernel, see SkinnyArgs::early)
+  int issued = 0;
+  auto issue = [&](int j) {
+    const int s = j % C::STAGES;
+    const int kb = kb_begin + j;
+    const uint32_t a_dst = sbase + C::OFF_A + s * C::A_BYTES;
+    const uint32_t b_dst = sbase + C::OFF_B + s * C::B_BYTES;
+    mbar_arrive_expect_tx(full_bar(s), C::TX);
+    if (C::A_MN) {
+      tma_load_2d(a_dst, &args.tm_a, full_bar(s), row0, kb * 64);
+      tma_load_2d(a_dst + 8192, &args.tm_a, full_bar(s), row0 + 64, kb * 64);
+    } else {
+      tma_load_2d(a_dst, &args.tm_a, full_bar(s), kb * 64, row0);
+    }
+    if (C::B_MN) {
+#pragma unroll
+      for (int c = 0; c < C::BN / 64; ++c) tma_load_2d(b_dst + c * 8192, &args.tm_b, full_bar(s), c * 64, kb * 64);
+    } else {
+      tma_load_2d(b_dst, &args.tm_b, full_bar(s), kb * 64, 0);
+    }
+  };
+  if (args.early && warp == 0 && lane == 0)
+    for (; issued < nk && issued < C::STAGES; ++issued) issue(issued);
   grid_dep_wait();
   grid_dep_launch();
   if (blockIdx.x == 0)
@@ -111,27 +137,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_cons
 
   if (warp == 0) {
     if (lane == 0) {
-      int issued = 0;
-      for (int j = 0; j < nk; ++j, ++issued) {
-        const int s = j % C::STAGES;
-        if (!mbar_wait(empty_bar(s), ((j / C::STAGES) & 1u) ^ 1u, s_abort)) break;
-        const int kb = kb_begin + j;
-        const uint32_t a_dst = sbase + C::OFF_A + s * C::A_BYTES;
-        const uint32_t b_dst = sbase + C::OFF_B + s * C::B_BYTES;
-        mbar_arrive_expect_tx(full_bar(s), C::TX);
-        if (C::A_MN) {
-          tma_load_2d(a_dst, &args.tm_a, full_bar(s), row0, kb * 64);
-          tma_load_2d(a_dst + 8192, &args.tm_a, full_bar(s), row0 + 64, kb * 64);
-        } else {
-          tma_load_2d(a_dst, &args.tm_a, full_bar(s), kb * 64, row0);
-        }
-        if (C::B_MN) {
-#pragma unroll
-          for (int c = 0; c < C::BN / 64; ++c)
-            tma_load_2d(b_dst + c * 8192, &args.tm_b, full_bar(s), c * 64, kb * 64);
-        } else {
-          tma_load_2d(b_dst, &args.tm_b, full_bar(s), kb * 64, 0);
-        }
+      for (; issued < nk; ++issued) {
+        const int s = issued % C::STAGES;
+        if (!mbar_wait(empty_bar(s), ((issued / C::STAGES) & 1u) ^ 1u, s_abort)) break;
+        issue(issued);
       }
       // wait (bounded) for this thread's copies still in flight
       const int inflight = issued < C::STAGES ? issued : C::STAGES;
@@ -218,13 +227,22 @@ __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_cons
       const int lrow = static_cast<int>(rank) * R + lr;
       const uint32_t off = static_cast<uint32_t>((lrow * C::PART_LD + c4 * 4) * 4);
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int sp = 0; sp < splits; ++sp) {
-        const float4 x = splits > 1 ? ld_cluster_f4(map_cluster(part_addr + off, sp))
-                                    : *reinterpret_cast<const float4 *>(smem + off);
-        v.x += x.x;
-        v.y += x.y;
-        v.z += x.z;
-        v.w += x.w;
+      if (splits > 1) {
+        // all peers' loads in flight at once, then summed in rank order
+        float4 x[8];
+#pragma unroll
+        for (int sp = 0; sp < 8; ++sp)
+          if (sp < splits) x[sp] = ld_cluster_f4(map_cluster(part_addr + off, sp));
+#pragma unroll
+        for (int sp = 0; sp < 8; ++sp)
+          if (sp < splits) {
+            v.x += x[sp].x;
+            v.y += x[sp].y;
+            v.z += x[sp].z;
+            v.w += x[sp].w;
+          }
+      } else {
+        v = *reinterpret_cast<const float4 *>(smem + off);
       }
       const int row = row0 + lrow;
       if (row >= args.rows) continue;

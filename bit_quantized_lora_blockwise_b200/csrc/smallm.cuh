@@ -188,6 +188,12 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
       ld_p += 128;
       ld_bi += 4;
     }
+    // the unit after this one: its packed rows into L2 now, so that its
+    // register loads (issued one unit later) hit L2
+    if (ld_row_ok && static_cast<int64_t>(ld_c) * 4 + t < kb_total) {
+      prefetch_l2(ld_p);
+      prefetch_l2(ld_p + 8 * row_bytes);
+    }
   };
 
   float acc[NT][4];
