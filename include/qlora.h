@@ -149,6 +149,9 @@ QLORA_API qlora_status qlora_dequant(const uint8_t *packed, const uint8_t *q, co
  * Accumulation in fp32; (X A) is rounded to bf16 (times s) before its
  * rank-r product. Requires M >= 1, N % 64 == 0, K % 64 == 0, N, K >= 64,
  * 1 <= r <= 256, r % 8 == 0, alpha finite, 16-byte aligned pointers.
+ * With M <= 16 tokens the product is memory-bound and runs as a single pass
+ * over the packed weight that dequantizes in registers; W' (the bf16 weight
+ * the MMAs see) is the same bit pattern on both paths.
  */
 QLORA_API qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const float *scale2,
                               const float nf4[16], const float t8[256],
@@ -222,7 +225,8 @@ QLORA_API qlora_status qlora_linear_fwd_noalloc(const uint8_t *packed, const uin
  * qlora_set_trace_events: when both are non-NULL, the next qlora_linear_fwd
  * and qlora_linear_bwd calls on this host thread record `start` (a
  * cudaEvent_t) on their stream just before their fused dequant-GEMM kernel
- * and `stop` just after it, so a caller can time that kernel alone with
+ * (for M <= 16 tokens: the register-dequant weight stream) and `stop` just
+ * after it, so a caller can time that kernel alone with
  * cudaEventElapsedTime. Pass NULL, NULL to stop. The events stay owned by the
  * caller.
  * qlora_launch_count: the number of kernels this library has launched in
