@@ -32,7 +32,7 @@ _STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_NULL", 2: "QLORA_ERR_SHAPE", 3: "QLORA_E
 EXPORTS = ("qlora_status_string", "qlora_abi_version", "qlora_nf4_levels", "qlora_dq_levels",
            "qlora_workspace_bytes", "qlora_quantize_nf4", "qlora_double_quant", "qlora_dequant",
            "qlora_linear_fwd", "qlora_linear_bwd", "qlora_device_error", "qlora_set_trace_events",
-           "qlora_launch_count", "qlora_linear_fwd_noalloc")
+           "qlora_launch_count", "qlora_linear_fwd_noalloc", "qlora_selftest_bounded_wait")
 
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -76,6 +76,8 @@ def load(path: str | None = None):
         lib.qlora_set_trace_events.argtypes = [P, P]
         lib.qlora_set_trace_events.restype = None
         lib.qlora_launch_count.restype = ctypes.c_uint64
+        lib.qlora_selftest_bounded_wait.argtypes = [P]
+        lib.qlora_selftest_bounded_wait.restype = I32
         for fn in ("qlora_quantize_nf4", "qlora_double_quant", "qlora_dequant", "qlora_linear_fwd",
                    "qlora_linear_bwd"):
             getattr(lib, fn).restype = I32
@@ -164,6 +166,14 @@ def workspace_bytes(M: int, N: int, K: int, r: int) -> int:
 
 def device_error(clear: bool = False) -> int:
     return int(load().qlora_device_error(1 if clear else 0))
+
+
+def selftest_bounded_wait():
+    """Launch the library's failure-path self-test on the current stream: a
+    kernel whose one wait never completes gives up after the bounded-wait
+    limit and sets bit 0 of the device error word (read it with
+    device_error)."""
+    _check(load().qlora_selftest_bounded_wait(_stream()), "qlora_selftest_bounded_wait")
 
 
 def launch_count() -> int:

@@ -351,30 +351,20 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint4 *__restrict__ 
 
 // ------------------------------------------------------------------------
 // Decoded block constants for the GEMMs, block-major: cprime[kb * N + n] =
-// t8[q_b] * scale2[b / 256] (fp32 product), b = n * KB + kb. One thread per
-// constant; consecutive threads take consecutive rows n of one kb, so the
-// stores are coalesced (the 8-bit codes are small and L2-resident). The
-// launch also zeroes `ncounters` split-K tile counters.
-__global__ void __launch_bounds__(256) decode_constants_kernel(const uint8_t *__restrict__ q,
-                                                               const float *__restrict__ scale2,
-                                                               int64_t N, int64_t KB,
-                                                               float *__restrict__ cprime,
-                                                               unsigned int *__restrict__ counters,
-                                                               int64_t ncounters, const CodecTables tabs) {
-  __shared__ float s_t8[256];
-  s_t8[threadIdx.x] = tabs.t8[threadIdx.x];
-  __syncthreads();
-  grid_dep_wait();
-  grid_dep_launch();
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (int64_t i = first; i < ncounters; i += stride) counters[i] = 0u;
+// t8[q_b] * scale2[b / 256] (fp32 product), b = n * KB + kb. Thread `first`
+// of `stride` threads takes every stride-th constant; consecutive threads
+// take consecutive rows n of one kb, so the stores are coalesced (the 8-bit
+// codes are small and L2-resident). t8 is a 256-entry table in shared memory.
+__device__ __forceinline__ void decode_constants_range(const uint8_t *__restrict__ q,
+                                                       const float *__restrict__ scale2, int64_t N, int64_t KB,
+                                                       float *__restrict__ cprime, const float *t8,
+                                                       int64_t first, int64_t stride) {
   const int64_t total = N * KB;
   for (int64_t t = first; t < total; t += stride) {
     const int64_t kb = t / N;
     const int64_t n = t - kb * N;
     const int64_t b = n * KB + kb;
-    cprime[t] = __fmul_rn(s_t8[__ldg(q + b)], __ldg(scale2 + (b >> 8)));
+    cprime[t] = __fmul_rn(t8[__ldg(q + b)], __ldg(scale2 + (b >> 8)));
   }
 }
 

@@ -250,16 +250,7 @@ qlora_status launch_gemm(const GemmArgs &args, int sms, cudaStream_t stream) {
 }
 
 // Block constants c' = t8[q] * S, block-major [K/64][N] fp32 (GEMM operand
-// staging; one small pass per linear call). The same launch zeroes the
-// split-K tile counters the call's GEMMs use (each GEMM leaves them zero).
-qlora_status launch_decode_constants(const uint8_t *q, const float *scale2, const float *t8, int64_t N,
-                                     int64_t KB, float *cprime, unsigned int *counters, int64_t ncounters,
-                                     int sms, cudaStream_t stream) {
-  const int grid = grid_for(N * KB, 256, sms, 8);
-  return launch_pdl(decode_constants_kernel, grid, 256, 0, stream, q, scale2, N, KB, cprime, counters,
-                    ncounters, make_tables(nullptr, t8));
-}
-
+// staging), decoded once per call by extra CTAs of the first skinny launch.
 size_t cprime_bytes(int64_t N, int64_t K) { return align256(static_cast<size_t>(N) * (K / 64) * 4); }
 
 // Layer sizes shared by forward and backward.
@@ -354,10 +345,10 @@ qlora_status plan_skinny_v(int64_t rows, int64_t kdim, int r, SkinnyPlan *p) {
 }
 
 template <int BN, bool AMN, bool BMN>
-qlora_status run_skinny_bn(const SkinnyArgs &a, int row_tiles, cudaStream_t st) {
+qlora_status run_skinny_bn(const SkinnyArgs &a, int grid, cudaStream_t st) {
   using C = typename SkinnyVariant<BN, AMN, BMN>::C;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(row_tiles * a.splits);
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(C::THREADS);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = st;
@@ -376,11 +367,20 @@ qlora_status run_skinny_bn(const SkinnyArgs &a, int row_tiles, cudaStream_t st) 
 }
 
 template <bool AMN, bool BMN>
-qlora_status run_skinny(const SkinnyArgs &a, int bn, int row_tiles, cudaStream_t st) {
-  if (bn == 64) return run_skinny_bn<64, AMN, BMN>(a, row_tiles, st);
-  if (bn == 128) return run_skinny_bn<128, AMN, BMN>(a, row_tiles, st);
-  return run_skinny_bn<256, AMN, BMN>(a, row_tiles, st);
+qlora_status run_skinny(const SkinnyArgs &a, int bn, int grid, cudaStream_t st) {
+  if (bn == 64) return run_skinny_bn<64, AMN, BMN>(a, grid, st);
+  if (bn == 128) return run_skinny_bn<128, AMN, BMN>(a, grid, st);
+  return run_skinny_bn<256, AMN, BMN>(a, grid, st);
 }
+
+// Constants pass folded into a skinny launch (extra CTAs, see SkinnyArgs).
+struct DecodeSpec {
+  const uint8_t *q;
+  const float *scale2;
+  float *cprime;
+  int64_t N, KB;
+  const float *t8;  // host table
+};
 
 // kind: SK_XA   Aop = X [M,K] (K-major),   Bop = A  [K,r] (MN-major), rows = M, kdim = K
 //       SK_G    Aop = dY [M,N] (K-major),  Bop = B  [r,N] (K-major),  rows = M, kdim = N
@@ -399,8 +399,7 @@ struct OutSpec {
 qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a_outer, const void *bop,
                     int64_t b_inner, int64_t b_outer, int64_t rows, int64_t kdim, int r, const OutSpec &o,
                     int sms, cudaStream_t st, unsigned int *zero_words = nullptr, int nzero = 0,
-                    bool early = false) {
-  (void)sms;
+                    bool early = false, const DecodeSpec *dc = nullptr) {
   SkinnyPlan p;
   qlora_status pst = kind == SK_XA  ? plan_skinny_v<false, true>(rows, kdim, r, &p)
                      : kind == SK_G ? plan_skinny_v<false, false>(rows, kdim, r, &p)
@@ -438,10 +437,27 @@ qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a
   a.nzero = nzero;
   a.early = early ? 1 : 0;
   const int row_tiles = static_cast<int>(cdiv(rows, 128));
+  a.gemm_ctas = row_tiles * p.splits;
+  int grid = a.gemm_ctas;
+  if (dc != nullptr) {
+    // about 8 constants per thread, on the slots the GEMM CTAs leave free
+    // (two resident CTAs per SM for r <= 128), in whole clusters
+    const int64_t want = cdiv(dc->N * dc->KB, 2048);
+    const int64_t free_slots = static_cast<int64_t>(p.bn <= 128 ? 2 : 1) * sms - a.gemm_ctas;
+    int64_t n = std::min(want, std::max<int64_t>(free_slots, p.splits));
+    n = cdiv(std::max<int64_t>(n, 1), p.splits) * p.splits;
+    grid += static_cast<int>(n);
+    a.dc_q = dc->q;
+    a.dc_scale2 = dc->scale2;
+    a.dc_cprime = dc->cprime;
+    a.dc_N = dc->N;
+    a.dc_KB = dc->KB;
+    std::memcpy(a.dc_t8, dc->t8, sizeof a.dc_t8);
+  }
   switch (kind) {
-    case SK_XA: return run_skinny<false, true>(a, p.bn, row_tiles, st);
-    case SK_G: return run_skinny<false, false>(a, p.bn, row_tiles, st);
-    default: return run_skinny<true, true>(a, p.bn, row_tiles, st);
+    case SK_XA: return run_skinny<false, true>(a, p.bn, grid, st);
+    case SK_G: return run_skinny<false, false>(a, p.bn, grid, st);
+    default: return run_skinny<true, true>(a, p.bn, grid, st);
   }
 }
 
@@ -572,6 +588,21 @@ void trace_begin(cudaStream_t s) {
 }
 void trace_end(cudaStream_t s) {
   if (t_trace_start && t_trace_stop) cudaEventRecord(t_trace_stop, s);
+}
+
+// Self-test of the failure path: one thread waits on an mbarrier phase that
+// nothing completes. mbar_wait gives up after kWaitTimeoutNs, raises the
+// abort flag and bit 0 of the device error word, and the kernel returns; no
+// trap, no fault, the context stays usable.
+__global__ void selftest_wait_kernel() {
+  __shared__ __align__(8) unsigned long long bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+    mbar_wait(smem_u32(&bar), 0u, &abort_flag);
+  }
 }
 
 qlora_status check_linear(const uint8_t *packed, const uint8_t *q, const float *scale2, const float *nf4,
@@ -756,19 +787,18 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
     return st;
   }
 
-  // 1) block constants c' for the GEMM producers (also zeroes the tile counters)
-  st = launch_decode_constants(q, scale2, t8, N, K / 64, cprime, counters, w.ncounters, d.sms, cs);
-  if (st != QLORA_OK) return st;
-
-  // 2) XA = X A -> XA_out = bf16(XA) (if wanted), xas = bf16(s XA)
+  // 1) XA = X A -> XA_out = bf16(XA) (if wanted), xas = bf16(s XA); the same
+  //    launch decodes the block constants c' for the GEMM producers and
+  //    zeroes the split-K tile counters. The first ring stages may go out
+  //    before the wait only when the launch before it is one of this call's.
   {
     OutSpec o{xas, r, scl, XA_out, r, 1.0f, false};
-    // X and A are inputs: the constants pass just before writes neither
-    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs, nullptr, 0, true);
+    const DecodeSpec dc{q, scale2, cprime, N, K / 64, t8};
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs, counters, static_cast<int>(w.ncounters), false, &dc);
     if (st != QLORA_OK) return st;
   }
 
-  // 3) Y^T[n, m] = W'[n, :] . X[m, :] + B^T[n, :] . xas[m, :]
+  // 2) Y^T[n, m] = W'[n, :] . X[m, :] + B^T[n, :] . xas[m, :]
   const FusedPlan fp = plan_fused(M, N, K / 64, d.sms);
   GemmArgs a;
   std::memset(&a, 0, sizeof a);
@@ -825,18 +855,16 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   float *cprime = reinterpret_cast<float *>(ws + w.counters + 2 * w.mr);
   float *part = reinterpret_cast<float *>(ws + w.counters + 2 * w.mr + w.cprime);
 
-  // 1) block constants c' (also zeroes the tile counters)
-  st = launch_decode_constants(q, scale2, t8, N, K / 64, cprime, counters, w.ncounters, d.sms, cs);
-  if (st != QLORA_OK) return st;
-
-  // 2) Gs = bf16(s * dY B^T)
+  // 1) Gs = bf16(s * dY B^T); the same launch decodes c' and zeroes the
+  //    tile counters (first kernel of the call: it waits before loading)
   {
     OutSpec o{gs, r, scl, nullptr, 0, 0.0f, false};
-    st = skinny(SK_G, dY, N, M, B, N, r, M, N, r, o, d.sms, cs, nullptr, 0, true);
+    const DecodeSpec dc{q, scale2, cprime, N, K / 64, t8};
+    st = skinny(SK_G, dY, N, M, B, N, r, M, N, r, o, d.sms, cs, counters, static_cast<int>(w.ncounters), false, &dc);
     if (st != QLORA_OK) return st;
   }
 
-  // 3) dX^T[k, m] = W'^T[k, :] . dY[m, :] + A[k, :] . Gs[m, :]
+  // 2) dX^T[k, m] = W'^T[k, :] . dY[m, :] + A[k, :] . Gs[m, :]
   const FusedPlan fp = plan_fused(M, K, N / 64, d.sms);
   GemmArgs a;
   std::memset(&a, 0, sizeof a);
@@ -866,7 +894,7 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   trace_end(cs);
   if (st != QLORA_OK) return st;
 
-  // 4) dA = X^T Gs   ([K, r])
+  // 3) dA = X^T Gs   ([K, r])
   {
     OutSpec o{dA, r, 1.0f, nullptr, 0, 0.0f, false};
     // Gs was written two kernels back (complete once the dX GEMM started)
@@ -874,7 +902,7 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
     if (st != QLORA_OK) return st;
   }
 
-  // 5) XA (saved or recomputed), then dB = s XA^T dY   ([r, N], from dB^T[n, j])
+  // 4) XA (saved or recomputed), then dB = s XA^T dY   ([r, N], from dB^T[n, j])
   const qlora_bf16 *xa = XA;
   if (xa == nullptr) {
     OutSpec o{xa_ws, r, 1.0f, nullptr, 0, 0.0f, false};
@@ -937,6 +965,15 @@ void qlora_set_trace_events(void *start, void *stop) {
 }
 
 uint64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+qlora_status qlora_selftest_bounded_wait(qlora_stream_t stream) {
+  qlora_status st;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != QLORA_OK) return st;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
 
 uint32_t qlora_device_error(int clear) {
   unsigned int v = 0;

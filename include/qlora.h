@@ -191,6 +191,16 @@ QLORA_API qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q,
 QLORA_API uint32_t qlora_device_error(int clear);
 
 /*
+ * Self-test of the failure path (no counterpart on the pages): launches one
+ * kernel whose single wait can never complete. After the bounded-wait limit
+ * (about 2 s) it gives up, sets bit 0 of the device error word and returns,
+ * exactly as a pipeline wait that ran out would; nothing traps or faults and
+ * the device stays usable. Asynchronous on `stream`; read the result with
+ * qlora_device_error.
+ */
+QLORA_API qlora_status qlora_selftest_bounded_wait(qlora_stream_t stream);
+
+/*
  * Forward without a caller workspace (the QLoRA pages have no counterpart:
  * this is an integration convenience, not part of the method).
  *
