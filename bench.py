@@ -249,7 +249,7 @@ class LinearState:
         self.dA = torch.empty((K, r), dtype=torch.bfloat16, **e)
         self.dB = torch.empty((r, N), dtype=torch.bfloat16, **e)
         self.ws_bytes = binding.workspace_bytes(M, N, K, r)
-        self.Xs = self.X[:SMALL_M].contiguous()
+        self.Xs = self.X[:SMALL_M]  # a view: rows are contiguous, and it follows X's contents
         self.Ys = torch.empty((SMALL_M, N), dtype=torch.bfloat16, **e)
         self.XAs = torch.empty((SMALL_M, r), dtype=torch.bfloat16, **e)
 
@@ -307,42 +307,45 @@ def run_native(args, rank, world, local_rank):
                                             "fwd_call", "bwd_call", "smallm_fwd")}
                 for _ in range(nl)]
 
-    def step(evs=None, trace=None):
-        """One pass of the hot path. evs: per-linear events around every call
-        (breakdown pass); trace: per-linear events around the fused GEMMs only
-        (recorded by the library on its stream; headline pass)."""
-        for i, L in enumerate(layers):
-            e = evs[i] if evs else None
-            if trace and not e:
-                binding.set_trace_events(*trace[i][0])
-                binding.quantize_nf4(L.W, packed=L.packed, absmax=L.absmax)
-                binding.double_quant(L.absmax, q=L.q, scale2=L.scale2)
-                binding.dequant(L.packed, L.q, L.scale2, L.N, L.K, out=L.Wq)
-                binding.linear_fwd(L.packed, L.q, L.scale2, L.X, L.A, L.B, L.alpha, L.N, L.K, Y=L.Y,
-                                   XA_out=L.XA, workspace=ws)
-                binding.set_trace_events(*trace[i][1])
-                binding.linear_bwd(L.packed, L.q, L.scale2, L.X, L.dY, L.A, L.B, L.alpha, L.N, L.K, XA=L.XA,
-                                   dX=L.dX, dA=L.dA, dB=L.dB, workspace=ws)
-                binding.set_trace_events(None, None)
-                binding.linear_fwd(L.packed, L.q, L.scale2, L.Xs, L.A, L.B, L.alpha, L.N, L.K, Y=L.Ys,
-                                   XA_out=L.XAs, workspace=ws)
-                continue
-            if e: e["quantize"][0].record()
+    def linear_step(L, e=None, tr=None):
+        """One linear's share of the step. e: events around every call
+        (breakdown pass); tr: events around the fused GEMMs only, recorded by
+        the library on its stream (headline pass)."""
+        if tr is not None and e is None:
+            binding.set_trace_events(*tr[0])
             binding.quantize_nf4(L.W, packed=L.packed, absmax=L.absmax)
-            if e: e["quantize"][1].record(); e["double_quant"][0].record()
             binding.double_quant(L.absmax, q=L.q, scale2=L.scale2)
-            if e: e["double_quant"][1].record(); e["dequant"][0].record()
             binding.dequant(L.packed, L.q, L.scale2, L.N, L.K, out=L.Wq)
-            if e: e["dequant"][1].record(); binding.set_trace_events(*e["fwd_gemm"]); e["fwd_call"][0].record()
             binding.linear_fwd(L.packed, L.q, L.scale2, L.X, L.A, L.B, L.alpha, L.N, L.K, Y=L.Y,
                                XA_out=L.XA, workspace=ws)
-            if e: e["fwd_call"][1].record(); binding.set_trace_events(*e["bwd_gemm"]); e["bwd_call"][0].record()
+            binding.set_trace_events(*tr[1])
             binding.linear_bwd(L.packed, L.q, L.scale2, L.X, L.dY, L.A, L.B, L.alpha, L.N, L.K, XA=L.XA,
                                dX=L.dX, dA=L.dA, dB=L.dB, workspace=ws)
-            if e: e["bwd_call"][1].record(); binding.set_trace_events(None, None); e["smallm_fwd"][0].record()
+            binding.set_trace_events(None, None)
             binding.linear_fwd(L.packed, L.q, L.scale2, L.Xs, L.A, L.B, L.alpha, L.N, L.K, Y=L.Ys,
                                XA_out=L.XAs, workspace=ws)
-            if e: e["smallm_fwd"][1].record()
+            return
+        if e: e["quantize"][0].record()
+        binding.quantize_nf4(L.W, packed=L.packed, absmax=L.absmax)
+        if e: e["quantize"][1].record(); e["double_quant"][0].record()
+        binding.double_quant(L.absmax, q=L.q, scale2=L.scale2)
+        if e: e["double_quant"][1].record(); e["dequant"][0].record()
+        binding.dequant(L.packed, L.q, L.scale2, L.N, L.K, out=L.Wq)
+        if e: e["dequant"][1].record(); binding.set_trace_events(*e["fwd_gemm"]); e["fwd_call"][0].record()
+        binding.linear_fwd(L.packed, L.q, L.scale2, L.X, L.A, L.B, L.alpha, L.N, L.K, Y=L.Y,
+                           XA_out=L.XA, workspace=ws)
+        if e: e["fwd_call"][1].record(); binding.set_trace_events(*e["bwd_gemm"]); e["bwd_call"][0].record()
+        binding.linear_bwd(L.packed, L.q, L.scale2, L.X, L.dY, L.A, L.B, L.alpha, L.N, L.K, XA=L.XA,
+                           dX=L.dX, dA=L.dA, dB=L.dB, workspace=ws)
+        if e: e["bwd_call"][1].record(); binding.set_trace_events(None, None); e["smallm_fwd"][0].record()
+        binding.linear_fwd(L.packed, L.q, L.scale2, L.Xs, L.A, L.B, L.alpha, L.N, L.K, Y=L.Ys,
+                           XA_out=L.XAs, workspace=ws)
+        if e: e["smallm_fwd"][1].record()
+
+    def step(evs=None, trace=None):
+        """One pass of the hot path over every linear."""
+        for i, L in enumerate(layers):
+            linear_step(L, evs[i] if evs else None, trace[i] if trace else None)
         if world > 1:
             # data parallel over tokens: sum the adapter gradients of all ranks
             allreduce_adapter_grads([t for L in layers for t in (L.dA, L.dB)])
@@ -444,14 +447,46 @@ def run_native(args, rank, world, local_rank):
                 for L in layers]
         d2h = sum(a.numel() * a.element_size() + b.numel() * b.element_size() for a, b in outs)
 
+        # Copies run on their own stream: linear i's inputs go up while the
+        # linears before it compute, and its dA, dB come back as soon as it
+        # is done. The compute of linear i waits for its copy; the next
+        # step's copy into linear i's buffers waits for this step's compute
+        # of linear i.
+        copy_stream = torch.cuda.Stream(device=dev)
+        done = [torch.cuda.Event() for _ in layers]
+        for d_ev in done:
+            d_ev.record()
+
         def e2e_step():
-            for L, h in zip(layers, host):
-                for k, t in h.items():
-                    getattr(L, k).copy_(t, non_blocking=True)
-            step()
-            for L, (a, b) in zip(layers, outs):
-                a.copy_(L.dA, non_blocking=True)
-                b.copy_(L.dB, non_blocking=True)
+            main = torch.cuda.current_stream()
+            start = torch.cuda.Event()
+            start.record(main)
+            arrived = []
+            with torch.cuda.stream(copy_stream):
+                copy_stream.wait_event(start)
+                for L, h, d_ev in zip(layers, host, done):
+                    copy_stream.wait_event(d_ev)
+                    for k, t in h.items():
+                        getattr(L, k).copy_(t, non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(copy_stream)
+                    arrived.append(ev)
+            for L, ev, d_ev in zip(layers, arrived, done):
+                main.wait_event(ev)
+                linear_step(L)
+                d_ev.record(main)
+            if world > 1:
+                allreduce_adapter_grads([t for L in layers for t in (L.dA, L.dB)])
+                for d_ev in done:
+                    d_ev.record(main)
+            with torch.cuda.stream(copy_stream):
+                for L, (a_h, b_h), d_ev in zip(layers, outs, done):
+                    copy_stream.wait_event(d_ev)
+                    a_h.copy_(L.dA, non_blocking=True)
+                    b_h.copy_(L.dB, non_blocking=True)
+                fin = torch.cuda.Event()
+                fin.record(copy_stream)
+            main.wait_event(fin)
 
         e2e_step()
         torch.cuda.synchronize()
