@@ -396,48 +396,69 @@ struct OutSpec {
   bool transpose;
 };
 
-qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a_outer, const void *bop,
-                    int64_t b_inner, int64_t b_outer, int64_t rows, int64_t kdim, int r, const OutSpec &o,
-                    int sms, cudaStream_t st, unsigned int *zero_words = nullptr, int nzero = 0,
-                    bool early = false, const DecodeSpec *dc = nullptr) {
+// One product's operands and output.
+struct SkinnyOperands {
+  const void *aop;
+  int64_t a_inner, a_outer;
+  const void *bop;
+  int64_t b_inner, b_outer;
+  int64_t rows, kdim;
+  OutSpec o;
+};
+
+// Launch one or two products of the same kind (same operand layouts and
+// reduction length) as one grid; optionally with the constants pass.
+qlora_status skinny_launch(SkinnyKind kind, const SkinnyOperands *ops, int nprob, int r, int sms,
+                           cudaStream_t st, unsigned int *zero_words, int nzero, bool early,
+                           const DecodeSpec *dc) {
+  int row_tiles[2] = {0, 0};
+  for (int i = 0; i < nprob; ++i) row_tiles[i] = static_cast<int>(cdiv(ops[i].rows, 128));
+  // the split is chosen for all row tiles of the launch together
   SkinnyPlan p;
-  qlora_status pst = kind == SK_XA  ? plan_skinny_v<false, true>(rows, kdim, r, &p)
-                     : kind == SK_G ? plan_skinny_v<false, false>(rows, kdim, r, &p)
-                                    : plan_skinny_v<true, true>(rows, kdim, r, &p);
+  const int64_t plan_rows = static_cast<int64_t>(row_tiles[0] + row_tiles[1]) * 128;
+  qlora_status pst = kind == SK_XA  ? plan_skinny_v<false, true>(plan_rows, ops[0].kdim, r, &p)
+                     : kind == SK_G ? plan_skinny_v<false, false>(plan_rows, ops[0].kdim, r, &p)
+                                    : plan_skinny_v<true, true>(plan_rows, ops[0].kdim, r, &p);
   if (pst != QLORA_OK) return pst;
   SkinnyArgs a;
   std::memset(&a, 0, sizeof a);
-  bool ok = true;
-  switch (kind) {
-    case SK_XA:
-      ok = map_kmajor(&a.tm_a, aop, a_inner, a_outer, 128) && map_mnmajor(&a.tm_b, bop, b_inner, b_outer);
-      break;
-    case SK_G:
-      ok = map_kmajor(&a.tm_a, aop, a_inner, a_outer, 128) &&
-           map_kmajor(&a.tm_b, bop, b_inner, b_outer, p.bn);
-      break;
-    case SK_DA:
-    case SK_DB:
-      ok = map_mnmajor(&a.tm_a, aop, a_inner, a_outer) && map_mnmajor(&a.tm_b, bop, b_inner, b_outer);
-      break;
+  for (int i = 0; i < nprob; ++i) {
+    const SkinnyOperands &op = ops[i];
+    SkinnyProblem &P = a.prob[i];
+    bool ok = true;
+    switch (kind) {
+      case SK_XA:
+        ok = map_kmajor(&P.tm_a, op.aop, op.a_inner, op.a_outer, 128) &&
+             map_mnmajor(&P.tm_b, op.bop, op.b_inner, op.b_outer);
+        break;
+      case SK_G:
+        ok = map_kmajor(&P.tm_a, op.aop, op.a_inner, op.a_outer, 128) &&
+             map_kmajor(&P.tm_b, op.bop, op.b_inner, op.b_outer, p.bn);
+        break;
+      case SK_DA:
+      case SK_DB:
+        ok = map_mnmajor(&P.tm_a, op.aop, op.a_inner, op.a_outer) &&
+             map_mnmajor(&P.tm_b, op.bop, op.b_inner, op.b_outer);
+        break;
+    }
+    if (!ok) return QLORA_ERR_CUDA;
+    P.out = op.o.out;
+    P.out_ld = op.o.ld;
+    P.out_scale = op.o.scale;
+    P.out2 = op.o.out2;
+    P.out2_ld = op.o.ld2;
+    P.out2_scale = op.o.scale2;
+    P.transpose = op.o.transpose ? 1 : 0;
+    P.rows = static_cast<int>(op.rows);
+    P.cols = r;
+    P.kblocks = static_cast<int>(cdiv(op.kdim, 64));
   }
-  if (!ok) return QLORA_ERR_CUDA;
-  a.out = o.out;
-  a.out_ld = o.ld;
-  a.out_scale = o.scale;
-  a.out2 = o.out2;
-  a.out2_ld = o.ld2;
-  a.out2_scale = o.scale2;
-  a.transpose = o.transpose ? 1 : 0;
-  a.rows = p.rows;
-  a.cols = r;
-  a.kblocks = p.kblocks;
   a.splits = p.splits;
+  a.prob0_ctas = row_tiles[0] * p.splits;
   a.zero_words = zero_words;
   a.nzero = nzero;
   a.early = early ? 1 : 0;
-  const int row_tiles = static_cast<int>(cdiv(rows, 128));
-  a.gemm_ctas = row_tiles * p.splits;
+  a.gemm_ctas = (row_tiles[0] + row_tiles[1]) * p.splits;
   int grid = a.gemm_ctas;
   if (dc != nullptr) {
     // about 8 constants per thread, on the slots the GEMM CTAs leave free
@@ -459,6 +480,14 @@ qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a
     case SK_G: return run_skinny<false, false>(a, p.bn, grid, st);
     default: return run_skinny<true, true>(a, p.bn, grid, st);
   }
+}
+
+qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a_outer, const void *bop,
+                    int64_t b_inner, int64_t b_outer, int64_t rows, int64_t kdim, int r, const OutSpec &o,
+                    int sms, cudaStream_t st, unsigned int *zero_words = nullptr, int nzero = 0,
+                    bool early = false, const DecodeSpec *dc = nullptr) {
+  const SkinnyOperands op{aop, a_inner, a_outer, bop, b_inner, b_outer, rows, kdim, o};
+  return skinny_launch(kind, &op, 1, r, sms, st, zero_words, nzero, early, dc);
 }
 
 // -------------------------------------------------------- fused GEMMs --
@@ -864,6 +893,16 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
     if (st != QLORA_OK) return st;
   }
 
+  // XA for dB, recomputed when the forward did not save it (X and A are
+  // inputs, Gs just before is not an operand)
+  const qlora_bf16 *xa = XA;
+  if (xa == nullptr) {
+    OutSpec o{xa_ws, r, 1.0f, nullptr, 0, 0.0f, false};
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs, nullptr, 0, true);
+    if (st != QLORA_OK) return st;
+    xa = xa_ws;
+  }
+
   // 2) dX^T[k, m] = W'^T[k, :] . dY[m, :] + A[k, :] . Gs[m, :]
   const FusedPlan fp = plan_fused(M, K, N / 64, d.sms);
   GemmArgs a;
@@ -894,25 +933,13 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   trace_end(cs);
   if (st != QLORA_OK) return st;
 
-  // 3) dA = X^T Gs   ([K, r])
-  {
-    OutSpec o{dA, r, 1.0f, nullptr, 0, 0.0f, false};
-    // Gs was written two kernels back (complete once the dX GEMM started)
-    st = skinny(SK_DA, X, K, M, gs, r, M, K, M, r, o, d.sms, cs, nullptr, 0, true);
-    if (st != QLORA_OK) return st;
-  }
-
-  // 4) XA (saved or recomputed), then dB = s XA^T dY   ([r, N], from dB^T[n, j])
-  const qlora_bf16 *xa = XA;
-  if (xa == nullptr) {
-    OutSpec o{xa_ws, r, 1.0f, nullptr, 0, 0.0f, false};
-    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs, nullptr, 0, true);
-    if (st != QLORA_OK) return st;
-    xa = xa_ws;
-  }
-  OutSpec o{dB, N, scl, nullptr, 0, 0.0f, true};
-  // a recomputed XA is written by the kernel just before: wait for it first
-  return skinny(SK_DB, dY, N, M, xa, r, M, N, M, r, o, d.sms, cs, nullptr, 0, XA != nullptr);
+  // 3) dA = X^T Gs ([K, r]) and dB = s XA^T dY ([r, N], from dB^T[n, j]) in one
+  //    launch; every operand was written at least two kernels back (complete
+  //    once the dX GEMM started), so the first stages load before the wait
+  const SkinnyOperands ops[2] = {
+      {X, K, M, gs, r, M, K, M, OutSpec{dA, r, 1.0f, nullptr, 0, 0.0f, false}},
+      {dY, N, M, xa, r, M, N, M, OutSpec{dB, N, scl, nullptr, 0, 0.0f, true}}};
+  return skinny_launch(SK_DA, ops, 2, r, d.sms, cs, nullptr, 0, true, nullptr);
 }
 
 }  // extern "C"

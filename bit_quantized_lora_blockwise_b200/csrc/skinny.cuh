@@ -23,7 +23,8 @@
 
 namespace qlora {
 
-struct SkinnyArgs {
+// One product of the launch.
+struct SkinnyProblem {
   CUtensorMap tm_a;  // A operand: K-major box {64, 128} or MN-major 64x64 chunks
   CUtensorMap tm_b;  // B operand: K-major box {64, BN} or MN-major 64x64 chunks
   void *out;         // bf16 [rows, cols] (ld out_ld) or transposed [cols, rows]
@@ -34,6 +35,13 @@ struct SkinnyArgs {
   int rows;     // extent of the 128-row MMA dimension
   int cols;     // r
   int kblocks;  // 64-deep K blocks in total
+};
+
+struct SkinnyArgs {
+  // Up to two independent products of the same operand layouts in one
+  // launch: CTAs [0, prob0_ctas) take prob[0], the next ones prob[1].
+  SkinnyProblem prob[2];
+  int prob0_ctas;
   int splits;   // CTAs per cluster (1, 2, 4 or 8), each taking a K range
   unsigned int *zero_words;  // optional: words CTA 0 sets to zero (tile counters of the next kernel)
   int nzero;
@@ -97,11 +105,14 @@ __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_cons
   volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
   const int splits = args.splits;
+  const int pi = static_cast<int>(blockIdx.x) >= args.prob0_ctas ? 1 : 0;
+  const SkinnyProblem &P = args.prob[pi];
+  const int local_block = static_cast<int>(blockIdx.x) - (pi ? args.prob0_ctas : 0);
   const uint32_t rank = splits > 1 ? cluster_ctarank() : 0u;
-  const int tile = blockIdx.x / splits;
+  const int tile = local_block / splits;
   const int row0 = tile * 128;
-  const int kb_begin = static_cast<int>((static_cast<int64_t>(rank) * args.kblocks) / splits);
-  const int kb_end = static_cast<int>((static_cast<int64_t>(rank + 1) * args.kblocks) / splits);
+  const int kb_begin = static_cast<int>((static_cast<int64_t>(rank) * P.kblocks) / splits);
+  const int kb_end = static_cast<int>((static_cast<int64_t>(rank + 1) * P.kblocks) / splits);
   const int nk = kb_end - kb_begin;
 
   if (threadIdx.x == 0) {
@@ -115,8 +126,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_cons
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&args.tm_a);
-    tma_prefetch_desc(&args.tm_b);
+    tma_prefetch_desc(&P.tm_a);
+    tma_prefetch_desc(&P.tm_b);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(s_tmem), C::TMEM_COLS);
@@ -136,16 +147,16 @@ __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_cons
     const uint32_t b_dst = sbase + C::OFF_B + s * C::B_BYTES;
     mbar_arrive_expect_tx(full_bar(s), C::TX);
     if (C::A_MN) {
-      tma_load_2d(a_dst, &args.tm_a, full_bar(s), row0, kb * 64);
-      tma_load_2d(a_dst + 8192, &args.tm_a, full_bar(s), row0 + 64, kb * 64);
+      tma_load_2d(a_dst, &P.tm_a, full_bar(s), row0, kb * 64);
+      tma_load_2d(a_dst + 8192, &P.tm_a, full_bar(s), row0 + 64, kb * 64);
     } else {
-      tma_load_2d(a_dst, &args.tm_a, full_bar(s), kb * 64, row0);
+      tma_load_2d(a_dst, &P.tm_a, full_bar(s), kb * 64, row0);
     }
     if (C::B_MN) {
 #pragma unroll
-      for (int c = 0; c < C::BN / 64; ++c) tma_load_2d(b_dst + c * 8192, &args.tm_b, full_bar(s), c * 64, kb * 64);
+      for (int c = 0; c < C::BN / 64; ++c) tma_load_2d(b_dst + c * 8192, &P.tm_b, full_bar(s), c * 64, kb * 64);
     } else {
-      tma_load_2d(b_dst, &args.tm_b, full_bar(s), kb * 64, 0);
+      tma_load_2d(b_dst, &P.tm_b, full_bar(s), kb * 64, 0);
     }
   };
   if (args.early && warp == 0 && lane == 0)
@@ -237,7 +248,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_cons
     const uint32_t part_addr = sbase;
     for (int u = threadIdx.x; u < units; u += C::THREADS) {
       int lr, c4;
-      if (args.transpose) {  // consecutive threads -> consecutive rows (coalesced transposed store)
+      if (P.transpose) {  // consecutive threads -> consecutive rows (coalesced transposed store)
         c4 = u / R;
         lr = u - c4 * R;
       } else {  // consecutive threads -> consecutive columns
@@ -265,18 +276,18 @@ __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_cons
         v = *reinterpret_cast<const float4 *>(smem + off);
       }
       const int row = row0 + lrow;
-      if (row >= args.rows) continue;
+      if (row >= P.rows) continue;
       const float vv[4] = {v.x, v.y, v.z, v.w};
       for (int o = 0; o < 2; ++o) {
-        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(o ? args.out2 : args.out);
+        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(o ? P.out2 : P.out);
         if (dst == nullptr) continue;
-        const float sc = o ? args.out2_scale : args.out_scale;
-        const int64_t ld = o ? args.out2_ld : args.out_ld;
+        const float sc = o ? P.out2_scale : P.out_scale;
+        const int64_t ld = o ? P.out2_ld : P.out_ld;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int col = c4 * 4 + e;
-          if (col >= args.cols) continue;
-          const int64_t idx = args.transpose ? static_cast<int64_t>(col) * ld + row
+          if (col >= P.cols) continue;
+          const int64_t idx = P.transpose ? static_cast<int64_t>(col) * ld + row
                                              : static_cast<int64_t>(row) * ld + col;
           dst[idx] = __float2bfloat16_rn(vv[e] * sc);
         }
