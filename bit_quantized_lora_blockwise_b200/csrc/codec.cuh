@@ -92,8 +92,11 @@ __device__ __forceinline__ uint32_t encode8(const float (&f)[8], float c, const 
       float x0, x1, y0, y1;
       f2_unpack(X, x0, x1);
       f2_unpack(Y, y0, y1);
-      const uint32_t j1 = min(__float_as_uint(y1) - __float_as_uint(kBucketMagic), 32u);
-      const uint32_t j0 = min(__float_as_uint(y0) - __float_as_uint(kBucketMagic), 32u);
+      // bits(y) = bits(1.5 * 2^23) + j with j in [0, 32] for |x| <= 1, and the
+      // magic's low six bits are zero, so j is the low six bits (any input,
+      // even a non-finite one, stays inside the padded 64-entry table)
+      const uint32_t j1 = __float_as_uint(y1) & 63u;
+      const uint32_t j0 = __float_as_uint(y0) & 63u;
       const float2 e1 = s_bk[j1], e0 = s_bk[j0];
       word = word * 16u + __float_as_uint(e1.y) + (x1 > e1.x ? 1u : 0u);
       word = word * 16u + __float_as_uint(e0.y) + (x0 > e0.x ? 1u : 0u);
@@ -127,10 +130,12 @@ __global__ void __launch_bounds__(256) quantize_nf4_kernel(const uint4 *__restri
                                                            float *__restrict__ absmax,
                                                            const CodecTables tabs, const BucketTable bt) {
   __shared__ float s_mid[16];
-  __shared__ float2 s_bk[33];
+  __shared__ float2 s_bk[64];  // 33 buckets, padded so that a 6-bit index is always in range
   if (threadIdx.x < 15)
     s_mid[threadIdx.x] = __fmul_rn(__fadd_rn(tabs.nf4[threadIdx.x], tabs.nf4[threadIdx.x + 1]), 0.5f);
-  if (threadIdx.x < 33) s_bk[threadIdx.x] = make_float2(bt.thr[threadIdx.x], __uint_as_float(bt.cand[threadIdx.x]));
+  if (threadIdx.x < 64)
+    s_bk[threadIdx.x] = threadIdx.x < 33 ? make_float2(bt.thr[threadIdx.x], __uint_as_float(bt.cand[threadIdx.x]))
+                                         : make_float2(2.0f, __uint_as_float(15u));
   __syncthreads();
   grid_dep_wait();
   grid_dep_launch();
