@@ -48,13 +48,15 @@ __device__ __forceinline__ float div_by_recip(float w, float c, float r) {
   return __fmaf_rn(e, r, q0);
 }
 
-// Bucketed encode. y = RN(16 x + 16 + 1.5 * 2^23) rounds 16 x + 16 to an
-// integer (the ulp at that magnitude is 1) and is monotone in x, so the
-// bucket j = bits(y) - bits(1.5 * 2^23) in [0, 32] is an interval of x
-// values (|x| <= 1). The host builds, for each bucket, the code of its first
-// x (cand) and the one midpoint that falls strictly inside it (thr; 2.0
-// when none), after checking that no bucket holds two; then
-// code(x) = cand[j] + (x > thr[j]) exactly. Tables whose midpoints are
+// Bucketed encode. y = RN(128 x + 128 + 1.5 * 2^23) rounds 128 x + 128 to an
+// integer t in [0, 256] (|x| <= 1; the ulp at that magnitude is 1) and is
+// monotone in x. Bucket j = t / 8 (width 1/16) is an interval of x values;
+// as the magic's low 22 bits are zero, bits(y) & 0x1F8 = 8 j is directly the
+// byte offset of the bucket's 8-byte entry, and a 64-entry table keeps any
+// input (even a non-finite one) in range. The host builds, for each bucket,
+// the code of its first x (cand) and the one midpoint that falls strictly
+// inside it (thr; 2.0 when none), after checking that no bucket holds two;
+// then code(x) = cand[j] + (x > thr[j]) exactly. Tables whose midpoints are
 // closer than a bucket width (1/16) use the binary search instead.
 struct BucketTable {
   float thr[33];
@@ -62,10 +64,19 @@ struct BucketTable {
 };
 constexpr float kBucketMagic = 12582912.0f;  // 1.5 * 2^23
 
+__device__ __forceinline__ float2 bucket_entry(const float2 *bk, float y) {
+  return *reinterpret_cast<const float2 *>(reinterpret_cast<const char *>(bk) + (__float_as_uint(y) & 0x1F8u));
+}
+
+// 0xFFFFFFFF when a > b, else 0 (false for NaN)
+__device__ __forceinline__ uint32_t set_gt_mask(float a, float b) {
+  uint32_t r;
+  asm("set.gt.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t nf4_code_bucket(float x, const float2 *bk) {
-  const float y = __fmaf_rn(x, 16.0f, 16.0f + kBucketMagic);
-  const uint32_t j = min(__float_as_uint(y) - __float_as_uint(kBucketMagic), 32u);  // |x| <= 1 keeps j <= 32
-  const float2 e = bk[j];
+  const float2 e = bucket_entry(bk, __fmaf_rn(x, 128.0f, 128.0f + kBucketMagic));
   return __float_as_uint(e.y) + (x > e.x ? 1u : 0u);
 }
 
@@ -79,8 +90,8 @@ __device__ __forceinline__ uint32_t encode8(const float (&f)[8], float c, const 
   if (BUCKET && c >= 0x1p-125f && c <= 0x1p125f) {
     const float r = __frcp_rn(c);
     const unsigned long long R = f2_pack(r, r), NC = f2_pack(-c, -c);
-    const unsigned long long S16 = f2_pack(16.0f, 16.0f);
-    const unsigned long long OFF = f2_pack(16.0f + kBucketMagic, 16.0f + kBucketMagic);
+    const unsigned long long S128 = f2_pack(128.0f, 128.0f);
+    const unsigned long long OFF = f2_pack(128.0f + kBucketMagic, 128.0f + kBucketMagic);
     uint32_t word = 0;
 #pragma unroll
     for (int i = 3; i >= 0; --i) {  // pairs (6,7), (4,5), ... so the word fills from the top nibble
@@ -88,18 +99,14 @@ __device__ __forceinline__ uint32_t encode8(const float (&f)[8], float c, const 
       const unsigned long long Q0 = f2_mul(W, R);       // RN(w r)
       const unsigned long long E = f2_fma(Q0, NC, W);   // w - q0 c, exact
       const unsigned long long X = f2_fma(E, R, Q0);    // RN(q0 + e r) = RN(w / c)
-      const unsigned long long Y = f2_fma(X, S16, OFF);  // bucket map
+      const unsigned long long Y = f2_fma(X, S128, OFF);  // bucket map
       float x0, x1, y0, y1;
       f2_unpack(X, x0, x1);
       f2_unpack(Y, y0, y1);
-      // bits(y) = bits(1.5 * 2^23) + j with j in [0, 32] for |x| <= 1, and the
-      // magic's low six bits are zero, so j is the low six bits (any input,
-      // even a non-finite one, stays inside the padded 64-entry table)
-      const uint32_t j1 = __float_as_uint(y1) & 63u;
-      const uint32_t j0 = __float_as_uint(y0) & 63u;
-      const float2 e1 = s_bk[j1], e0 = s_bk[j0];
-      word = word * 16u + __float_as_uint(e1.y) + (x1 > e1.x ? 1u : 0u);
-      word = word * 16u + __float_as_uint(e0.y) + (x0 > e0.x ? 1u : 0u);
+      const float2 e1 = bucket_entry(s_bk, y1), e0 = bucket_entry(s_bk, y0);
+      // code = cand + (x > thr): the compare gives an all-ones mask, subtracted
+      word = word * 16u + __float_as_uint(e1.y) - set_gt_mask(x1, e1.x);
+      word = word * 16u + __float_as_uint(e0.y) - set_gt_mask(x0, e0.x);
     }
     return word;
   }
@@ -130,12 +137,15 @@ __global__ void __launch_bounds__(256) quantize_nf4_kernel(const uint4 *__restri
                                                            float *__restrict__ absmax,
                                                            const CodecTables tabs, const BucketTable bt) {
   __shared__ float s_mid[16];
-  __shared__ float2 s_bk[64];  // 33 buckets, padded so that a 6-bit index is always in range
+  // 33 buckets, padded to 64 so that every offset bits(y) & 0x1F8 is in range;
+  // a NaN quotient (NaN weight, or inf / inf) lands in a padding entry and
+  // gets code 0, as no midpoint lies strictly below NaN
+  __shared__ float2 s_bk[64];
   if (threadIdx.x < 15)
     s_mid[threadIdx.x] = __fmul_rn(__fadd_rn(tabs.nf4[threadIdx.x], tabs.nf4[threadIdx.x + 1]), 0.5f);
   if (threadIdx.x < 64)
     s_bk[threadIdx.x] = threadIdx.x < 33 ? make_float2(bt.thr[threadIdx.x], __uint_as_float(bt.cand[threadIdx.x]))
-                                         : make_float2(2.0f, __uint_as_float(15u));
+                                         : make_float2(2.0f, __uint_as_float(0u));
   __syncthreads();
   grid_dep_wait();
   grid_dep_launch();
@@ -188,25 +198,47 @@ __global__ void __launch_bounds__(256) quantize_nf4_kernel(const uint4 *__restri
 
 // ------------------------------------------------------------------------
 // Double quantization: one warp per group of 256 constants, 8 per lane.
-// S = group max; q = number of fp32 midpoints of t8 strictly below c / S
-// (8-step binary search over the 255 midpoints); a group of zeros -> x = 0.
+// S = group max; q = number of fp32 midpoints of t8 strictly below
+// x = RN(c / S); a group of zeros gives x = 0.
+//
+// Bucketed search. With every midpoint m in [2^-100, 1] and no two closer
+// than 1/256, y = RN(256 x + 1.5 * 2^23) gives j = bits(y) - bits(1.5 * 2^23)
+// = RNE(256 x) in [0, 256] for x in [0, 1]: a monotone map onto 257 buckets
+// of width 1/256 with at most one midpoint strictly inside each. The host
+// fills cand[j] (midpoints below every x of bucket j) and thr[j] (the one
+// inside, 2.0 when none) and checks those conditions; then
+// q = cand[j] + (x > thr[j]). Any other j (x < -1/512 or NaN: no midpoint
+// lies strictly below such an x) is clamped to entry 257, which gives 0.
+// Tables that fail the check use an 8-step binary search over the 255
+// midpoints instead.
+struct DqBucketTable {
+  float thr[258];
+  unsigned int cand[258];
+};
+
+template <bool BUCKET>
 __global__ void __launch_bounds__(256) double_quant_kernel(const float *__restrict__ absmax,
                                                            int64_t nb, uint8_t *__restrict__ q,
                                                            float *__restrict__ scale2,
-                                                           const CodecTables tabs) {
-  __shared__ float s_mid[256];
-  if (threadIdx.x < 255)
-    s_mid[threadIdx.x] = __fmul_rn(__fadd_rn(tabs.t8[threadIdx.x], tabs.t8[threadIdx.x + 1]), 0.5f);
+                                                           const CodecTables tabs, const DqBucketTable bt) {
+  __shared__ float s_mid[BUCKET ? 1 : 256];
+  __shared__ float2 s_bk[BUCKET ? 258 : 1];
+  if constexpr (BUCKET) {
+    for (int i = threadIdx.x; i < 258; i += blockDim.x)
+      s_bk[i] = make_float2(bt.thr[i], __uint_as_float(bt.cand[i]));
+  } else {
+    if (threadIdx.x < 255)
+      s_mid[threadIdx.x] = __fmul_rn(__fadd_rn(tabs.t8[threadIdx.x], tabs.t8[threadIdx.x + 1]), 0.5f);
+  }
   __syncthreads();
   grid_dep_wait();
   grid_dep_launch();
   const int lane = threadIdx.x & 31;
   const int64_t ng = (nb + 255) / 256;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t g = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       g < ng; g += warps) {
+  // this lane's 8 constants of group g (zeros past the end)
+  auto load = [&](int64_t g, float (&c)[8]) {
     const int64_t base = g * 256 + lane * 8;
-    float c[8];
     if (base + 8 <= nb) {
       const float4 a = __ldg(reinterpret_cast<const float4 *>(absmax + base));
       const float4 b = __ldg(reinterpret_cast<const float4 *>(absmax + base + 4));
@@ -216,21 +248,46 @@ __global__ void __launch_bounds__(256) double_quant_kernel(const float *__restri
 #pragma unroll
       for (int i = 0; i < 8; ++i) c[i] = (base + i < nb) ? absmax[base + i] : 0.0f;
     }
+  };
+  int64_t g = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  float cn[8];
+  if (g < ng) load(g, cn);
+  for (; g < ng; g += warps) {
+    float c[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = cn[i];
+    if (g + warps < ng) load(g + warps, cn);  // the next group's loads go out first
     float s = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) s = fmaxf(s, c[i]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s = fmaxf(s, __shfl_xor_sync(0xFFFFFFFFu, s, o));
     uint32_t codes[8];
+    if constexpr (BUCKET) {
+      // RN(c / S) through the correctly rounded reciprocal (Markstein, as in
+      // encode8) when S is well inside the normal range, else the IEEE divide
+      const bool fast = s >= 0x1p-125f && s <= 0x1p125f;
+      const float r = fast ? __frcp_rn(s) : 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float x = (s == 0.0f) ? 0.0f : __fdiv_rn(c[i], s);
-      uint32_t k = 0;
+      for (int i = 0; i < 8; ++i) {
+        const float x = (s == 0.0f) ? 0.0f : (fast ? div_by_recip(c[i], s, r) : __fdiv_rn(c[i], s));
+        const float y = __fmaf_rn(x, 256.0f, kBucketMagic);
+        const uint32_t j = min(__float_as_uint(y) - __float_as_uint(kBucketMagic), 257u);
+        const float2 e = s_bk[j];
+        codes[i] = __float_as_uint(e.y) + (x > e.x ? 1u : 0u);
+      }
+    } else {
 #pragma unroll
-      for (uint32_t step = 128; step > 0; step >>= 1)
-        if (x > s_mid[k + step - 1]) k += step;
-      codes[i] = k;
+      for (int i = 0; i < 8; ++i) {
+        const float x = (s == 0.0f) ? 0.0f : __fdiv_rn(c[i], s);
+        uint32_t k = 0;
+#pragma unroll
+        for (uint32_t step = 128; step > 0; step >>= 1)
+          if (x > s_mid[k + step - 1]) k += step;
+        codes[i] = k;
+      }
     }
+    const int64_t base = g * 256 + lane * 8;
     if (base + 8 <= nb) {
       uint2 packed8;
       packed8.x = codes[0] | (codes[1] << 8) | (codes[2] << 16) | (codes[3] << 24);
@@ -356,20 +413,44 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint4 *__restrict__ 
 
 // ------------------------------------------------------------------------
 // Decoded block constants for the GEMMs, block-major: cprime[kb * N + n] =
-// t8[q_b] * scale2[b / 256] (fp32 product), b = n * KB + kb. Thread `first`
-// of `stride` threads takes every stride-th constant; consecutive threads
-// take consecutive rows n of one kb, so the stores are coalesced (the 8-bit
-// codes are small and L2-resident). t8 is a 256-entry table in shared memory.
+// t8[q_b] * scale2[b / 256] (fp32 product), b = n * KB + kb. One work item
+// is 16 consecutive blocks of one row n: its codes come in with one 16-byte
+// load (byte loads when KB is not a multiple of 16), its one or two
+// second-level scales with two loads, all issued before any is used, so a
+// thread waits for memory once per item rather than once per constant.
+// Consecutive threads take consecutive rows of the same 16 blocks, so every
+// one of the 16 stores is coalesced across the warp. Thread `first` of
+// `stride` threads takes every stride-th item. t8 is a 256-entry table in
+// shared memory.
 __device__ __forceinline__ void decode_constants_range(const uint8_t *__restrict__ q,
                                                        const float *__restrict__ scale2, int64_t N, int64_t KB,
                                                        float *__restrict__ cprime, const float *t8,
                                                        int64_t first, int64_t stride) {
-  const int64_t total = N * KB;
-  for (int64_t t = first; t < total; t += stride) {
-    const int64_t kb = t / N;
-    const int64_t n = t - kb * N;
-    const int64_t b = n * KB + kb;
-    cprime[t] = __fmul_rn(t8[__ldg(q + b)], __ldg(scale2 + (b >> 8)));
+  const int64_t items = N * ((KB + 15) / 16);
+  const bool vec = (KB & 15) == 0;  // every row's 16-block groups are 16-byte aligned
+  for (int64_t w = first; w < items; w += stride) {
+    const int64_t g = w / N;
+    const int64_t n = w - g * N;
+    const int64_t kb0 = g * 16;
+    const int nv = static_cast<int>(KB - kb0 < 16 ? KB - kb0 : 16);
+    const int64_t b0 = n * KB + kb0;
+    uint32_t code[16];
+    if (vec) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(q + b0));
+      const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 16; ++i) code[i] = (wd[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) code[i] = i < nv ? __ldg(q + b0 + i) : 0u;
+    }
+    const int64_t grp0 = b0 >> 8;  // 16 consecutive blocks span at most two 256-groups
+    const float s0 = __ldg(scale2 + grp0);
+    const float s1 = __ldg(scale2 + ((b0 + nv - 1) >> 8));
+    float *dst = cprime + kb0 * N + n;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < nv) dst[i * N] = __fmul_rn(t8[code[i]], ((b0 + i) >> 8) == grp0 ? s0 : s1);
   }
 }
 

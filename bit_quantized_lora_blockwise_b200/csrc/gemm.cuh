@@ -514,17 +514,25 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
           const int sp = my_ms % C::SP;
           if (!warp_wait_all(p_full(sp), (my_ms / C::SP) & 1u, s_abort)) { ok = false; break; }
           const uint8_t *pslot = smem + C::OFF_P + sp * C::P_BYTES;
-          uint32_t p_off, c_idx;
+          // The codes arrive swizzled (TMA 128-byte swizzle on 128-byte rows
+          // for the forward, 64-byte swizzle on 64-byte rows for the
+          // backward): 16-byte chunk c of a row sits at c ^ (row bits), so
+          // the 8 threads of each quarter-warp read 8 different bank groups.
+          uint32_t p_off0, p_off1, c_idx;
           if (C::ASRC == A_DEQ_K) {  // [128 rows][KSUP x 32 B], c' [KSUP][128]
-            p_off = p * (32 * C::KSUP) + sub * 32;
+            const uint32_t x = p & 7;
+            p_off0 = p * (32 * C::KSUP) + (((2 * sub) ^ x) << 4);
+            p_off1 = p * (32 * C::KSUP) + (((2 * sub + 1) ^ x) << 4);
             c_idx = sub * 128 + p;
           } else {  // [KSUP x 64 rows][2 x 32 B], c' [2][KSUP x 64]
-            p_off = (sub * 64 + (p & 63)) * 64 + (p >> 6) * 32;
+            const uint32_t row = sub * 64 + (p & 63), x = (row >> 1) & 3, c0 = 2 * (p >> 6);
+            p_off0 = row * 64 + ((c0 ^ x) << 4);
+            p_off1 = row * 64 + (((c0 + 1) ^ x) << 4);
             c_idx = (p >> 6) * (64 * C::KSUP) + sub * 64 + (p & 63);
           }
           const float cp = reinterpret_cast<const float *>(pslot + C::P_CP)[c_idx];
-          const uint4 w0 = *reinterpret_cast<const uint4 *>(pslot + p_off);
-          const uint4 w1 = *reinterpret_cast<const uint4 *>(pslot + p_off + 16);
+          const uint4 w0 = *reinterpret_cast<const uint4 *>(pslot + p_off0);
+          const uint4 w1 = *reinterpret_cast<const uint4 *>(pslot + p_off1);
           __syncwarp();
           if (lane == 0) {  // this sub-job's share of the slot is consumed
             // a short last superjob releases the missing sub-jobs' shares too

@@ -95,12 +95,12 @@ CodecTables make_tables(const float *nf4, const float *t8) {
 // Host float arithmetic here is IEEE binary32 with the same operation order
 // as the device (sum then halve; one fused multiply-add for the bucket).
 bool build_buckets(const float *L, BucketTable *bt) {
-  auto bucket = [](float x) {  // same arithmetic as nf4_code_bucket (|x| <= 1)
-    const float y = std::fmaf(x, 16.0f, 16.0f + kBucketMagic);
+  auto bucket = [](float x) {  // same arithmetic as nf4_code_bucket (|x| <= 1): (RNE(128 x + 128)) / 8
+    const float y = std::fmaf(x, 128.0f, 128.0f + kBucketMagic);
     uint32_t a, b;
     std::memcpy(&a, &y, 4);
     std::memcpy(&b, &kBucketMagic, 4);
-    return static_cast<int>(a - b);
+    return static_cast<int>((a - b) >> 3);
   };
   int jm[15], jp[15], inside[33] = {0};
   for (int j = 0; j < 33; ++j) bt->thr[j] = 2.0f;
@@ -116,6 +116,47 @@ bool build_buckets(const float *L, BucketTable *bt) {
   for (int j = 0; j < 33; ++j) {
     unsigned int c = 0;
     for (int i = 0; i < 15; ++i) c += (jp[i] < j || (jp[i] == j && jm[i] < j)) ? 1u : 0u;
+    bt->cand[j] = c;
+  }
+  return true;
+}
+
+// Bucket table of the double-quantization encode (see DqBucketTable):
+// false when a midpoint lies outside [2^-100, 1] or two share a bucket
+// (the binary search is used then). Same fp32 arithmetic as the device.
+bool build_dq_buckets(const float *t8, DqBucketTable *bt) {
+  auto bucket = [](float x) {  // RNE(256 x) for x in [0, 1], as the kernel computes it
+    const float y = std::fmaf(x, 256.0f, kBucketMagic);
+    uint32_t a, b;
+    std::memcpy(&a, &y, 4);
+    std::memcpy(&b, &kBucketMagic, 4);
+    return static_cast<int>(a - b);
+  };
+  int jm[255], jp[255], inside[257] = {0};
+  for (int j = 0; j < 258; ++j) {
+    bt->thr[j] = 2.0f;
+    bt->cand[j] = 0u;
+  }
+  for (int i = 0; i < 255; ++i) {
+    const float m = (t8[i] + t8[i + 1]) * 0.5f;
+    if (!(m >= 0x1p-100f && m <= 1.0f)) return false;
+    jm[i] = bucket(m);
+    jp[i] = bucket(std::nextafter(m, 2.0f));
+    if (jm[i] == jp[i]) {
+      if (inside[jm[i]]++) return false;
+      bt->thr[jm[i]] = m;
+    }
+  }
+  // midpoint i lies below every x of bucket j from j = jp[i] on when it is the
+  // last value of bucket jm[i] < jp[i], else from jp[i] + 1: count by prefix sum
+  unsigned int from[258] = {0};
+  for (int i = 0; i < 255; ++i) {
+    const int j0 = jm[i] < jp[i] ? jp[i] : jp[i] + 1;
+    ++from[j0 < 257 ? j0 : 257];
+  }
+  unsigned int c = 0;
+  for (int j = 0; j < 257; ++j) {
+    c += from[j];
     bt->cand[j] = c;
   }
   return true;
@@ -188,8 +229,10 @@ EncodeTiledFn encode_fn() {
 // {box_inner, box_outer}; out-of-range elements read as zero.
 enum MapType { MAP_BF16, MAP_U8, MAP_F32 };
 
+enum MapSwizzle { SW_NONE, SW_64B, SW_128B };
+
 bool make_map(CUtensorMap *map, const void *base, MapType type, uint64_t inner, uint64_t outer,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, MapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const CUtensorMapDataType dt = type == MAP_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -201,18 +244,20 @@ bool make_map(CUtensorMap *map, const void *base, MapType type, uint64_t inner, 
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(map, dt, 2,
                         const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        swz == SW_128B ? CU_TENSOR_MAP_SWIZZLE_128B
+                        : swz == SW_64B ? CU_TENSOR_MAP_SWIZZLE_64B
+                                        : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 // bf16 operand [outer rows, inner] read as K-major tiles (box {64, box_rows})
 bool map_kmajor(CUtensorMap *m, const void *p, int64_t inner, int64_t outer, uint32_t box_rows) {
-  return make_map(m, p, MAP_BF16, inner, outer, inner * 2, 64, box_rows, true);
+  return make_map(m, p, MAP_BF16, inner, outer, inner * 2, 64, box_rows, SW_128B);
 }
 // bf16 operand [outer rows, inner] read as MN-major 64x64 chunks
 bool map_mnmajor(CUtensorMap *m, const void *p, int64_t inner, int64_t outer) {
-  return make_map(m, p, MAP_BF16, inner, outer, inner * 2, 64, 64, true);
+  return make_map(m, p, MAP_BF16, inner, outer, inner * 2, 64, 64, SW_128B);
 }
 
 // X [M, K] bf16 viewed as {64, K/64, M} (k within a block, block, token):
@@ -461,9 +506,9 @@ qlora_status skinny_launch(SkinnyKind kind, const SkinnyOperands *ops, int nprob
   a.gemm_ctas = (row_tiles[0] + row_tiles[1]) * p.splits;
   int grid = a.gemm_ctas;
   if (dc != nullptr) {
-    // about 8 constants per thread, on the slots the GEMM CTAs leave free
-    // (two resident CTAs per SM for r <= 128), in whole clusters
-    const int64_t want = cdiv(dc->N * dc->KB, 2048);
+    // one item (16 constants of a row) per thread, on the slots the GEMM CTAs
+    // leave free (two resident CTAs per SM for r <= 128), in whole clusters
+    const int64_t want = cdiv(dc->N * cdiv(dc->KB, 16), 256);
     const int64_t free_slots = static_cast<int64_t>(p.bn <= 128 ? 2 : 1) * sms - a.gemm_ctas;
     int64_t n = std::min(want, std::max<int64_t>(free_slots, p.splits));
     n = cdiv(std::max<int64_t>(n, 1), p.splits) * p.splits;
@@ -737,10 +782,24 @@ qlora_status qlora_double_quant(const float *absmax, int64_t nb, const float t8[
   if (st != QLORA_OK) return st;
   DeviceInfo d;
   if ((st = device_info(&d)) != QLORA_OK) return st;
+  // the table is rebuilt only when t8 differs from this thread's last one
+  static DqBucketTable no_buckets;
+  thread_local float last_t8[256];
+  thread_local DqBucketTable bt;
+  thread_local bool have_last = false, bucketed = false;
+  if (!have_last || std::memcmp(last_t8, t8, sizeof last_t8) != 0) {
+    std::memcpy(last_t8, t8, sizeof last_t8);
+    bucketed = build_dq_buckets(t8, &bt);
+    have_last = true;
+  }
+  // one group per warp; at most two CTAs per SM (each fills its own table),
+  // warps with more groups load the next one ahead
   const int64_t ng = cdiv(nb, 256);
-  const int grid = grid_for(ng, 8, d.sms, 16);
-  return launch_pdl(double_quant_kernel, grid, 256, 0, static_cast<cudaStream_t>(stream), absmax, nb, q, scale2,
-                    make_tables(nullptr, t8));
+  const int grid = grid_for(ng, 8, d.sms, 2);
+  return bucketed ? launch_pdl(double_quant_kernel<true>, grid, 256, 0, static_cast<cudaStream_t>(stream), absmax,
+                               nb, q, scale2, make_tables(nullptr, t8), bt)
+                  : launch_pdl(double_quant_kernel<false>, grid, 256, 0, static_cast<cudaStream_t>(stream), absmax,
+                               nb, q, scale2, make_tables(nullptr, t8), no_buckets);
 }
 
 qlora_status qlora_dequant(const uint8_t *packed, const uint8_t *q, const float *scale2, int64_t N, int64_t K,
@@ -832,8 +891,8 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   GemmArgs a;
   std::memset(&a, 0, sizeof a);
   if (!map_kmajor(&a.tm_b, X, K, M, fp.bn) ||
-      !make_map(&a.tm_pk, packed, MAP_U8, K / 2, N, K / 2, 128, 128, false) ||
-      !make_map(&a.tm_cp, cprime, MAP_F32, N, K / 64, N * 4, 128, 4, false) ||
+      !make_map(&a.tm_pk, packed, MAP_U8, K / 2, N, K / 2, 128, 128, SW_128B) ||
+      !make_map(&a.tm_cp, cprime, MAP_F32, N, K / 64, N * 4, 128, 4, SW_NONE) ||
       !map_mnmajor(&a.tm_a2, B, N, r) || !map_kmajor(&a.tm_b2, xas, r, M, fp.bn))
     return QLORA_ERR_CUDA;
   a.w_kblocks = K / 64;
@@ -908,8 +967,8 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   GemmArgs a;
   std::memset(&a, 0, sizeof a);
   if (!map_kmajor(&a.tm_b, dY, N, M, fp.bn) ||
-      !make_map(&a.tm_pk, packed, MAP_U8, K / 2, N, K / 2, 64, 256, false) ||
-      !make_map(&a.tm_cp, cprime, MAP_F32, N, K / 64, N * 4, 256, 2, false) ||
+      !make_map(&a.tm_pk, packed, MAP_U8, K / 2, N, K / 2, 64, 256, SW_64B) ||
+      !make_map(&a.tm_cp, cprime, MAP_F32, N, K / 64, N * 4, 256, 2, SW_NONE) ||
       !map_kmajor(&a.tm_a2, A, r, K, 128) || !map_kmajor(&a.tm_b2, gs, r, M, fp.bn))
     return QLORA_ERR_CUDA;
   a.w_kblocks = K / 64;

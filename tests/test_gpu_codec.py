@@ -109,3 +109,78 @@ def test_custom_tables_are_honoured():
     assert np.array_equal(pk.cpu().numpy(), pk_o)
     assert np.array_equal(q.cpu().numpy(), q_o)
     assert np.array_equal(bf16_bits(wq).reshape(-1), wq_o)
+
+
+def _dq_boundary_constants(t8: np.ndarray, rng) -> np.ndarray:
+    """Groups of 256 constants whose ratios c / S sit on and next to every
+    fp32 midpoint of t8, for several group maxima S, plus degenerate groups."""
+    t8 = t8.astype(np.float32)
+    mids = ((t8[:-1] + t8[1:]) * np.float32(0.5)).astype(np.float32)
+    near = np.concatenate([mids, np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(2))])
+    groups = []
+    for S in (np.float32(1.0), np.float32(0.37), np.float32(3.0e-3), np.float32(2.5e4)):
+        vals = (near * S).astype(np.float32)
+        vals = np.concatenate([vals, np.nextafter(vals, np.float32(0)), np.nextafter(vals, np.float32(np.inf))])
+        vals = np.clip(vals, 0, S).astype(np.float32)
+        vals = vals[rng.permutation(vals.size)]
+        for i in range(0, vals.size, 255):
+            g = np.concatenate([[S], vals[i:i + 255]]).astype(np.float32)
+            groups.append(np.concatenate([g, np.zeros(256 - g.size, np.float32)]))
+    tiny = np.float32(2.0 ** -130)           # subnormal group maximum: IEEE divide path
+    groups.append(np.concatenate([[tiny], (rng.random(255) * tiny).astype(np.float32)]))
+    big = np.float32(2.0 ** 126)             # group maximum above the reciprocal range
+    groups.append(np.concatenate([[big], (rng.random(255) * big).astype(np.float32)]))
+    groups.append(np.zeros(256, np.float32))                                  # all zero
+    groups.append(np.concatenate([[np.float32(1.0)], -rng.random(255).astype(np.float32)]))  # negatives
+    odd = rng.random(256).astype(np.float32)
+    odd[3], odd[9], odd[17] = np.nan, -0.0, np.float32(1e-42)
+    groups.append(odd)
+    inf = rng.random(256).astype(np.float32)
+    inf[5] = np.inf
+    groups.append(inf)
+    return np.concatenate(groups).astype(np.float32)
+
+
+@pytest.mark.parametrize("table", ["default", "grid256", "shifted"])
+def test_double_quant_midpoint_boundaries(table):
+    """Every midpoint, its fp32 neighbours, several group scales, negative,
+    NaN, infinite, zero and subnormal constants: bit-exact against the
+    oracle for tables on the bucketed encode and the binary search."""
+    rng = np.random.default_rng(11)
+    if table == "default":
+        t8 = oracle.dq_levels()
+    elif table == "grid256":
+        # midpoints (k + 1/2) / 256 fall exactly on bucket edges
+        t8 = (np.arange(256, dtype=np.float64) / 256.0).astype(np.float32)
+    else:
+        t8 = (0.001 + np.arange(256, dtype=np.float64) * (0.999 / 255.0)).astype(np.float32)
+    am = _dq_boundary_constants(t8, rng)
+    am = np.concatenate([am, rng.random(77).astype(np.float32)])  # short last group
+    q_o, s2_o = oracle.double_quant(am, t8)
+    q, s2 = binding.double_quant(torch.from_numpy(am).cuda(), t8=t8)
+    torch.cuda.synchronize()
+    assert np.array_equal(s2.cpu().numpy().view(np.uint32), s2_o.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), q_o)
+    assert binding.device_error() == 0
+
+
+def test_quantize_nonfinite_weights():
+    """NaN and infinite weights: the block maximum ignores NaN, a NaN
+    quotient (NaN weight, or inf / inf) has no midpoint below it (code 0),
+    finite weights of a block with an infinite maximum quantize to zero."""
+    rng = np.random.default_rng(5)
+    K = 512
+    rows = []
+    for special in (0x7FC0, 0xFFC0, 0x7F80, 0xFF80):   # +NaN, -NaN, +inf, -inf
+        r = weight_bf16(1, K, 0.02, seed=int(special)).view(torch.int16).numpy().view(np.uint16).reshape(-1).copy()
+        idx = rng.choice(K, 9, replace=False)
+        r[idx] = special
+        rows.append(r)
+    bits = np.stack(rows)
+    pk_o, am_o = oracle.quantize_nf4(bits)
+    W = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+    pk, am = binding.quantize_nf4(W)
+    torch.cuda.synchronize()
+    assert np.array_equal(am.cpu().numpy().view(np.uint32), am_o.view(np.uint32)), "absmax"
+    assert np.array_equal(pk.cpu().numpy(), pk_o), "packed nibbles"
+    assert binding.device_error() == 0
