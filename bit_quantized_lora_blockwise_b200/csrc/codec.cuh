@@ -127,10 +127,12 @@ __device__ __forceinline__ uint32_t encode8(const float (&f)[8], float c, const 
   return word;
 }
 
-// One 64-weight block per 8 lanes; each lane encodes 8 consecutive weights
-// (one 16-byte load) into one 32-bit word of 8 nibbles. A warp takes 8
-// blocks per iteration (two independent 16-byte loads per lane in flight).
-template <bool BUCKET>
+// One 64-weight block per 4 lanes; each lane encodes 16 consecutive weights
+// (one 32-byte load, or two 16-byte loads when W is only 16-byte aligned)
+// into two 32-bit words of 8 nibbles. A warp takes 16 blocks per iteration
+// (two independent loads per lane in flight), and the next iteration's loads
+// are issued before this one is encoded.
+template <bool BUCKET, bool V8>
 __global__ void __launch_bounds__(256) quantize_nf4_kernel(const uint4 *__restrict__ W,
                                                            int64_t nblocks,
                                                            uint32_t *__restrict__ packed,
@@ -150,47 +152,61 @@ __global__ void __launch_bounds__(256) quantize_nf4_kernel(const uint4 *__restri
   grid_dep_wait();
   grid_dep_launch();
   const float mid7 = s_mid[7];
-  const uint32_t sub = threadIdx.x & 7u;
   const uint32_t lane = threadIdx.x & 31u;
-  const int64_t nwords = nblocks * 8;
+  const int64_t nunits = nblocks * 4;  // 32-byte units of 16 weights
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x * 2;
   // The loop runs per warp (base is warp-uniform) so the shuffles below
-  // always see all 32 lanes; lanes past the end compute on zeros. The next
-  // iteration's two 16-byte loads are issued before this one is encoded.
+  // always see all 32 lanes; lanes past the end compute on zeros.
   int64_t base = (static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31u)) * 2;
-  uint4 vn[2];
-  auto load = [&](int64_t b, uint4 (&v)[2]) {
+  uint32_t vn[2][8];
+  auto load = [&](int64_t b) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int64_t t = b + 32 * h + lane;
-      v[h] = t < nwords ? __ldg(&W[t]) : make_uint4(0u, 0u, 0u, 0u);
+      if (t < nunits) {
+        if (V8) {
+          ld_stream_32B(W + 2 * t, vn[h]);
+        } else {
+          const uint4 lo = __ldg(W + 2 * t), hi = __ldg(W + 2 * t + 1);
+          vn[h][0] = lo.x; vn[h][1] = lo.y; vn[h][2] = lo.z; vn[h][3] = lo.w;
+          vn[h][4] = hi.x; vn[h][5] = hi.y; vn[h][6] = hi.z; vn[h][7] = hi.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) vn[h][i] = 0u;
+      }
     }
   };
-  if (base < nwords) load(base, vn);
-  for (; base < nwords; base += stride) {
-    uint4 v[2] = {vn[0], vn[1]};
-    if (base + stride < nwords) load(base + stride, vn);
+  if (base < nunits) load(base);
+  for (; base < nunits; base += stride) {
+    uint32_t v[2][8];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[h][i] = vn[h][i];
+    if (base + stride < nunits) load(base + stride);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int64_t t = base + 32 * h + lane;
-      const uint32_t wd[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
-      float f[8];
+      float f0[8], f1[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(wd[i] << 16);
-        f[2 * i + 1] = __uint_as_float(wd[i] & 0xFFFF0000u);
+        f0[2 * i] = __uint_as_float(v[h][i] << 16);
+        f0[2 * i + 1] = __uint_as_float(v[h][i] & 0xFFFF0000u);
+        f1[2 * i] = __uint_as_float(v[h][4 + i] << 16);
+        f1[2 * i + 1] = __uint_as_float(v[h][4 + i] & 0xFFFF0000u);
       }
       float m = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
-      // each 8-lane group (one 64-block) reduces independently
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fmaxf(fabsf(f0[i]), fabsf(f1[i])));
+      // each 4-lane group (one 64-block) reduces independently
       m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
       m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
-      const uint32_t word = encode8<BUCKET>(f, m, s_mid, mid7, s_bk);
-      if (t < nwords) {
-        packed[t] = word;
-        if (sub == 0) absmax[t >> 3] = m;
+      const uint32_t w0 = encode8<BUCKET>(f0, m, s_mid, mid7, s_bk);
+      const uint32_t w1 = encode8<BUCKET>(f1, m, s_mid, mid7, s_bk);
+      if (t < nunits) {
+        *reinterpret_cast<uint2 *>(packed + 2 * t) = make_uint2(w0, w1);
+        if ((lane & 3u) == 0) absmax[t >> 2] = m;
       }
     }
   }

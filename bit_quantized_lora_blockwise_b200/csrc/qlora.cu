@@ -763,11 +763,14 @@ qlora_status qlora_quantize_nf4(const qlora_bf16 *W, int64_t N, int64_t K, const
   const int64_t nblocks = N * (K / 64);
   BucketTable bt;
   const bool bucketed = build_buckets(nf4, &bt);
-  auto kernel = bucketed ? quantize_nf4_kernel<true> : quantize_nf4_kernel<false>;
-  // one resident wave (a grid-stride loop covers the rest)
-  const int grid = grid_for(nblocks * 8, 512, d.sms,
-                            bucketed ? resident_per_sm<quantize_nf4_kernel<true>>(256)
-                                     : resident_per_sm<quantize_nf4_kernel<false>>(256));
+  // 32-byte loads when W allows them
+  const bool v8 = (reinterpret_cast<uintptr_t>(W) & 31u) == 0;
+  auto kernel = bucketed ? (v8 ? quantize_nf4_kernel<true, true> : quantize_nf4_kernel<true, false>)
+                         : (v8 ? quantize_nf4_kernel<false, true> : quantize_nf4_kernel<false, false>);
+  // one resident wave (a grid-stride loop covers the rest); 512 32-byte units per CTA pass
+  const int grid = grid_for(nblocks * 4, 512, d.sms,
+                            bucketed ? resident_per_sm<quantize_nf4_kernel<true, true>>(256)
+                                     : resident_per_sm<quantize_nf4_kernel<false, true>>(256));
   return launch_pdl(kernel, grid, 256, 0,
                     static_cast<cudaStream_t>(stream), reinterpret_cast<const uint4 *>(W), nblocks,
                     reinterpret_cast<uint32_t *>(packed), absmax, make_tables(nf4, nullptr), bt);

@@ -184,3 +184,19 @@ def test_quantize_nonfinite_weights():
     assert np.array_equal(am.cpu().numpy().view(np.uint32), am_o.view(np.uint32)), "absmax"
     assert np.array_equal(pk.cpu().numpy(), pk_o), "packed nibbles"
     assert binding.device_error() == 0
+
+
+def test_quantize_input_only_16_byte_aligned():
+    """A weight that starts 16 bytes into an allocation (16- but not
+    32-byte aligned) takes the 16-byte load path; results are identical."""
+    N, K = 96, 1024
+    W = weight_bf16(N, K, 0.02, seed=3, outlier_frac=0.001)
+    buf = torch.zeros(N * K + 64, dtype=torch.bfloat16, device="cuda")
+    Wv = buf[8:8 + N * K].view(N, K)
+    Wv.copy_(W.cuda())
+    assert Wv.data_ptr() % 32 == 16
+    pk_o, am_o = oracle.quantize_nf4(bf16_bits(W))
+    pk, am = binding.quantize_nf4(Wv)
+    torch.cuda.synchronize()
+    assert np.array_equal(am.cpu().numpy(), am_o)
+    assert np.array_equal(pk.cpu().numpy(), pk_o)
