@@ -320,6 +320,7 @@ int rank_tile(int r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
 
 // Ring depth per rank tile: 4 stages of 24 KB (r <= 64) or 3 of 32 KB
 // (r <= 128) keep two CTAs on an SM; r <= 256 uses 4 stages of 48 KB.
+// (Rings of about 192 KB per CTA, one CTA per SM, measured no faster.)
 constexpr int skinny_stages(int bn) { return bn == 64 ? 4 : (bn == 128 ? 3 : 4); }
 
 // One skinny-GEMM variant: its shared-memory opt-in and how many clusters
@@ -328,14 +329,22 @@ constexpr int skinny_stages(int bn) { return bn == 64 ? 4 : (bn == 128 ? 3 : 4);
 template <int BN, bool AMN, bool BMN>
 struct SkinnyVariant {
   using C = SkinnyCfg<BN, AMN, BMN, skinny_stages(BN)>;
-  static qlora_status prepare(int (&max_clusters)[4]) {
+  static qlora_status prepare(int (&max_clusters)[4], int *per_sm) {
     static std::once_flag once[kMaxDevices];
     static cudaError_t err[kMaxDevices];
     static int cached[kMaxDevices][4];
+    static int resident[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
     std::call_once(once[dev], [&] {
       err[dev] = cudaFuncSetAttribute(skinny_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+      int n1 = 0;
+      if (err[dev] != cudaSuccess ||
+          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, skinny_kernel<C>, C::THREADS, C::SMEM_BYTES) !=
+              cudaSuccess ||
+          n1 < 1)
+        n1 = 1;
+      resident[dev] = n1;
       cached[dev][0] = 0;
       for (int l = 1; l <= 3; ++l) {
         cudaLaunchConfig_t cfg = {};
@@ -359,12 +368,14 @@ struct SkinnyVariant {
       cudaGetLastError();  // an unsupported cluster size only means "not that one"
     });
     for (int l = 0; l < 4; ++l) max_clusters[l] = cached[dev][l];
+    *per_sm = resident[dev];
     return err[dev] == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
   }
 };
 
 struct SkinnyPlan {
   int rows, kblocks, splits, bn;
+  int per_sm;  // resident CTAs per SM
 };
 
 // Split K over a cluster of 2, 4 or 8 CTAs per 128-row tile: the largest
@@ -376,9 +387,9 @@ qlora_status plan_skinny_v(int64_t rows, int64_t kdim, int r, SkinnyPlan *p) {
   p->kblocks = static_cast<int>(cdiv(kdim, 64));
   p->bn = rank_tile(r);
   int maxc[4];
-  const qlora_status st = p->bn == 64    ? SkinnyVariant<64, AMN, BMN>::prepare(maxc)
-                          : p->bn == 128 ? SkinnyVariant<128, AMN, BMN>::prepare(maxc)
-                                         : SkinnyVariant<256, AMN, BMN>::prepare(maxc);
+  const qlora_status st = p->bn == 64    ? SkinnyVariant<64, AMN, BMN>::prepare(maxc, &p->per_sm)
+                          : p->bn == 128 ? SkinnyVariant<128, AMN, BMN>::prepare(maxc, &p->per_sm)
+                                         : SkinnyVariant<256, AMN, BMN>::prepare(maxc, &p->per_sm);
   const int row_tiles = static_cast<int>(cdiv(rows, 128));
   p->splits = 1;
   for (int l = 3; l >= 1; --l)
@@ -455,7 +466,7 @@ struct SkinnyOperands {
 // reduction length) as one grid; optionally with the constants pass.
 qlora_status skinny_launch(SkinnyKind kind, const SkinnyOperands *ops, int nprob, int r, int sms,
                            cudaStream_t st, unsigned int *zero_words, int nzero, bool early,
-                           const DecodeSpec *dc) {
+                           const DecodeSpec *dc, bool late = false) {
   int row_tiles[2] = {0, 0};
   for (int i = 0; i < nprob; ++i) row_tiles[i] = static_cast<int>(cdiv(ops[i].rows, 128));
   // the split is chosen for all row tiles of the launch together
@@ -503,13 +514,14 @@ qlora_status skinny_launch(SkinnyKind kind, const SkinnyOperands *ops, int nprob
   a.zero_words = zero_words;
   a.nzero = nzero;
   a.early = early ? 1 : 0;
+  a.late = late ? 1 : 0;
   a.gemm_ctas = (row_tiles[0] + row_tiles[1]) * p.splits;
   int grid = a.gemm_ctas;
   if (dc != nullptr) {
-    // one item (16 constants of a row) per thread, on the slots the GEMM CTAs
-    // leave free (two resident CTAs per SM for r <= 128), in whole clusters
+    // one item (16 constants of a row) per thread, on the CTA slots the GEMM
+    // CTAs leave free, in whole clusters
     const int64_t want = cdiv(dc->N * cdiv(dc->KB, 16), 256);
-    const int64_t free_slots = static_cast<int64_t>(p.bn <= 128 ? 2 : 1) * sms - a.gemm_ctas;
+    const int64_t free_slots = static_cast<int64_t>(p.per_sm) * sms - a.gemm_ctas;
     int64_t n = std::min(want, std::max<int64_t>(free_slots, p.splits));
     n = cdiv(std::max<int64_t>(n, 1), p.splits) * p.splits;
     grid += static_cast<int>(n);
@@ -996,12 +1008,16 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   if (st != QLORA_OK) return st;
 
   // 3) dA = X^T Gs ([K, r]) and dB = s XA^T dY ([r, N], from dB^T[n, j]) in one
-  //    launch; every operand was written at least two kernels back (complete
-  //    once the dX GEMM started), so the first stages load before the wait
+  //    launch. Every operand was written at least two kernels back: this
+  //    launch can only start once every dX CTA has passed its own wait for
+  //    those kernels, so they are complete; and the dX GEMM neither reads dA,
+  //    dB nor writes anything read here. So the launch runs "late": its CTAs
+  //    compute on the SMs the dX GEMM's last wave leaves idle and wait for it
+  //    only before exiting (the call still ends after dX is written).
   const SkinnyOperands ops[2] = {
       {X, K, M, gs, r, M, K, M, OutSpec{dA, r, 1.0f, nullptr, 0, 0.0f, false}},
       {dY, N, M, xa, r, M, N, M, OutSpec{dB, N, scl, nullptr, 0, 0.0f, true}}};
-  return skinny_launch(SK_DA, ops, 2, r, d.sms, cs, nullptr, 0, true, nullptr);
+  return skinny_launch(SK_DA, ops, 2, r, d.sms, cs, nullptr, 0, true, nullptr, true);
 }
 
 }  // extern "C"

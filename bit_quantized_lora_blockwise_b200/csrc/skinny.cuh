@@ -47,6 +47,9 @@ struct SkinnyArgs {
   int nzero;
   int early;  // 1: neither operand is written by the kernel just before this one in the stream, so the
               // first ring stages may be loaded before waiting for that kernel (programmatic launch)
+  int late;   // 1: every operand is complete when this launch starts and nothing it writes is touched by
+              // the kernel before it, so the whole product runs without waiting for that kernel; each
+              // thread waits for it only before exiting, so this grid still completes after it
   // Optional constants pass for the fused GEMM that follows, run by the CTAs
   // from gemm_ctas on (whole clusters): cprime[kb * dc_N + n] = t8[q] * S.
   int gemm_ctas;
@@ -159,9 +162,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_cons
       tma_load_2d(b_dst, &P.tm_b, full_bar(s), kb * 64, 0);
     }
   };
-  if (args.early && warp == 0 && lane == 0)
+  if (args.early && !args.late && warp == 0 && lane == 0)
     for (; issued < nk && issued < C::STAGES; ++issued) issue(issued);
-  grid_dep_wait();
+  if (!args.late) grid_dep_wait();
   grid_dep_launch();
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < args.nzero; i += blockDim.x) args.zero_words[i] = 0u;
@@ -300,6 +303,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_cons
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
+  if (args.late) grid_dep_wait();
 }
 
 }  // namespace qlora

@@ -143,6 +143,39 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
     uint32_t q[2];
     float s[2];
   };
+  // L2 prefetch: a second walk over the same units, kPfAhead units ahead of
+  // the register loads, so that those loads hit L2 rather than DRAM
+  constexpr int kPfAhead = 4;
+  int pf_band = u_begin / a.kc, pf_c = u_begin - (u_begin / a.kc) * a.kc, pf_idx = 0;
+  const uint8_t *pf_p = nullptr, *pf_q = nullptr;
+  bool pf_row_ok = false;
+  auto pf_setup = [&]() {
+    const int64_t row = static_cast<int64_t>(pf_band) * C::BAND + warp * 16 + g;
+    pf_row_ok = row < a.N;
+    const int64_t bi = row * kb_total + static_cast<int64_t>(pf_c) * 4 + t;
+    pf_p = a.packed + bi * 32;
+    pf_q = a.q + bi;
+  };
+  auto pf_step = [&]() {  // prefetch the walk's unit (rows g and g + 8), then advance
+    if (pf_idx >= nunits) return;
+    if (pf_row_ok && static_cast<int64_t>(pf_c) * 4 + t < kb_total) {
+      prefetch_l2(pf_p);
+      prefetch_l2(pf_p + 8 * row_bytes);
+      prefetch_l2(pf_q);
+      prefetch_l2(pf_q + 8 * kb_total);
+    }
+    ++pf_idx;
+    if (++pf_c == a.kc) {
+      pf_c = 0;
+      ++pf_band;
+      pf_setup();
+    } else {
+      pf_p += 128;
+      pf_q += 4;
+    }
+  };
+  pf_setup();
+  for (int k = 0; k < kPfAhead; ++k) pf_step();  // units 0 .. kPfAhead - 1 up front
   int ld_band = u_begin / a.kc, ld_c = u_begin - (u_begin / a.kc) * a.kc;
   const uint8_t *ld_p = nullptr;  // row g of the band, chunk ld_c, block t
   int64_t ld_bi = 0;              // block index of that row and block
@@ -188,12 +221,7 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
       ld_p += 128;
       ld_bi += 4;
     }
-    // the unit after this one: its packed rows into L2 now, so that its
-    // register loads (issued one unit later) hit L2
-    if (ld_row_ok && static_cast<int64_t>(ld_c) * 4 + t < kb_total) {
-      prefetch_l2(ld_p);
-      prefetch_l2(ld_p + 8 * row_bytes);
-    }
+    pf_step();
   };
 
   float acc[NT][4];

@@ -171,7 +171,10 @@ QLORA_API qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q,
  *   dB = s (X A)^T dY
  *   X [M, K], dY [M, N], A [K, r], B [r, N]: device bf16.
  *   XA: device bf16 [M, r] saved by the forward, or NULL to recompute X A.
- *   dX [M, K], dA [K, r], dB [r, N]: device bf16 outputs.
+ *   dX [M, K], dA [K, r], dB [r, N]: device bf16 outputs. They must not
+ *   overlap any input or each other: the dA/dB kernel runs concurrently with
+ *   the tail of the dX GEMM (the call still completes, in stream order, only
+ *   after every output is written).
  * Same requirements as qlora_linear_fwd.
  */
 QLORA_API qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const float *scale2,
