@@ -338,6 +338,11 @@ struct SkinnyVariant {
     cudaGetDevice(&dev);
     std::call_once(once[dev], [&] {
       err[dev] = cudaFuncSetAttribute(skinny_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+      // ask for the largest shared-memory carveout, so that two CTAs of
+      // about 100 KB share an SM and the occupancy queries below count them
+      if (err[dev] == cudaSuccess)
+        err[dev] = cudaFuncSetAttribute(skinny_kernel<C>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                        static_cast<int>(cudaSharedmemCarveoutMaxShared));
       int n1 = 0;
       if (err[dev] != cudaSuccess ||
           cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, skinny_kernel<C>, C::THREADS, C::SMEM_BYTES) !=
