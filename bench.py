@@ -25,6 +25,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -72,11 +73,24 @@ def peaks():
         return dict(PEAKS_FALLBACK), "fallback"
 
 
-def kernel_source_hash():
+def _code_only(text: str) -> str:
+    """Kernel source without comments and blank space, so that an edit to a
+    comment does not mark the profiled kernels as changed."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
+def kernel_source_hash(read=None):
+    """Hash of the kernel sources' code (comments and spacing ignored)."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        if read is None:
+            with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+                text = f.read()
+        else:
+            text = read(rel)
+        h.update(_code_only(text).encode())
     return h.hexdigest()[:16]
 
 

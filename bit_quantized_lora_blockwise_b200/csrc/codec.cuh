@@ -6,10 +6,11 @@
 // "QLoRA: Finetuning 65B Models on a Single GPU", sections "4-bit
 // NormalFloat" and "Double Quantization and Paged Optimizers".
 //
-// All three kernels are HBM-bound streaming kernels: 128-bit loads, one warp
-// lane per 8 (quantize) or 16 (dequant) consecutive weights, warp shuffles
-// for the per-block reduction, grid-stride loops over a grid sized to the
-// SM count.
+// Quantize and dequant are HBM-bound streaming kernels: wide vector loads
+// (one lane takes 16 consecutive weights to quantize, or a whole 64-block to
+// dequantize), warp shuffles for the per-block reduction, grid-stride loops
+// over a grid sized to the SM count. Double quantization has far fewer
+// bytes and is bound by latency: one warp per group of 256 constants.
 #pragma once
 
 #include "ptx.cuh"
