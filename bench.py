@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-compare", action="store_true",
+                    help="skip the dequantize-then-cuBLAS comparison leg")
     ap.add_argument("--linears", default="", help="comma list of linear names to keep (profiling runs)")
     return ap.parse_args()
 
@@ -290,6 +292,53 @@ class LinearState:
                 "dequant": n // 2 + n // 64 + ((n // 64 + 255) // 256) * 4 + n * 2}
 
 
+def compare_dequant_then_library_gemm(layers, ws, steps):
+    """The design the pages describe, dequantize then multiply, timed against
+    the fused calls (a comparison, not the product and not the headline).
+    Per linear: this library's dequant writes the bf16 W' to HBM and
+    cuBLAS (torch.matmul) computes the same forward and backward products
+    (X A, Y, dY B^T, dX, dA, dB in bf16); against it, qlora_linear_fwd +
+    qlora_linear_bwd. Both are queued behind a GPU sleep and timed on the
+    device over the 7 linears."""
+    import torch
+    from bit_quantized_lora_blockwise_b200 import binding
+
+    def fused(L):
+        binding.linear_fwd(L.packed, L.q, L.scale2, L.X, L.A, L.B, L.alpha, L.N, L.K, Y=L.Y, XA_out=L.XA,
+                           workspace=ws)
+        binding.linear_bwd(L.packed, L.q, L.scale2, L.X, L.dY, L.A, L.B, L.alpha, L.N, L.K, XA=L.XA, dX=L.dX,
+                           dA=L.dA, dB=L.dB, workspace=ws)
+
+    def library(L):
+        s = L.alpha / L.r
+        binding.dequant(L.packed, L.q, L.scale2, L.N, L.K, out=L.Wq)
+        xas = (L.X @ L.A) * s
+        torch.addmm(xas @ L.B, L.X, L.Wq.t())              # Y
+        g = (L.dY @ L.B.t()) * s
+        torch.addmm(g @ L.A.t(), L.dY, L.Wq)               # dX
+        L.X.t() @ g                                        # dA
+        xas.t() @ L.dY                                     # dB
+
+    out = {}
+    for name, fn in (("fused_ms", fused), ("dequant_then_cublas_ms", library)):
+        for L in layers:  # warm (cuBLAS heuristics, allocator)
+            fn(L)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(QUEUE_AHEAD_CYCLES)
+        e0.record()
+        for _ in range(steps):
+            for L in layers:
+                fn(L)
+        e1.record()
+        torch.cuda.synchronize()
+        out[name] = round(e0.elapsed_time(e1) / steps, 4)
+    out["fused_speedup"] = round(out["dequant_then_cublas_ms"] / out["fused_ms"], 3)
+    out["what"] = ("fwd + bwd of the 7 linears per step; library path = dequant kernel (bf16 W' in HBM) "
+                   "+ torch.matmul (cuBLAS) bf16 GEMMs; fused path = qlora_linear_fwd + qlora_linear_bwd")
+    return out
+
+
 def run_native(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -427,6 +476,7 @@ def run_native(args, rank, world, local_rank):
         c1.record()
         torch.cuda.synchronize()
         codec_run_ms[name] = c0.elapsed_time(c1) / args.steps
+    compare = compare_dequant_then_library_gemm(layers, ws, args.steps) if not args.no_compare else None
     ms = t_start.elapsed_time(t_stop) / args.steps
     if world > 1:
         t = torch.tensor([ms], device=dev)
@@ -570,7 +620,8 @@ def run_native(args, rank, world, local_rank):
                            "step": "per linear: quantize_nf4, double_quant, dequant, linear_fwd, linear_bwd, "
                                    f"linear_fwd on the first {SMALL_M} tokens"},
                 "phases": phases, "roofline": roofline, "gpu_launches": launches,
-                "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "device_error": err}
+                "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
+                "compare_dequant_then_library_gemm": compare, "device_error": err}
         print(json.dumps(line), flush=True)
 
 

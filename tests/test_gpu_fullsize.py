@@ -113,3 +113,47 @@ def test_llama65b_few_token_forward_full_size(cuda_device, li, M):
     Yo, XAo = oracle.linear_fwd(bf16_bits(X), wq, bf16_bits(A), bf16_bits(B), wl.alpha, wl.r)
     assert _rel(Y, Yo) <= TOL
     assert _rel(XA, XAo) <= TOL
+
+
+@pytest.mark.parametrize("li", [0, 4, 6])  # q 4096^2, gate 4096 -> 11008, down 11008 -> 4096
+def test_llama7b_every_output_against_dequant_then_fp32_matmul(cuda_device, li):
+    """Every element of Y, dX, dA and dB at full size (M = 2048), against the
+    dequantize-then-multiply formulation computed with fp32 matmuls on the
+    device, from the library's own dequantized W' (bit-exact to the oracle
+    by the codec tests). Complements the fp64 oracle's sampled rows above."""
+    wl = WORKLOADS["llama7b_set"]
+    M = 2048
+    inp = layer_inputs(wl, li, M)
+    W, X, A, B, dY = (inp[k].cuda() for k in ("W", "X", "A", "B", "dY"))
+    N, K = W.shape
+    r, alpha = wl.r, wl.alpha
+    s = alpha / r
+    pk, am = binding.quantize_nf4(W)
+    q, s2 = binding.double_quant(am)
+    wq = binding.dequant(pk, q, s2, N, K)
+    XA = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    Y = binding.linear_fwd(pk, q, s2, X, A, B, alpha, N, K, XA_out=XA)
+    dX, dA, dB = binding.linear_bwd(pk, q, s2, X, dY, A, B, alpha, N, K, XA=XA)
+    torch.cuda.synchronize()
+    assert binding.device_error() == 0
+    tf32 = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        Xf, Wf, Af, Bf, dYf = X.float(), wq.float(), A.float(), B.float(), dY.float()
+        XAf = Xf @ Af
+        Yr = Xf @ Wf.t() + s * (XAf @ Bf)
+        G = dYf @ Bf.t()
+        dXr = dYf @ Wf + s * (G @ Af.t())
+        dAr = s * (Xf.t() @ G)
+        dBr = s * (XAf.t() @ dYf)
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = tf32
+
+    def rel(got, want):
+        return float((got.float() - want).abs().max() / want.abs().max())
+
+    assert rel(Y, Yr) <= TOL
+    assert rel(XA, XAf) <= TOL
+    assert rel(dX, dXr) <= TOL
+    assert rel(dA, dAr) <= TOL
+    assert rel(dB, dBr) <= TOL
