@@ -136,9 +136,11 @@ def test_packed_weight_untouched_by_backward():
     assert torch.equal(before[0], L.pk) and torch.equal(before[1], L.q) and torch.equal(before[2], L.s2)
 
 
-@pytest.mark.parametrize("M", [1, 4, 16])
+@pytest.mark.parametrize("M", [1, 4, 16, 17, 24, 32])
 def test_small_m_split_k(M):
-    """Few tokens: the forward splits K across CTAs (fp32 partials + reduce)."""
+    """Few tokens. M <= 16: the register-dequant weight stream; 16 < M <= 32:
+    the fused GEMM on 32-token tiles, K split across CTAs (fp32 partials +
+    reduce). The backward always takes the fused GEMM."""
     L = Layer(M, 1024, 2048, 64, seed=100 + M, w_std=0.015)
     Y, XA = L.fwd()
     Yo, XAo = L.oracle_fwd()
