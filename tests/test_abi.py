@@ -92,3 +92,18 @@ def test_argument_checks_before_any_launch(lib):
     assert fwd(alpha=float("inf")) == 4
     assert lib.qlora_workspace_bytes(16, 96, 128, 8) == 0
     assert lib.qlora_workspace_bytes(16, 128, 128, 8) > 0
+    # a NaN level is refused like a descending table
+    nan8 = np.arange(256, dtype=np.float32) / 255
+    nan8[17] = np.nan
+    assert lib.qlora_double_quant(_fake(), 10, (ctypes.c_float * 256)(*nan8), _fake(), _fake(), s) == 8
+    # dequant: NULL output, K % 64, misaligned output
+    assert lib.qlora_dequant(_fake(), _fake(), _fake(), 64, 64, tb.nf4, tb.t8, None, s) == 1
+    assert lib.qlora_dequant(_fake(), _fake(), _fake(), 64, 96, tb.nf4, tb.t8, _fake(), s) == 2
+    assert lib.qlora_dequant(_fake(), _fake(), _fake(), 64, 64, tb.nf4, tb.t8, _fake(0x10004), s) == 3
+
+    def bwd(**kw):
+        a = {**args, **kw}
+        return lib.qlora_linear_bwd(_fake(), _fake(), _fake(), tb.nf4, tb.t8, a["M"], a["N"], a["K"],
+                                    _fake(), _fake(), _fake(), _fake(), None, a["r"], a["alpha"],
+                                    _fake(), _fake(), _fake(), _fake(), 1 << 30, s)
+    assert bwd(r=0) == 4 and bwd(r=257) == 4 and bwd(N=100) == 2 and bwd(alpha=float("nan")) == 4
