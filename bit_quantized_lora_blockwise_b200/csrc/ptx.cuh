@@ -1,7 +1,7 @@
 // Inline-PTX wrappers for sm_100a: mbarriers, TMA tiled loads, tcgen05
 // (TMEM allocation, MMA, commit, TMEM loads) and a few fences.
-// Only the forms used by this library are wrapped; no cluster multicast
-// anywhere.
+// Only the forms used by this library are wrapped; every TMA load targets
+// the issuing CTA's own shared memory.
 #pragma once
 
 #include <cuda.h>
