@@ -1,9 +1,10 @@
 // Few-token forward: Y = X W'^T + B^T-term for M <= 16 tokens, a stream of
 // the packed weight with the dequantization done in registers.
 //
-// QLoRA (Dettmers et al.), section 3 "QLoRA Finetuning", the forward of one
-// linear: the base weight is stored as NF4 codes with double-quantized block
-// constants and is dequantized to bf16 before it is multiplied. With a few
+// The forward of one QLoRA linear (intvml.com "DL0087 QLoRA: 4-bit Quantized
+// LoRA", opening paragraph and Figure 1): the base weight is stored as NF4
+// codes with double-quantized block constants and is dequantized to bf16
+// just before it is multiplied. With a few
 // tokens the layer reads 0.516 bytes of packed weight per parameter and does
 // 2 M flops with it, so it is bound by HBM. This kernel therefore never
 // stages the weight in shared memory: every packed byte is loaded once, by

@@ -193,3 +193,26 @@ def test_storage_matches_page_figures():
     assert abs(16 * g["params"] / 8 / 1e9 - g["value"]) <= g["rounded_to"]
     assert 16 * GOLDEN["storage_70b_16bit_gb"]["params"] / 8 / 1e9 == GOLDEN["storage_70b_16bit_gb"]["value"]
     assert payload * GOLDEN["storage_70b_4bit_gb"]["params"] / 8 / 1e9 == GOLDEN["storage_70b_4bit_gb"]["value"]
+
+
+def test_bf16_conversions_match_torch():
+    """The oracle's fp32 <-> bf16 helpers against torch's conversions (an
+    independent library routine): widening is exact, narrowing rounds to
+    nearest even, on ties (low half 0x8000), neighbours of ties, subnormals,
+    infinities and the largest finite values."""
+    import torch
+    rng = np.random.default_rng(7)
+    hi = rng.integers(0, 1 << 16, 4096, dtype=np.uint32)
+    lows = np.array([0x0000, 0x0001, 0x7FFF, 0x8000, 0x8001, 0xFFFF], np.uint32)
+    bits = (hi[:, None] << 16 | lows[None, :]).reshape(-1)
+    bits = np.concatenate([bits, np.array([0x7F7FFFFF, 0xFF7FFFFF, 0x7F800000, 0xFF800000, 0x00000001,
+                                           0x807FFFFF, 0x00008000, 0x7F7F8000], np.uint32)])
+    x = bits.view(np.float32)
+    finite_or_inf = ~np.isnan(x)
+    x = x[finite_or_inf]
+    got = oracle.f32_to_bf16(x)
+    want = torch.from_numpy(x.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, want)
+    back = oracle.bf16_to_f32(got)
+    want_back = torch.from_numpy(want.view(np.int16).copy()).view(torch.bfloat16).float().numpy()
+    assert np.array_equal(back.view(np.uint32), want_back.view(np.uint32))

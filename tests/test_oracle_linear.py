@@ -6,8 +6,8 @@
   L = <dY, Y> (the layer is linear in X, A and B, so the differences are
   exact up to rounding);
 * B = 0 reproduces the quantized base exactly and gives dA = 0; A = 0 gives
-  dB = 0 (intvml.com "DL0087 QLoRA", formulation list: B starts at zero so
-  the layer initially reproduces the quantized base model);
+  dB = 0 (intvml.com "DL0087 QLoRA", formulation list: with the adapter B
+  at its zero initial value the layer equals the quantized base);
 * a planted mistake (an operand transposed in a copy of the backward) is
   caught by the finite-difference pin.
 """

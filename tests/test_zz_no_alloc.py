@@ -3,15 +3,17 @@ allocate device memory (a plugin inside a framework that owns every device
 allocation, or a loop that must never enter the allocator).
 
 The entry point takes no workspace: it runs the forward on the library's
-fixed device scratch array. Its output must match the ordinary
-qlora_linear_fwd (caller workspace) within the layer tolerance, on two calls
-in a row with different inputs (the scratch keeps the previous call's
-contents, so the second call checks that nothing leaks between calls), and a
-shape whose scratch would exceed the fixed size must be refused.
+fixed device scratch array. It launches the same deterministic kernels as
+the ordinary qlora_linear_fwd (caller workspace), so its outputs must be
+bit-identical to that call's, on two calls in a row. The two calls use
+different inputs, with adapters at N(0, 1) so that the adapter term is
+most of Y: the scratch keeps the previous call's contents (among them the
+scaled X A operand), and anything that leaked from the first call into the
+second would change bits. A shape whose scratch would exceed the fixed
+size must be refused.
 
 Named test_zz_* so that pytest collects it last.
 """
-import numpy as np
 import pytest
 import torch
 
@@ -19,14 +21,6 @@ from bit_quantized_lora_blockwise_b200 import binding
 from bit_quantized_lora_blockwise_b200.inputs import normal_bf16, weight_bf16
 
 pytestmark = pytest.mark.gpu
-TOL = 1e-2
-
-
-def _rel(a: torch.Tensor, b: torch.Tensor) -> float:
-    a64 = a.float().cpu().numpy().astype(np.float64)
-    b64 = b.float().cpu().numpy().astype(np.float64)
-    den = np.max(np.abs(b64))
-    return float(np.max(np.abs(a64 - b64)) / (den if den > 0 else 1.0))
 
 
 def _layer(M, N, K, r, seed):
@@ -34,8 +28,8 @@ def _layer(M, N, K, r, seed):
     pk, am = binding.quantize_nf4(W)
     q, s2 = binding.double_quant(am)
     X = normal_bf16((M, K), 1.0, seed + 1).cuda()
-    A = normal_bf16((K, r), 0.01, seed + 2).cuda()
-    B = normal_bf16((r, N), 0.01, seed + 3).cuda()
+    A = normal_bf16((K, r), 1.0, seed + 2).cuda()
+    B = normal_bf16((r, N), 1.0, seed + 3).cuda()
     return pk, q, s2, X, A, B
 
 
@@ -52,8 +46,8 @@ def test_noalloc_matches_workspace_forward_two_calls(M, N, K, r):
         binding.linear_fwd_noalloc(pk, q, s2, X, A, B, 16.0, N, K, Y=Y, XA_out=XA)
         torch.cuda.synchronize()
         assert binding.device_error() == 0
-        assert _rel(Y, Y_ref) <= TOL, f"call {call}: Y"
-        assert _rel(XA, XA_ref) <= TOL, f"call {call}: XA"
+        assert torch.equal(Y, Y_ref), f"call {call}: Y differs from the workspace forward"
+        assert torch.equal(XA, XA_ref), f"call {call}: XA differs from the workspace forward"
 
 
 def test_noalloc_refuses_oversized_scratch():
