@@ -61,6 +61,9 @@ def parse():
     ap.add_argument("--no-compare", action="store_true",
                     help="skip the dequantize-then-cuBLAS comparison leg")
     ap.add_argument("--linears", default="", help="comma list of linear names to keep (profiling runs)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the diagnostic rows of the other workloads (single linear, 13B codec sweep, "
+                         "65B forwards, 33B block)")
     return ap.parse_args()
 
 
@@ -260,7 +263,7 @@ def cpu_threads():
         return os.cpu_count()
 
 
-def cpu_baseline(wl, budget_s=12.0):
+def _oracle_rate(wl, budget_s):
     t0 = time.perf_counter()
     flops = 0
     n = 0
@@ -272,8 +275,23 @@ def cpu_baseline(wl, budget_s=12.0):
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{n} x ({sample}); {dt:.1f} s"}
+    return flops / dt / 1e12, f"{n} x ({sample}); {dt:.1f} s"
+
+
+def cpu_baseline(wl, budget_s=8.0):
+    """The oracle on the host: all cores (its float64 matmuls use the BLAS
+    thread pool; the C codec is single-threaded), and limited to one thread."""
+    value, sample = _oracle_rate(wl, budget_s)
+    single = None
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            v1, s1 = _oracle_rate(wl, budget_s)
+        single = {"value": v1, "unit": UNIT, "cores": 1, "sample": s1}
+    except ImportError:
+        pass
+    return {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle", "sample": sample,
+            "single_thread": single}
 
 
 def run_reference(args, rank):
@@ -399,6 +417,181 @@ def compare_dequant_then_library_gemm(layers, ws, steps):
     out["fused_speedup"] = round(out["dequant_then_cublas_ms"] / out["fused_ms"], 3)
     out["what"] = ("fwd + bwd of the 7 linears per step; library path = dequant kernel (bf16 W' in HBM) "
                    "+ torch.matmul (cuBLAS) bf16 GEMMs; fused path = qlora_linear_fwd + qlora_linear_bwd")
+    return out
+
+
+def device_ms(fn, reps, warm=2):
+    """Device time of one fn() (mean of `reps` back to back), queued behind a
+    GPU sleep so that the events time the device, not the host's enqueue."""
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(QUEUE_AHEAD_CYCLES)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def workload_phases(dev, hbm_gbs, tc_tflops, quick=False):
+    """Every other workload the hot path is specified on, timed on the
+    device after the headline (diagnostic rows, not the headline):
+      single_1024          one 1024x1024 linear, M = 16, r = 8: fwd + bwd latency
+      llama13b_quant_sweep quantize + double quant, and dequant, over 40 layers x 7 linears
+      llama65b_fwd         7 linears: few-token forwards (M = 1, 4, 16) and M = 4096
+      llama33b_block       7 linears, M = 2048: fwd (saving XA) + bwd recomputing XA
+    Rates are against the measured peaks and the spec ones (8 TB/s HBM,
+    2.25 PFLOP/s dense bf16)."""
+    import torch
+    from bit_quantized_lora_blockwise_b200 import binding
+    from bit_quantized_lora_blockwise_b200.inputs import WORKLOADS, layer_inputs, weight_bf16, seed_for
+    out = {}
+
+    def frac_hbm(gbs):
+        return {"GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm_gbs, 3), "frac_8tbs": round(gbs / SPEC_HBM_GBS, 3)}
+
+    def frac_tc(tf):
+        return {"TFLOP/s": round(tf, 1), "frac_tensor": round(tf / tc_tflops, 3),
+                "frac_spec": round(tf / SPEC_BF16_TFLOPS, 3)}
+
+    def quantized(W):
+        pk, am = binding.quantize_nf4(W)
+        q, s2 = binding.double_quant(am)
+        return pk, q, s2
+
+    # -- single linear (latency; every tensor L2-resident)
+    wl = WORKLOADS["single_1024"]
+    inp = layer_inputs(wl, 0, wl.M[0], device=dev)
+    N, K, M, r = wl.linears[0].N, wl.linears[0].K, wl.M[0], wl.r
+    pk, q, s2 = quantized(inp["W"])
+    ws = torch.empty(binding.workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    Y, XA = torch.empty((M, N), dtype=torch.bfloat16, device=dev), torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+    dX, dA, dB = (torch.empty(sh, dtype=torch.bfloat16, device=dev) for sh in ((M, K), (K, r), (r, N)))
+
+    def c1():
+        binding.linear_fwd(pk, q, s2, inp["X"], inp["A"], inp["B"], wl.alpha, N, K, Y=Y, XA_out=XA, workspace=ws)
+        binding.linear_bwd(pk, q, s2, inp["X"], inp["dY"], inp["A"], inp["B"], wl.alpha, N, K, XA=XA, dX=dX,
+                           dA=dA, dB=dB, workspace=ws)
+    ms = device_ms(c1, 50)
+    out["single_1024"] = {"what": "qlora_linear_fwd + qlora_linear_bwd, 1024x1024, M=16, r=8 (L2-resident)",
+                          "us_per_fwd_bwd": round(ms * 1e3, 2),
+                          "TFLOP/s": round(linear_flops(M, N, K, r) / (ms * 1e-3) / 1e12, 3)}
+    del inp, pk, q, s2, ws
+
+    # -- 13B-equivalent codec sweep: one layer's buffers, refilled per layer (outside the timed calls)
+    wl = WORKLOADS["llama13b_quant_sweep"]
+    layers = 4 if quick else wl.layers
+    bufs = []
+    for lin in wl.linears:
+        n = lin.N * lin.K
+        bufs.append({"N": lin.N, "K": lin.K, "W": torch.empty((lin.N, lin.K), dtype=torch.bfloat16, device=dev),
+                     "pk": torch.empty(n // 2, dtype=torch.uint8, device=dev),
+                     "am": torch.empty(n // 64, dtype=torch.float32, device=dev),
+                     "q": torch.empty(n // 64, dtype=torch.uint8, device=dev),
+                     "s2": torch.empty((n // 64 + 255) // 256, dtype=torch.float32, device=dev),
+                     "Wq": torch.empty((lin.N, lin.K), dtype=torch.bfloat16, device=dev)})
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 2x L2: written between timed calls
+    t_q = t_dq = t_d = 0.0
+    params = 0
+    for layer in range(layers):
+        for li, b in enumerate(bufs):
+            b["W"].copy_(weight_bf16(b["N"], b["K"], wl.w_std, seed_for(wl.index, li, 0, layer), device=dev))
+        flush.zero_()
+        t_q += device_ms(lambda: [binding.quantize_nf4(b["W"], packed=b["pk"], absmax=b["am"]) for b in bufs], 1, 0)
+        flush.zero_()
+        t_dq += device_ms(lambda: [binding.double_quant(b["am"], q=b["q"], scale2=b["s2"]) for b in bufs], 1, 0)
+        flush.zero_()
+        t_d += device_ms(lambda: [binding.dequant(b["pk"], b["q"], b["s2"], b["N"], b["K"], out=b["Wq"])
+                                  for b in bufs], 1, 0)
+        params += sum(b["N"] * b["K"] for b in bufs)
+    n = params
+    q_in, q_out = 2 * n, n // 2 + n // 64 * 4
+    dq_in, dq_out = n // 64 * 4, n // 64 + n // 16384 * 4
+    d_in, d_out = n // 2 + n // 64 + n // 16384 * 4, 2 * n
+    out["llama13b_quant_sweep"] = {
+        "what": f"{layers} layers x 7 linears (d=5120, ffn=13824), {n / 1e9:.3f} G params, per-call events summed",
+        "quantize": {"ms": round(t_q, 3), "GB_in": round(q_in / 1e9, 3), "GB_out": round(q_out / 1e9, 3),
+                     **frac_hbm((q_in + q_out) / (t_q * 1e-3) / 1e9)},
+        "double_quant": {"ms": round(t_dq, 3), **frac_hbm((dq_in + dq_out) / (t_dq * 1e-3) / 1e9)},
+        "quantize_plus_double_quant": {"ms": round(t_q + t_dq, 3),
+                                       **frac_hbm((q_in + q_out + dq_in + dq_out) / ((t_q + t_dq) * 1e-3) / 1e9)},
+        "dequant": {"ms": round(t_d, 3), "GB_in": round(d_in / 1e9, 3), "GB_out": round(d_out / 1e9, 3),
+                    **frac_hbm((d_in + d_out) / (t_d * 1e-3) / 1e9)}}
+    del bufs, flush
+
+    # -- 65B-shaped forwards: few tokens (HBM-bound) and M = 4096 (tensor-bound)
+    wl = WORKLOADS["llama65b_fwd"]
+    packed = []
+    for li, lin in enumerate(wl.linears):
+        W = weight_bf16(lin.N, lin.K, wl.w_std, seed_for(wl.index, li, 0), device=dev)
+        packed.append((lin, *quantized(W)))
+        del W
+    torch.cuda.synchronize()
+    Mmax = max(wl.M)
+    Kmax = max(lin.K for lin in wl.linears)
+    Nmax = max(lin.N for lin in wl.linears)
+    acts = []
+    for li, (lin, _, _, _) in enumerate(packed):
+        acts.append({"X": torch.randn((Mmax, lin.K), device=dev).to(torch.bfloat16),
+                     "A": (torch.randn((lin.K, wl.r), device=dev) * 0.01).to(torch.bfloat16),
+                     "B": (torch.randn((wl.r, lin.N), device=dev) * 0.01).to(torch.bfloat16)})
+    Ybuf = torch.empty(Mmax * Nmax, dtype=torch.bfloat16, device=dev)
+    XAbuf = torch.empty(Mmax * wl.r, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(binding.workspace_bytes(m, lin.N, lin.K, wl.r) for m in wl.M for lin, *_ in packed),
+                     dtype=torch.uint8, device=dev)
+    c4 = {"what": "7 linears (d=8192, ffn=22016), r=64: one qlora_linear_fwd per linear, summed"}
+    for m in wl.M:
+        def fwd_all(m=m):
+            for (lin, pk, q, s2), a in zip(packed, acts):
+                binding.linear_fwd(pk, q, s2, a["X"][:m], a["A"], a["B"], wl.alpha, lin.N, lin.K,
+                                   Y=Ybuf[:m * lin.N].view(m, lin.N), XA_out=XAbuf[:m * wl.r].view(m, wl.r),
+                                   workspace=ws)
+        ms = device_ms(fwd_all, 3 if m > 16 else 10)
+        flops = sum(2 * m * lin.N * lin.K + 2 * m * wl.r * (lin.N + lin.K) for lin, *_ in packed)
+        if m <= 16:
+            nbytes = sum(lin.N * lin.K // 2 + lin.N * lin.K // 64 + (lin.N * lin.K // 16384) * 4 +
+                         2 * (m * lin.K + lin.K * wl.r + wl.r * lin.N + m * lin.N + m * wl.r) for lin, *_ in packed)
+            c4[f"M{m}"] = {"ms": round(ms, 4), "MB": round(nbytes / 1e6, 1), **frac_hbm(nbytes / (ms * 1e-3) / 1e9)}
+        else:
+            c4[f"M{m}"] = {"ms": round(ms, 4), **frac_tc(flops / (ms * 1e-3) / 1e12)}
+    out["llama65b_fwd"] = c4
+    del packed, acts, Ybuf, XAbuf, ws
+
+    # -- 33B-shaped block: forward saving XA, backward recomputing XA (checkpoint style)
+    wl = WORKLOADS["llama33b_block"]
+    M = wl.M[0]
+    state = []
+    for li, lin in enumerate(wl.linears):
+        inp = layer_inputs(wl, li, M, device=dev)
+        pk, q, s2 = quantized(inp["W"])
+        del inp["W"]
+        state.append((lin, pk, q, s2, inp, torch.empty((M, lin.N), dtype=torch.bfloat16, device=dev),
+                      torch.empty((M, wl.r), dtype=torch.bfloat16, device=dev),
+                      torch.empty((M, lin.K), dtype=torch.bfloat16, device=dev),
+                      torch.empty((lin.K, wl.r), dtype=torch.bfloat16, device=dev),
+                      torch.empty((wl.r, lin.N), dtype=torch.bfloat16, device=dev)))
+    ws = torch.empty(max(binding.workspace_bytes(M, lin.N, lin.K, wl.r) for lin, *_ in state),
+                     dtype=torch.uint8, device=dev)
+
+    def block():
+        for lin, pk, q, s2, inp, Y, XA, dX, dA, dB in state:
+            binding.linear_fwd(pk, q, s2, inp["X"], inp["A"], inp["B"], wl.alpha, lin.N, lin.K, Y=Y, XA_out=XA,
+                               workspace=ws)
+        for lin, pk, q, s2, inp, Y, XA, dX, dA, dB in reversed(state):
+            binding.linear_bwd(pk, q, s2, inp["X"], inp["dY"], inp["A"], inp["B"], wl.alpha, lin.N, lin.K, XA=None,
+                               dX=dX, dA=dA, dB=dB, workspace=ws)
+    ms = device_ms(block, 3)
+    flops = sum(linear_flops(M, lin.N, lin.K, wl.r) + 2 * M * lin.K * wl.r for lin, *_ in state)
+    out["llama33b_block"] = {"what": "7 linears (d=6656, ffn=17920), M=2048, r=64: fwd saving XA, then bwd "
+                                     "recomputing XA and re-dequantizing W",
+                             "ms": round(ms, 4), "GFLOP": round(flops / 1e9, 1),
+                             **frac_tc(flops / (ms * 1e-3) / 1e12)}
+    del state, ws
+    torch.cuda.empty_cache()
     return out
 
 
@@ -547,7 +740,6 @@ def run_native(args, rank, world, local_rank):
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
-    err = binding.device_error()
 
     step_flops = sum(L.flops() for L in layers)
     value = step_flops * world / (ms * 1e-3) / 1e12
@@ -686,6 +878,10 @@ def run_native(args, rank, world, local_rank):
         e2e = {"value": step_flops * world / (ems * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ems,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
+    workloads = None
+    if rank == 0 and not args.no_workloads:
+        workloads = workload_phases(dev, hbm, tc)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl)
@@ -702,7 +898,8 @@ def run_native(args, rank, world, local_rank):
                                    f"linear_fwd on the first {SMALL_M} tokens"},
                 "phases": phases, "roofline": roofline, "gpu_launches": launches,
                 "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
-                "compare_dequant_then_library_gemm": compare, "device_error": err}
+                "compare_dequant_then_library_gemm": compare, "workloads": workloads,
+                "device_error": binding.device_error()}
         print(json.dumps(line), flush=True)
 
 

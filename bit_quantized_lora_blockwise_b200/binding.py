@@ -30,6 +30,7 @@ _STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_NULL", 2: "QLORA_ERR_SHAPE", 3: "QLORA_E
 
 # every symbol include/qlora.h declares
 EXPORTS = ("qlora_status_string", "qlora_abi_version", "qlora_nf4_levels", "qlora_dq_levels",
+           "qlora_int4_levels", "qlora_fp4_levels", "qlora_dq_signed_levels", "qlora_dq_dynamic_levels",
            "qlora_workspace_bytes", "qlora_quantize_nf4", "qlora_double_quant", "qlora_dequant",
            "qlora_linear_fwd", "qlora_linear_bwd", "qlora_device_error", "qlora_set_trace_events",
            "qlora_launch_count", "qlora_linear_fwd_noalloc", "qlora_selftest_bounded_wait")
@@ -59,8 +60,10 @@ def load(path: str | None = None):
         lib.qlora_status_string.argtypes = [I32]
         lib.qlora_status_string.restype = ctypes.c_char_p
         lib.qlora_abi_version.restype = I32
-        lib.qlora_nf4_levels.argtypes = [P]
-        lib.qlora_dq_levels.argtypes = [P]
+        for fn in ("qlora_nf4_levels", "qlora_dq_levels", "qlora_int4_levels", "qlora_fp4_levels",
+                   "qlora_dq_signed_levels", "qlora_dq_dynamic_levels"):
+            getattr(lib, fn).argtypes = [P]
+            getattr(lib, fn).restype = None
         lib.qlora_workspace_bytes.argtypes = [I64, I64, I64, I32]
         lib.qlora_workspace_bytes.restype = SZ
         lib.qlora_quantize_nf4.argtypes = [P, I64, I64, P, P, P, P]
@@ -154,6 +157,32 @@ def dq_levels() -> np.ndarray:
     out = (ctypes.c_float * 256)()
     load().qlora_dq_levels(out)
     return np.frombuffer(out, dtype=np.float32).copy()
+
+
+def _table(fn: str, n: int) -> np.ndarray:
+    out = (ctypes.c_float * n)()
+    getattr(load(), fn)(out)
+    return np.frombuffer(out, dtype=np.float32).copy()
+
+
+def int4_levels() -> np.ndarray:
+    """16 levels i / 7, i = -8..7 (absmax 4-bit integers), for the nf4= argument."""
+    return _table("qlora_int4_levels", 16)
+
+
+def fp4_levels() -> np.ndarray:
+    """The E2M1 values / 6 plus an unused top level, for the nf4= argument."""
+    return _table("qlora_fp4_levels", 16)
+
+
+def dq_signed_levels() -> np.ndarray:
+    """Signed linear 8-bit map (2k - 255) / 255, for the t8= argument."""
+    return _table("qlora_dq_signed_levels", 256)
+
+
+def dq_dynamic_levels() -> np.ndarray:
+    """Dynamic-exponent 8-bit map over [0, 1], for the t8= argument."""
+    return _table("qlora_dq_dynamic_levels", 256)
 
 
 def abi_version() -> int:

@@ -1,8 +1,8 @@
-// Warp-specialised tcgen05 GEMM for sm_100a, with an optional NF4-dequant
-// producer for the A operand and an optional low-rank (LoRA) product folded
+// Warp-specialised tcgen05 GEMM for sm_100a whose A operand is an NF4
+// weight tile dequantized on chip, with the low-rank (LoRA) product folded
 // into the same TMEM accumulator.
 //
-//   D[row, col] = sum_k A[row, k] B[col, k]   (+ sum_j A2[row, j] B2[col, j])
+//   D[row, col] = sum_k W'[row, k] B[col, k]  +  sum_j A2[row, j] B2[col, j]
 //
 // The QLoRA layer (intvml.com "DL0087 QLoRA", Figure 1: the NF4 weight is
 // dequantized to a bf16 tile just before the matmul and discarded) maps
@@ -12,20 +12,49 @@
 // A is rebuilt from the packed codes by "producer" warps that write bf16
 // straight into the 128-byte-swizzled shared-memory layout the tensor core
 // reads (K-major rows of W for the forward, MN-major for the backward); no
-// bf16 copy of W ever reaches global memory. The same kernel, with A and B
-// both loaded by TMA and fp32 split-K partials as output, computes the
-// skinny adapter products (X A, dY B^T, X^T G, dY^T XA).
+// bf16 copy of W ever reaches global memory. The token operand (X or dY) and
+// the low-rank operands arrive by TMA.
+//
+// CTA pairs (PAIR = true): a cluster of two CTAs on neighbouring SMs computes
+// a 256-row weight tile with the pair form of the MMA (cta_group::2). Each
+// CTA decodes its own 128 weight rows into its own A stage and loads half of
+// the tile's tokens into its own B stage; the leader (cluster rank 0) issues
+// M = 256 MMAs that read both CTAs' stages, and each CTA's TMEM receives its
+// own 128 rows over all the tile's tokens. Both CTAs' copies complete on the
+// leader's stage barrier (CTA-pair form of the TMA load, no multicast); the
+// peer's producers and epilogue arrive on the leader's barriers remotely; the
+// leader's commits release the stages and accumulators of both CTAs.
+//
+// Token stages. On this part a TMA load costs about the same time whether it
+// moves 16 KB or 64 KB, so one B stage holds BKB consecutive 64-deep K blocks
+// of the CTA's tokens, fetched by one 3-D box (the token operand viewed as
+// {64, tokens, K/64}); the MMAs of BKB jobs read it before it is released.
+// Low-rank K blocks take one B stage each (two 2-D boxes: B2 and A2).
+//
+// Token sub-tiles (NTT). Every 64-deep job has fixed costs (a decoded tile
+// handed from the producers to the MMA thread, a stage released, barrier
+// round trips) that on this part take about as long as the four MMAs of a
+// 256-token tile. With NTT = 2 each decoded weight tile feeds the MMAs of two
+// 256-token sub-tiles, one TMEM accumulator each (the whole 512 columns), so
+// those costs and the decode are spread over twice the FLOPs. The two
+// accumulators are then not double-buffered across tiles; instead each has
+// its own full/empty barriers, the epilogue drains sub-tile 0 first, and the
+// next tile's sub-tile-0 MMAs start while sub-tile 1 is still being drained.
+// Each CTA loads NTT x B_ROWS consecutive tokens; accumulator column c of
+// sub-tile t holds token col0 + (c / B_ROWS) NTT B_ROWS + t B_ROWS + c % B_ROWS.
 //
 // Roles (one CTA per SM, persistent over output tiles):
 //   warps 0-3  epilogue: TMEM -> registers -> global (lane quadrant = warp)
-//   warp 4     TMA issue (one lane)
-//   warp 5     TMEM allocation + MMA issue (one lane)
-//   warps 6..  dequant producers (NPW warps, in groups of 4 that take turns)
-// Pipeline: STAGES shared-memory stages guarded by mbarriers (tma_full,
-// deq_full, empty); two TMEM accumulators (tmem_full, tmem_empty) so the
-// epilogue of one tile overlaps the mainloop of the next. Every wait is
-// bounded (mbar_wait); on a timeout the CTA drains its own copies and MMAs,
-// frees TMEM and returns with the device error word set.
+//   warp 4     TMA issue for the B ring and the low-rank operands (one lane)
+//   warp 5     TMEM allocation + MMA issue (one lane of the leader)
+//   warp 6     TMA issue for the packed-code ring (one lane)
+//   warps 7..  dequant producers (NPW warps, in groups of 4 that take turns)
+// Rings (mbarrier-guarded): B (SB stages), dequantized A (SA stages, one per
+// 64-deep job), packed codes + block constants (SP slots of KSUP jobs); two
+// TMEM accumulators (tmem_full, tmem_empty) so the epilogue of one tile
+// overlaps the mainloop of the next. Every wait is bounded (mbar_wait); on a
+// timeout the CTA drains its own copies and MMAs, frees TMEM and returns with
+// the device error word set.
 #pragma once
 
 #include "codec.cuh"
@@ -33,59 +62,54 @@
 
 namespace qlora {
 
-enum : int { A_TMA_K = 0, A_TMA_MN = 1, A_DEQ_K = 2, A_DEQ_MN = 3 };
-enum : int { B_TMA_K = 0, B_TMA_MN = 1 };
-enum : int { L2_NONE = 0, L2_A_MN = 1, L2_A_K = 2 };  // A2 major-ness (B2 is K-major)
+enum : int { A_DEQ_K = 2, A_DEQ_MN = 3 };
+enum : int { L2_A_MN = 1, L2_A_K = 2 };  // A2 major-ness (B2 is K-major)
 
 struct GemmArgs {
-  CUtensorMap tm_a;   // A operand (TMA variants)
-  CUtensorMap tm_b;   // B operand
-  CUtensorMap tm_pk;  // packed NF4 codes (dequant variants)
+  CUtensorMap tm_b;   // token operand viewed as {64, tokens, kdim / 64}: box {64, B_ROWS, BKB}
+  CUtensorMap tm_pk;  // packed NF4 codes
   CUtensorMap tm_a2;  // low-rank A2
-  CUtensorMap tm_b2;  // low-rank B2
-  CUtensorMap tm_cp;  // decoded block constants c' [K/64][N] fp32 (dequant variants)
-  // Output: bf16 out[row * out_ld + col] (transpose = 0) or
-  // out[col * out_ld + row] (transpose = 1), times out_scale; optionally a
-  // second copy out2 (same layout, out2_ld) times out2_scale.
+  CUtensorMap tm_b2;  // low-rank B2 [tokens, r]: box {64, B_ROWS}
+  CUtensorMap tm_cp;  // decoded block constants c' [K/64][N] fp32
+  // Output: bf16 out[col * out_ld + row] (the transposed tile).
   void *out;
-  void *out2;
   int64_t out_ld;
-  int64_t out2_ld;
   float *part;             // fp32 split-K partials [splits][rows_pad][cols_pad] (splits > 1)
   unsigned int *counters;  // one per output tile; zero on entry, left zero (splits > 1)
-  int64_t w_kblocks;      // 64-blocks per weight row (K / 64)
-  int rows;               // extent of the 128-row MMA dimension
-  int cols;               // extent of the BN-column MMA dimension
+  int rows;               // extent of the weight-row MMA dimension
+  int cols;               // extent of the token MMA dimension
   int kblocks;            // 64-deep K blocks of the main product
   int splits;             // split-K count (> 1: partials reduced by the last CTA of a tile)
   int lora_kblocks;       // 64-deep K blocks of the low-rank product (last split only)
-  int w_rows;             // A_DEQ_K: rows of W (N)
-  float out_scale;
-  float out2_scale;
-  int transpose;
   float nf4[16];
 };
 
-template <int BN_, int ASRC_, int BSRC_, int L2_, int SB_, int SA_, int SP_, int NPW_>
+template <int BN_, int ASRC_, int L2_, int BKB_, int SB_, int SA_, int SP_, int NPW_, bool PAIR_, int NTT_ = 1>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 64, BN = BN_;
-  static constexpr int ASRC = ASRC_, BSRC = BSRC_, L2 = L2_;
-  static constexpr int SB = SB_, SA = SA_, SP = SP_, NPW = NPW_;
-  static constexpr bool DEQ = ASRC_ >= A_DEQ_K;
-  static constexpr bool A_MN = (ASRC_ == A_TMA_MN) || (ASRC_ == A_DEQ_MN);
-  static constexpr bool B_MN = BSRC_ == B_TMA_MN;
-  static constexpr int NGROUPS = NPW_ >= 4 ? NPW_ / 4 : 1;
-  static_assert(!DEQ || (NPW_ % 4 == 0 && NPW_ >= 4 && SP_ >= 2), "dequant needs producer groups and a P ring");
-  static_assert(DEQ || (SA_ == SB_ && SP_ == 0 && NPW_ == 0), "TMA-only A shares the B ring");
-  // (a 16-warp, 3-slot configuration timed out on B200: keep a slot per
-  // producer group and one spare)
-  static_assert(!DEQ || SA_ > NPW_ / 4, "dequantized-tile ring needs more slots than producer groups");
-  static_assert(DEQ || L2_ == L2_NONE, "low-rank steps only in the dequant variants");
-  static_assert(BN_ % 16 == 0 && BN_ >= 16 && BN_ <= 256, "MMA N");
+  static constexpr int ASRC = ASRC_, L2 = L2_;
+  static constexpr int BKB = BKB_, SB = SB_, SA = SA_, SP = SP_, NPW = NPW_;
+  static constexpr bool PAIR = PAIR_;
+  static constexpr int NTT = NTT_;                 // token sub-tiles (accumulators) per job
+  static constexpr int NCTA = PAIR_ ? 2 : 1;       // CTAs per tile
+  static constexpr int TILE_ROWS = 128 * NCTA;     // weight rows per tile
+  static constexpr int TILE_COLS = BN_ * NTT_;     // tokens per tile
+  static constexpr int B_ROWS = BN_ / NCTA;        // tokens of one sub-tile this CTA loads
+  static constexpr int CTA_TOK = B_ROWS * NTT_;    // tokens of the tile this CTA loads
+  static_assert(NTT_ == 1 || NTT_ == 2, "one or two token sub-tiles");
+  static_assert(CTA_TOK <= 256, "a TMA box spans at most 256 tokens");
+  static constexpr bool A_MN = ASRC_ == A_DEQ_MN;
+  static constexpr int NGROUPS = NPW_ / 4;
+  static_assert(NPW_ % 4 == 0 && NPW_ >= 4 && SP_ >= 2, "producer groups of 4 warps and a packed-code ring");
+  // (a 16-warp, 3-slot configuration timed out on B200: every producer group
+  // needs a slot of its own plus a spare, or the groups wait on each other)
+  static_assert(SA_ > NPW_ / 4, "dequantized-tile ring needs more slots than producer groups");
+  static_assert(BN_ % 16 == 0 && BN_ >= 16 && BN_ <= 256 && B_ROWS % 8 == 0, "MMA N");
+  static_assert(BKB_ >= 1 && BKB_ <= 4, "K blocks per token stage");
   static constexpr int NCHUNK = (BN_ + 31) / 32;  // epilogue chunks of 32 columns (last may hold 16)
-  static_assert(!B_MN || BN_ % 64 == 0, "MN-major B needs whole 64-wide chunks");
-  static constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int A_BYTES = BM * BK * 2;     // 16 KB
+  static constexpr int KB_BYTES = CTA_TOK * BK * 2;  // one K block of this CTA's tokens
+  static constexpr int B_BYTES = KB_BYTES * BKB;
   // P slot: the packed codes of KSUP consecutive 64-deep K blocks of the
   // 128-row weight tile (128 contiguous bytes per weight row: forward;
   // 64 bytes of 4 x 64 rows: backward), then their 4 x 128 decoded block
@@ -104,38 +128,44 @@ struct GemmCfg {
   // misc: tmem base, abort flag, last-CTA flag (16 B), then the 16 NF4 levels
   static constexpr int OFF_MISC = ((OFF_BAR + NBARS * 8) + 15) & ~15;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 64;
-  static constexpr int WARPS = DEQ ? 7 + NPW_ : 6;
+  static constexpr int WARPS = 7 + NPW_;
   static constexpr int THREADS = WARPS * 32;
+  // two accumulators of BN columns: double-buffered tiles (NTT = 1) or the
+  // two sub-tiles of one tile (NTT = 2)
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64
                                         : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
   static constexpr uint32_t ACC_STRIDE = TMEM_COLS / 2;  // column offset of accumulator 1
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-  static constexpr uint32_t MAIN_TX = B_BYTES + (DEQ ? 0 : A_BYTES);
-  static constexpr uint32_t LORA_TX = A_BYTES + B_BYTES;
+  // bytes the (leader's) stage barrier expects: both CTAs' copies for a pair
+  static constexpr uint32_t MAIN_TX = B_BYTES * NCTA;
+  static constexpr uint32_t LORA_TX = (A_BYTES + KB_BYTES) * NCTA;
+  static constexpr uint32_t GROUP_ARRIVALS = 4 * NCTA;  // a_full / tmem_empty: 4 warps per CTA
 };
 
 struct TileCoord {
-  int row0, col0, split, rc, kb_begin, nmain, nlora;  // rc: (row tile, col tile) index
+  int row0, col0, split, rc, kb_begin, nmain, nlora;  // rc: (128-row tile, col tile) index
 };
 
+// Tile `tile` of a grid of row_tiles x col_tiles tiles of (128 ncta) rows x
+// BN columns per split; row0 is the first of this CTA's 128 rows (`rank` in
+// the pair).
 __device__ __forceinline__ TileCoord tile_coord(const GemmArgs &a, int tile, int row_tiles,
-                                                int col_tiles, int BN) {
+                                                int col_tiles, int tile_cols, int ncta, int rank) {
   TileCoord t;
   const int per_split = row_tiles * col_tiles;
   t.split = tile / per_split;
   const int rem = tile - t.split * per_split;
-  t.rc = rem;
   const int rt = rem / col_tiles;
   const int ct = rem - rt * col_tiles;
-  t.row0 = rt * 128;
-  t.col0 = ct * BN;
+  t.rc = (rt * ncta + rank) * col_tiles + ct;
+  t.row0 = (rt * ncta + rank) * 128;
+  t.col0 = ct * tile_cols;
   t.kb_begin = static_cast<int>((static_cast<int64_t>(t.split) * a.kblocks) / a.splits);
   const int kb_end = static_cast<int>((static_cast<int64_t>(t.split + 1) * a.kblocks) / a.splits);
   t.nmain = kb_end - t.kb_begin;
   t.nlora = (t.split == a.splits - 1) ? a.lora_kblocks : 0;
   return t;
 }
-
 
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_constant__ GemmArgs args) {
@@ -165,7 +195,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
       mbar_init(b_empty(s), 1);
     }
     for (int s = 0; s < C::SA; ++s) {
-      mbar_init(a_full(s), 4);
+      mbar_init(a_full(s), C::GROUP_ARRIVALS);
       mbar_init(a_empty(s), 1);
     }
     for (int s = 0; s < C::SP; ++s) {
@@ -174,7 +204,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tmem_full(a), 1);
-      mbar_init(tmem_empty(a), 4);
+      mbar_init(tmem_empty(a), C::GROUP_ARRIVALS);
     }
     mbar_init(drain_bar, 1);
     *s_abort = 0;
@@ -183,85 +213,108 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
   if (threadIdx.x < 16) reinterpret_cast<float *>(smem + C::OFF_MISC + 16)[threadIdx.x] = args.nf4[threadIdx.x];
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&args.tm_b);
-    if (!C::DEQ) tma_prefetch_desc(&args.tm_a);
-    if (C::L2 != L2_NONE) {
-      tma_prefetch_desc(&args.tm_a2);
-      tma_prefetch_desc(&args.tm_b2);
-    }
+    tma_prefetch_desc(&args.tm_a2);
+    tma_prefetch_desc(&args.tm_b2);
   }
-  if (C::DEQ && warp == 6 && lane == 0) {
+  if (warp == 6 && lane == 0) {
     tma_prefetch_desc(&args.tm_pk);
     tma_prefetch_desc(&args.tm_cp);
   }
   if (warp == 5) {
-    tmem_alloc(smem_u32(s_tmem), C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (C::PAIR) {
+      tmem_alloc_pair(smem_u32(s_tmem), C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(s_tmem), C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  // a pair: both CTAs' barriers are initialised (and their TMEM allocated)
+  // before either CTA's copies, arrivals or commits reach the other
+  if constexpr (C::PAIR) cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
+  // pair rank (0 = leader, which issues the MMAs)
+  const uint32_t rank = C::PAIR ? cluster_ctarank() : 0u;
+  // Arrivals on barriers the leader waits on. In a pair the arriving thread
+  // signals that its own CTA's shared memory (a decoded A half) or TMEM (an
+  // accumulator half it has read) is ready; only its own SM's tensor core
+  // touches that memory next, so the arrival carries the default CTA-scope
+  // release. (A cluster-scope release here cost a third of the kernel's
+  // throughput on B200.)
+  auto arrive_leader = [&](uint32_t bar) {
+    if constexpr (C::PAIR) mbar_arrive_remote(map_cluster(bar, 0u));
+    else mbar_arrive(bar);
+  };
+  auto wait_warp = [&](uint32_t bar, uint32_t par) -> bool {
+    return __all_sync(0xFFFFFFFFu, mbar_wait(bar, par, s_abort));
+  };
   // everything above overlaps the previous kernel's tail; its outputs are
   // read only below
   grid_dep_wait();
   grid_dep_launch();
 
-  const int row_tiles = (args.rows + 127) / 128;
-  const int col_tiles = (args.cols + C::BN - 1) / C::BN;
+  // tiles of TILE_ROWS weight rows x BN tokens; a pair (cluster) takes every
+  // (number of pairs)-th tile
+  const int row_tiles = (args.rows + C::TILE_ROWS - 1) / C::TILE_ROWS;
+  const int col_tiles = (args.cols + C::TILE_COLS - 1) / C::TILE_COLS;
   const int num_tiles = row_tiles * col_tiles * args.splits;
+  const int first_tile = static_cast<int>(blockIdx.x) / C::NCTA;
+  const int tile_step = static_cast<int>(gridDim.x) / C::NCTA;
+  auto coord = [&](int tile) { return tile_coord(args, tile, row_tiles, col_tiles, C::TILE_COLS, C::NCTA, rank); };
 
   if (warp == 4) {
-    // ---------------------------------------- TMA: B ring (and A when TMA) --
+    // --------------------------------- TMA: token stages, low-rank operands --
     if (lane == 0) {
-      uint32_t job = 0;
+      uint32_t job = 0, bs = 0;  // A-ring job and B-ring stage counters
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        const TileCoord t = tile_coord(args, tile, row_tiles, col_tiles, C::BN);
-        const int njobs = t.nmain + t.nlora;
-        for (int jj = 0; jj < njobs; ++jj, ++job) {
-          const int sb = job % C::SB;
-          if (!mbar_wait(b_empty(sb), ((job / C::SB) & 1u) ^ 1u, s_abort)) { ok = false; break; }
+      // one stage load: into this CTA's slot, counted on the leader's barrier
+      auto load = [&](uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
+        if constexpr (C::PAIR) tma_load_2d_pair(dst, map, map_cluster(bar, 0u), x, y);
+        else tma_load_2d(dst, map, bar, x, y);
+      };
+      for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
+        const TileCoord t = coord(tile);
+        const int nbm = (t.nmain + C::BKB - 1) / C::BKB;
+        for (int st = 0; st < nbm + t.nlora; ++st, ++bs) {
+          const int sb = bs % C::SB;
+          if (!mbar_wait(b_empty(sb), ((bs / C::SB) & 1u) ^ 1u, s_abort)) { ok = false; break; }
           const uint32_t b_dst = sbase + C::OFF_B + sb * C::B_BYTES;
-          if (jj < t.nmain) {
-            const int kb = t.kb_begin + jj;
-            mbar_arrive_expect_tx(b_full(sb), C::MAIN_TX);
-            if (C::BSRC == B_TMA_K) {
-              tma_load_2d(b_dst, &args.tm_b, b_full(sb), kb * 64, t.col0);
-            } else {
-#pragma unroll
-              for (int c = 0; c < C::BN / 64; ++c)
-                tma_load_2d(b_dst + c * 8192, &args.tm_b, b_full(sb), t.col0 + c * 64, kb * 64);
-            }
-            if (!C::DEQ) {  // A shares the B ring slot index
-              const uint32_t a_dst = sbase + C::OFF_A + sb * C::A_BYTES;
-              if (C::ASRC == A_TMA_K) {
-                tma_load_2d(a_dst, &args.tm_a, b_full(sb), kb * 64, t.row0);
-              } else {
-                tma_load_2d(a_dst, &args.tm_a, b_full(sb), t.row0, kb * 64);
-                tma_load_2d(a_dst + 8192, &args.tm_a, b_full(sb), t.row0 + 64, kb * 64);
-              }
-            }
+          if (st < nbm) {
+            // BKB K blocks of this CTA's tokens, one 3-D box
+            if (rank == 0) mbar_arrive_expect_tx(b_full(sb), C::MAIN_TX);
+            const int kb = t.kb_begin + st * C::BKB;
+            const int tok = t.col0 + static_cast<int>(rank) * C::CTA_TOK;
+            if constexpr (C::PAIR) tma_load_3d_pair(b_dst, &args.tm_b, map_cluster(b_full(sb), 0u), 0, tok, kb);
+            else tma_load_3d(b_dst, &args.tm_b, b_full(sb), 0, tok, kb);
+            job += (st + 1 < nbm) ? C::BKB : t.nmain - st * C::BKB;
           } else {
-            // low-rank step: A2 into the A ring slot of this job, B2 into B
-            const int lk = jj - t.nmain;
+            // low-rank K block: B2 into the stage, A2 into this job's A slot
+            const int lk = st - nbm;
             const int sa = job % C::SA;
             if (!mbar_wait(a_empty(sa), ((job / C::SA) & 1u) ^ 1u, s_abort)) { ok = false; break; }
             const uint32_t a_dst = sbase + C::OFF_A + sa * C::A_BYTES;
-            mbar_arrive_expect_tx(b_full(sb), C::LORA_TX);
-            tma_load_2d(b_dst, &args.tm_b2, b_full(sb), lk * 64, t.col0);
+            if (rank == 0) mbar_arrive_expect_tx(b_full(sb), C::LORA_TX);
+            load(b_dst, &args.tm_b2, b_full(sb), lk * 64, t.col0 + static_cast<int>(rank) * C::CTA_TOK);
             if (C::L2 == L2_A_MN) {
-              tma_load_2d(a_dst, &args.tm_a2, b_full(sb), t.row0, lk * 64);
-              tma_load_2d(a_dst + 8192, &args.tm_a2, b_full(sb), t.row0 + 64, lk * 64);
+              load(a_dst, &args.tm_a2, b_full(sb), t.row0, lk * 64);
+              load(a_dst + 8192, &args.tm_a2, b_full(sb), t.row0 + 64, lk * 64);
             } else {
-              tma_load_2d(a_dst, &args.tm_a2, b_full(sb), lk * 64, t.row0);
+              load(a_dst, &args.tm_a2, b_full(sb), lk * 64, t.row0);
             }
+            ++job;
           }
         }
       }
-      // wait (bounded) for this thread's copies still in flight
-      const uint32_t inflight = job < (uint32_t)C::SB ? job : (uint32_t)C::SB;
+      // wait (bounded) for this thread's copies still in flight (a pair's
+      // copies complete on the leader's barriers, which count both halves;
+      // the peer stays resident until the leader is past this point: the
+      // cluster barrier at the end)
+      const uint32_t inflight = rank != 0 ? 0u : (bs < (uint32_t)C::SB ? bs : (uint32_t)C::SB);
       for (uint32_t i = 0; i < inflight; ++i) {
-        const uint32_t jb = job - 1 - i;
+        const uint32_t jb = bs - 1 - i;
         const unsigned long long t0 = globaltimer_ns();
         while (!mbar_try_wait(b_full(jb % C::SB), (jb / C::SB) & 1u)) {
           if (globaltimer_ns() - t0 > kWaitTimeoutNs) break;
@@ -271,56 +324,79 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     __syncwarp();
   } else if (warp == 5) {
     // ------------------------------------------------------ MMA issue --
-    // One thread issues every MMA of the CTA, so this loop is kept lean: the
-    // fixed bits of both descriptor layouts and both instruction descriptors
-    // are formed once, and each MMA only adds its K offset to the start
-    // address field.
-    if (lane == 0) {
+    // One thread issues every MMA of the CTA (of the pair: the leader's),
+    // so this loop is kept lean: the fixed bits of both descriptor layouts
+    // and both instruction descriptors are formed once, and each MMA only
+    // adds its K offset to the start address field. A pair's MMAs read both
+    // CTAs' stages (same offsets), so the leader's barriers count both CTAs'
+    // copies and producers, and its commits release the stage in both CTAs
+    // (mask 0b11).
+    if (lane == 0 && rank == 0) {
       constexpr uint64_t DK = smem_desc_const(16, 1024);    // K-major, 128B swizzle
       constexpr uint64_t DM = smem_desc_const(8192, 1024);  // MN-major, 128B swizzle
-      constexpr uint32_t ID_MAIN = make_idesc_bf16(128, C::BN, C::A_MN ? 1 : 0, C::B_MN ? 1 : 0);
-      constexpr uint32_t ID_LORA = make_idesc_bf16(128, C::BN, C::L2 == L2_A_MN ? 1 : 0, 0);
+      constexpr uint32_t ID_MAIN = make_idesc_bf16(C::TILE_ROWS, C::BN, C::A_MN ? 1 : 0, 0);
+      constexpr uint32_t ID_LORA = make_idesc_bf16(C::TILE_ROWS, C::BN, C::L2 == L2_A_MN ? 1 : 0, 0);
+      auto wait_full = [&](uint32_t bar, uint32_t par) -> bool {
+        return mbar_try_wait(bar, par) || mbar_wait(bar, par, s_abort);
+      };
+      auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t id, uint32_t accum) {
+        if constexpr (C::PAIR) tc_mma_ss_pair(d, ad, bd, id, accum);
+        else tc_mma_ss(d, ad, bd, id, accum);
+      };
+      auto commit = [&](uint32_t bar) {
+        if constexpr (C::PAIR) tc_commit_pair(bar, 0x3);
+        else tc_commit(bar);
+      };
       const uint32_t a_base = sbase + C::OFF_A, b_base = sbase + C::OFF_B;
-      uint32_t job = 0, iter = 0;
+      uint32_t job = 0, bs = 0, iter = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++iter) {
-        const TileCoord t = tile_coord(args, tile, row_tiles, col_tiles, C::BN);
+      for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step, ++iter) {
+        const TileCoord t = coord(tile);
         const int njobs = t.nmain + t.nlora;
-        const int acc = iter & 1;
-        if (!mbar_wait(tmem_empty(acc), ((iter >> 1) & 1u) ^ 1u, s_abort)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * C::ACC_STRIDE;
-        int sb = job % C::SB, sa = C::DEQ ? (int)(job % C::SA) : sb;
-        uint32_t pb = (job / C::SB) & 1u, pa = (job / C::SA) & 1u;
+        // accumulator use u = iter * NTT + sub-tile: accumulator u & 1, phase u >> 1
+        const uint32_t u0 = iter * C::NTT;
+        int sa = job % C::SA;
+        uint32_t pa = (job / C::SA) & 1u;
         for (int jj = 0; jj < njobs; ++jj, ++job) {
-          if (!mbar_try_wait(b_full(sb), pb) && !mbar_wait(b_full(sb), pb, s_abort)) { ok = false; break; }
-          if (C::DEQ && !mbar_try_wait(a_full(sa), pa) && !mbar_wait(a_full(sa), pa, s_abort)) { ok = false; break; }
-          tc_fence_after();
           const bool main_job = jj < t.nmain;
+          const int sub = main_job ? jj % C::BKB : 0;  // K block within the token stage
+          const bool last_of_stage = !main_job || sub == C::BKB - 1 || jj == t.nmain - 1;
+          const int sb = bs % C::SB;
+          if (sub == 0 && !wait_full(b_full(sb), (bs / C::SB) & 1u)) { ok = false; break; }
+          if (!wait_full(a_full(sa), pa)) { ok = false; break; }
+          tc_fence_after();
           const bool a_mn = main_job ? C::A_MN : (C::L2 == L2_A_MN);
-          const bool b_mn = main_job && C::B_MN;
           const uint64_t ad = (a_mn ? DM : DK) | (((a_base + sa * C::A_BYTES) >> 4) & 0x3FFFu);
-          const uint64_t bd = (b_mn ? DM : DK) | (((b_base + sb * C::B_BYTES) >> 4) & 0x3FFFu);
-          const uint32_t astep = a_mn ? 2048u >> 4 : 32u >> 4, bstep = b_mn ? 2048u >> 4 : 32u >> 4;
+          const uint64_t bd = DK | (((b_base + sb * C::B_BYTES + sub * C::KB_BYTES) >> 4) & 0x3FFFu);
+          const uint32_t astep = a_mn ? 2048u >> 4 : 32u >> 4, bstep = 32u >> 4;
           const uint32_t idesc = main_job ? ID_MAIN : ID_LORA;
-          tc_mma_ss(d_tmem, ad, bd, idesc, jj > 0 ? 1u : 0u);
-          tc_mma_ss(d_tmem, ad + astep, bd + bstep, idesc, 1u);
-          tc_mma_ss(d_tmem, ad + 2 * astep, bd + 2 * bstep, idesc, 1u);
-          tc_mma_ss(d_tmem, ad + 3 * astep, bd + 3 * bstep, idesc, 1u);
-          tc_commit(b_empty(sb));
-          if (C::DEQ) tc_commit(a_empty(sa));
-          if (++sb == C::SB) { sb = 0; pb ^= 1u; }
-          if (C::DEQ) {
-            if (++sa == C::SA) { sa = 0; pa ^= 1u; }
-          } else {
-            sa = sb;
+#pragma unroll
+          for (int st = 0; st < C::NTT; ++st) {
+            const uint32_t u = u0 + st;
+            if (jj == 0) {  // the accumulator's previous tile has been drained
+              if (!wait_full(tmem_empty(u & 1u), ((u >> 1) & 1u) ^ 1u)) { ok = false; break; }
+              tc_fence_after();
+            }
+            const uint32_t d_tmem = tmem_base + (u & 1u) * C::ACC_STRIDE;
+            const uint64_t bst = bd + ((st * C::B_ROWS * 128) >> 4);  // sub-tile st's tokens of the stage
+            mma(d_tmem, ad, bst, idesc, jj > 0 ? 1u : 0u);
+            mma(d_tmem, ad + astep, bst + bstep, idesc, 1u);
+            mma(d_tmem, ad + 2 * astep, bst + 2 * bstep, idesc, 1u);
+            mma(d_tmem, ad + 3 * astep, bst + 3 * bstep, idesc, 1u);
+            if (jj == njobs - 1) commit(tmem_full(u & 1u));  // this sub-tile's sum is complete
           }
+          if (!ok) break;
+          commit(a_empty(sa));
+          if (last_of_stage) {
+            commit(b_empty(sb));
+            ++bs;
+          }
+          if (++sa == C::SA) { sa = 0; pa ^= 1u; }
         }
-        if (!ok) break;
-        tc_commit(tmem_full(acc));
       }
       // all MMAs issued by this thread have completed once drain_bar flips
-      tc_commit(drain_bar);
+      if constexpr (C::PAIR) tc_commit_pair(drain_bar, 0x1);
+      else tc_commit(drain_bar);
       const unsigned long long t0 = globaltimer_ns();
       while (!mbar_try_wait(drain_bar, 0)) {
         if (globaltimer_ns() - t0 > kWaitTimeoutNs) break;
@@ -334,9 +410,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     // (atomic counter) sums the partials in split order (deterministic) and
     // writes the bf16 output.
     volatile int *s_last = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
-    const int64_t rows_pad = static_cast<int64_t>(row_tiles) * 128;
-    // partial rows are padded to whole 32-column chunks per tile
-    const int64_t cols_pad = static_cast<int64_t>(col_tiles) * C::NCHUNK * 32;
+    const int64_t rows_pad = static_cast<int64_t>(row_tiles) * C::TILE_ROWS;
+    // partial rows are padded to whole 32-column chunks per sub-tile
+    constexpr int TILE_PCOLS = C::NTT * C::NCHUNK * 32;
+    const int64_t cols_pad = static_cast<int64_t>(col_tiles) * TILE_PCOLS;
     uint32_t iter = 0;
     const int qrow = warp * 32 + lane;  // TMEM lane of this thread
     // chunk ch of the accumulator row (32 columns; a 16-column tail is zero-padded)
@@ -353,72 +430,55 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
         tmem_ld_32x32b_x32(tcol + ch * 32, u);
       }
     };
-    // col_end: first column past this tile (a 240-wide tile's last chunk
-    // must not spill into the next tile)
-    auto store_out = [&](int row, int col_base, int col_end, const float (&v)[32]) {
+    // out[token][row] for the 32 consecutive tokens from tok (clipped at the
+    // last token); each warp store covers 32 consecutive rows
+    auto store_out = [&](int row, int tok, const float (&v)[32]) {
       if (row >= args.rows) return;
-      const int lim = col_end < args.cols ? col_end : args.cols;
-      const int ncol = lim - col_base < 32 ? lim - col_base : 32;
-      for (int o = 0; o < 2; ++o) {
-        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(o ? args.out2 : args.out);
-        if (dst == nullptr) continue;
-        const float sc = o ? args.out2_scale : args.out_scale;
-        const int64_t ld = o ? args.out2_ld : args.out_ld;
-        if (args.transpose) {
+      const int ncol = args.cols - tok < 32 ? args.cols - tok : 32;
+      __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(args.out);
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j < ncol) dst[static_cast<int64_t>(col_base + j) * ld + row] = __float2bfloat16_rn(v[j] * sc);
-        } else if (ncol == 32) {
-          uint32_t w[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(v[2 * j] * sc, v[2 * j + 1] * sc);
-          uint4 *d4 = reinterpret_cast<uint4 *>(dst + static_cast<int64_t>(row) * ld + col_base);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) d4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j < ncol) dst[static_cast<int64_t>(row) * ld + col_base + j] = __float2bfloat16_rn(v[j] * sc);
-        }
-      }
+      for (int j = 0; j < 32; ++j)
+        if (j < ncol) dst[static_cast<int64_t>(tok + j) * args.out_ld + row] = __float2bfloat16_rn(v[j]);
     };
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++iter) {
-      const TileCoord t = tile_coord(args, tile, row_tiles, col_tiles, C::BN);
-      const int acc = iter & 1;
-      if (!warp_wait_all(tmem_full(acc), (iter >> 1) & 1u, s_abort)) break;
-      tc_fence_after();
+    bool ok = true;
+    for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step, ++iter) {
+      const TileCoord t = coord(tile);
       const int row = t.row0 + qrow;
-      const uint32_t tcol = tmem_base + ((uint32_t)(warp * 32) << 16) + acc * C::ACC_STRIDE;
-      if (args.splits == 1) {
+      // first token of chunk ch of sub-tile st (32 columns never straddle the CTA halves)
+      auto tok0 = [&](int st, int ch) {
+        const int c0 = ch * 32;
+        return t.col0 + (c0 / C::B_ROWS) * C::CTA_TOK + st * C::B_ROWS + c0 % C::B_ROWS;
+      };
+      float *prow = args.part + (static_cast<int64_t>(t.split) * rows_pad + row) * cols_pad +
+                    static_cast<int64_t>(t.col0 / C::TILE_COLS) * TILE_PCOLS;
+#pragma unroll 1
+      for (int st = 0; st < C::NTT; ++st) {
+        const uint32_t u = iter * C::NTT + st;
+        if (!wait_warp(tmem_full(u & 1u), (u >> 1) & 1u)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tcol = tmem_base + ((uint32_t)(warp * 32) << 16) + (u & 1u) * C::ACC_STRIDE;
 #pragma unroll 1
         for (int ch = 0; ch < C::NCHUNK; ++ch) {
-          uint32_t u[32];
-          load_chunk(tcol, ch, u);
-          float v[32];
+          uint32_t w[32];
+          load_chunk(tcol, ch, w);
+          if (args.splits == 1) {
+            float v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(u[j]);
-          store_out(row, t.col0 + ch * 32, t.col0 + C::BN, v);
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(w[j]);
+            store_out(row, tok0(st, ch), v);
+          } else {
+            float4 *o = reinterpret_cast<float4 *>(prow + (st * C::NCHUNK + ch) * 32);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              o[j] = make_float4(__uint_as_float(w[4 * j]), __uint_as_float(w[4 * j + 1]),
+                                 __uint_as_float(w[4 * j + 2]), __uint_as_float(w[4 * j + 3]));
+          }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(tmem_empty(acc));
-        continue;
+        if (lane == 0) arrive_leader(tmem_empty(u & 1u));  // accumulator free (its partial is in memory)
       }
-      float *prow = args.part + (static_cast<int64_t>(t.split) * rows_pad + row) * cols_pad +
-                    (t.col0 / C::BN) * (C::NCHUNK * 32);
-#pragma unroll 1
-      for (int ch = 0; ch < C::NCHUNK; ++ch) {
-        uint32_t u[32];
-        load_chunk(tcol, ch, u);
-        float4 *o = reinterpret_cast<float4 *>(prow + ch * 32);
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          o[j] = make_float4(__uint_as_float(u[4 * j]), __uint_as_float(u[4 * j + 1]),
-                             __uint_as_float(u[4 * j + 2]), __uint_as_float(u[4 * j + 3]));
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tmem_empty(acc));  // accumulator free: partial is in memory
+      if (!ok || args.splits == 1) continue;
       __threadfence();
       named_bar_sync(1, 128);
       if (warp == 0 && lane == 0) {
@@ -431,14 +491,14 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
       if (*s_last) {
         __threadfence();
 #pragma unroll 1
-        for (int ch = 0; ch < C::NCHUNK; ++ch) {
+        for (int pc = 0; pc < C::NTT * C::NCHUNK; ++pc) {
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = 0.0f;
           for (int sp = 0; sp < args.splits; ++sp) {
             const float4 *src = reinterpret_cast<const float4 *>(
                 args.part + (static_cast<int64_t>(sp) * rows_pad + row) * cols_pad +
-                (t.col0 / C::BN) * (C::NCHUNK * 32) + ch * 32);
+                static_cast<int64_t>(t.col0 / C::TILE_COLS) * TILE_PCOLS + pc * 32);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               const float4 x = __ldcg(src + j);
@@ -448,22 +508,21 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
               v[4 * j + 3] += x.w;
             }
           }
-          store_out(row, t.col0 + ch * 32, t.col0 + C::BN, v);
+          store_out(row, tok0(pc / C::NCHUNK, pc % C::NCHUNK), v);
         }
       }
     }
-  } else if constexpr (C::DEQ) {
-   if (warp == 6) {
+  } else if (warp == 6) {
     // ------------------------------------------------ P ring: TMA issue --
-    // Runs up to SP main K blocks ahead of the producers, gated only by them:
-    // the packed codes of the 128 x 64 weight tile and its 128 decoded block
-    // constants (c' is block-major, so they are one contiguous 512-byte row
-    // for the forward and two 256-byte rows for the backward).
+    // Runs up to SP superjobs ahead of the producers, gated only by them:
+    // the packed codes of the 128 x (64 KSUP) weight tile and its decoded
+    // block constants (c' is block-major, so they are contiguous 512-byte
+    // rows for the forward and 256-byte rows for the backward).
     if (lane == 0) {
       uint32_t ms = 0;  // superjob counter (KSUP main jobs each, per tile)
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        const TileCoord t = tile_coord(args, tile, row_tiles, col_tiles, C::BN);
+      for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
+        const TileCoord t = coord(tile);
         for (int u = 0; u * C::KSUP < t.nmain; ++u, ++ms) {
           const int sp = ms % C::SP;
           if (!mbar_wait(p_empty(sp), ((ms / C::SP) & 1u) ^ 1u, s_abort)) { ok = false; break; }
@@ -490,7 +549,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
       }
     }
     __syncwarp();
-   } else {
+  } else {
     // ------------------------------------------------ dequant producers --
     const int pw = warp - 7;
     const int group = pw >> 2;
@@ -499,20 +558,20 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     const uint32_t swz = p & 7;
     uint32_t job = 0, ms = 0;  // ms: superjob counter at the start of the tile
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-      const TileCoord t = tile_coord(args, tile, row_tiles, col_tiles, C::BN);
+    for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
+      const TileCoord t = coord(tile);
       const int njobs = t.nmain + t.nlora;
       const int nsup = (t.nmain + C::KSUP - 1) / C::KSUP;
       for (int jj = 0; jj < njobs; ++jj, ++job) {
         const bool main_job = jj < t.nmain;
         if ((int)(job % C::NGROUPS) != group) continue;
         const int sa = job % C::SA;
-        if (!warp_wait_all(a_empty(sa), ((job / C::SA) & 1u) ^ 1u, s_abort)) { ok = false; break; }
+        if (!wait_warp(a_empty(sa), ((job / C::SA) & 1u) ^ 1u)) { ok = false; break; }
         if (main_job) {
           const uint32_t my_ms = ms + jj / C::KSUP;
           const int sub = jj % C::KSUP;
           const int sp = my_ms % C::SP;
-          if (!warp_wait_all(p_full(sp), (my_ms / C::SP) & 1u, s_abort)) { ok = false; break; }
+          if (!wait_warp(p_full(sp), (my_ms / C::SP) & 1u)) { ok = false; break; }
           const uint8_t *pslot = smem + C::OFF_P + sp * C::P_BYTES;
           // The codes arrive swizzled (TMA 128-byte swizzle on 128-byte rows
           // for the forward, 64-byte swizzle on 64-byte rows for the
@@ -562,18 +621,21 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
           fence_proxy_async_smem();
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(a_full(sa));
+        if (lane == 0) arrive_leader(a_full(sa));
       }
       ms += nsup;
     }
-   }
   }
 
   tc_fence_before();
   __syncthreads();
+  // a pair: neither CTA frees its TMEM or exits while the other may still
+  // read its shared memory (the leader's MMAs) or signal its barriers
+  if constexpr (C::PAIR) cluster_sync();
   if (warp == 5) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (C::PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 

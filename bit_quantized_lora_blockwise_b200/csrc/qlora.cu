@@ -91,10 +91,16 @@ CodecTables make_tables(const float *nf4, const float *t8) {
 }
 
 // Bucket table of the exact bucketed encode (see BucketTable): false when
-// two midpoints fall inside one bucket (the binary search is used then).
-// Host float arithmetic here is IEEE binary32 with the same operation order
-// as the device (sum then halve; one fused multiply-add for the bucket).
+// a midpoint lies outside [-1, 1] (the buckets cover only the range of
+// x = w / c) or two midpoints fall inside one bucket; the binary search is
+// used then. Host float arithmetic here is IEEE binary32 with the same
+// operation order as the device (sum then halve; one fused multiply-add for
+// the bucket).
 bool build_buckets(const float *L, BucketTable *bt) {
+  for (int i = 0; i < 15; ++i) {
+    const float m = (L[i] + L[i + 1]) * 0.5f;
+    if (!(m >= -1.0f && m <= 1.0f)) return false;
+  }
   auto bucket = [](float x) {  // same arithmetic as nf4_code_bucket (|x| <= 1): (RNE(128 x + 128)) / 8
     const float y = std::fmaf(x, 128.0f, 128.0f + kBucketMagic);
     uint32_t a, b;
@@ -260,6 +266,22 @@ bool map_mnmajor(CUtensorMap *m, const void *p, int64_t inner, int64_t outer) {
   return make_map(m, p, MAP_BF16, inner, outer, inner * 2, 64, 64, SW_128B);
 }
 
+// Token operand T [tokens, kdim] bf16 viewed as {64, tokens, kdim/64} (k
+// within a 64-block, token, block): box {64, box_rows, bkb} lands as bkb
+// consecutive K-major 128-byte-swizzled [box_rows][64] tiles.
+bool map_tokens_3d(CUtensorMap *map, const void *T, int64_t tokens, int64_t kdim, uint32_t box_rows, uint32_t bkb) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(tokens), static_cast<cuuint64_t>(kdim / 64)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kdim) * 2, 128};
+  const cuuint32_t box[3] = {64, box_rows, bkb};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(T), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // X [M, K] bf16 viewed as {64, K/64, M} (k within a block, block, token):
 // box {64, 4, tokens} = four quantization blocks of K for every token row.
 bool map_x_blocks(CUtensorMap *map, const void *X, int64_t M, int64_t K, uint32_t tokens) {
@@ -277,7 +299,7 @@ bool map_x_blocks(CUtensorMap *map, const void *X, int64_t M, int64_t K, uint32_
 
 // ------------------------------------------------------- GEMM launcher --
 template <class C>
-qlora_status launch_gemm(const GemmArgs &args, int sms, cudaStream_t stream) {
+qlora_status launch_gemm(const GemmArgs &args, int sms, int pair_slots, cudaStream_t stream) {
   static std::once_flag once[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -287,11 +309,65 @@ qlora_status launch_gemm(const GemmArgs &args, int sms, cudaStream_t stream) {
                                     C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return QLORA_ERR_CUDA;
-  const int row_tiles = (args.rows + 127) / 128;
-  const int col_tiles = (args.cols + C::BN - 1) / C::BN;
+  const int row_tiles = (args.rows + C::TILE_ROWS - 1) / C::TILE_ROWS;
+  const int col_tiles = (args.cols + C::TILE_COLS - 1) / C::TILE_COLS;
   const int tiles = row_tiles * col_tiles * args.splits;
-  const int grid = tiles < sms ? tiles : sms;
-  return launch_pdl(qgemm_kernel<C>, grid, C::THREADS, C::SMEM_BYTES, stream, args);
+  if constexpr (!C::PAIR) {
+    const int grid = tiles < sms ? tiles : sms;
+    return launch_pdl(qgemm_kernel<C>, grid, C::THREADS, C::SMEM_BYTES, stream, args);
+  } else {
+    // persistent: one cluster of two CTAs per resident pair slot, at most one per tile
+    const int clusters = std::min(tiles, pair_slots);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, qgemm_kernel<C>, args);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  }
+}
+
+// Clusters of two CTAs of pair variant C that can be resident at once on
+// this device (asked of the runtime once per device; 0 if none or on error).
+template <class C>
+int resident_pairs() {
+  static std::once_flag once[kMaxDevices];
+  static int cached[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::call_once(once[dev], [&] {
+    int n = 0;
+    if (cudaFuncSetAttribute(qgemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2);
+      cfg.blockDim = dim3(C::THREADS);
+      cfg.dynamicSmemBytes = C::SMEM_BYTES;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 2;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void *>(qgemm_kernel<C>), &cfg) != cudaSuccess)
+        n = 0;
+    }
+    cudaGetLastError();
+    cached[dev] = n;
+  });
+  return cached[dev];
 }
 
 // Block constants c' = t8[q] * S, block-major [K/64][N] fp32 (GEMM operand
@@ -307,7 +383,8 @@ struct Shape {
 // One counter per output tile of any GEMM of the call (tiles are at least
 // 128 x 32).
 int64_t counters_needed(const Shape &s) {
-  const int64_t rows = std::max(std::max(cdiv(s.M, 128), cdiv(s.N, 128)), cdiv(s.K, 128));
+  // 128-row halves of the 256-row pair tiles included
+  const int64_t rows = std::max(std::max(cdiv(s.M, 128), 2 * cdiv(s.N, 256)), 2 * cdiv(s.K, 256));
   return rows * std::max<int64_t>(1, cdiv(s.M, 32));
 }
 
@@ -553,46 +630,89 @@ qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a
 }
 
 // -------------------------------------------------------- fused GEMMs --
+// The pair variants of the fused GEMM (256 weight rows x 256 tokens per
+// cluster of two CTAs): token stages of kPairBkb K blocks of 128 tokens
+// (one TMA box each), dequantized-weight stages of one K block (16 KB) and
+// packed-code slots of 4 K blocks (18 KB).
+constexpr int kPairBkb = 2, kPairSb = 3, kPairSa = 4, kPairSp = 2, kPairNpw = 8;
+using FwdPairCfg = GemmCfg<256, A_DEQ_K, L2_A_MN, kPairBkb, kPairSb, kPairSa, kPairSp, kPairNpw, true>;
+using BwdPairCfg = GemmCfg<256, A_DEQ_MN, L2_A_K, kPairBkb, kPairSb, kPairSa, kPairSp, kPairNpw, true>;
+// Two 256-token sub-tiles per job (512 tokens per tile, each CTA loading 256
+// of them): token stages of 2 K blocks (64 KB boxes), 3 dequantized-weight
+// stages, 2 packed-code slots (212 KB of shared memory).
+constexpr int kPair2Bkb = 2, kPair2Sb = 2, kPair2Sa = 3, kPair2Sp = 2, kPair2Npw = 8;
+using FwdPair2Cfg = GemmCfg<256, A_DEQ_K, L2_A_MN, kPair2Bkb, kPair2Sb, kPair2Sa, kPair2Sp, kPair2Npw, true, 2>;
+using BwdPair2Cfg = GemmCfg<256, A_DEQ_MN, L2_A_K, kPair2Bkb, kPair2Sb, kPair2Sa, kPair2Sp, kPair2Npw, true, 2>;
+// token counts from which a tile holds two 256-token sub-tiles
+constexpr int64_t kTwoSubtileTokens = 1024;
+// K blocks per token stage of the one-CTA variants: 32-token tiles take 4
+// (a 16 KB box), the 256-token fallback 1 (a 32 KB box).
+constexpr int single_bkb(int bn) { return bn == 32 ? 4 : 1; }
+
+// Resident pair slots for the fused GEMMs on this device (both variants have
+// the same shared memory and threads), 0 if the runtime reports none.
+int fused_pair_slots(int sms) {
+  const int n = std::min(std::min(resident_pairs<FwdPairCfg>(), resident_pairs<BwdPairCfg>()),
+                         std::min(resident_pairs<FwdPair2Cfg>(), resident_pairs<BwdPair2Cfg>()));
+  return std::min(n, sms / 2);
+}
+
 struct FusedPlan {
   int bn, splits;
+  bool pair;      // 256-row tiles over a cluster of two CTAs
+  int ntt;        // token sub-tiles of bn tokens per tile (pairs: 1 or 2)
+  int slots;      // persistent units: CTAs (one-CTA tiles) or clusters (pairs)
   size_t part_bytes;
+  // tokens one CTA loads per K block (the token operand's TMA box height)
+  uint32_t cta_tokens() const { return static_cast<uint32_t>(bn * ntt / (pair ? 2 : 1)); }
 };
 
-// Token tile: 32 for a few tokens; otherwise 256, or 240 when that needs
-// clearly fewer (rounds x width) of persistent CTA work.
-FusedPlan plan_fused(int64_t M, int64_t rows, int64_t kblocks, int sms) {
+// Token tile: 32 tokens (one CTA per 128 weight rows) for a few tokens;
+// otherwise 256 tokens on CTA pairs (256 weight rows), when the device can
+// hold them, else on single CTAs. K is split across CTAs (or pairs) when
+// there are fewer tiles than persistent units.
+FusedPlan plan_fused(int64_t M, int64_t rows, int64_t kblocks, int sms, int pair_slots) {
   FusedPlan p;
-  if (M <= 32) {
-    p.bn = 32;
-  } else {
-    const int64_t rt = cdiv(rows, 128);
-    const int64_t w256 = cdiv(rt * cdiv(M, 256), sms) * 256;
-    const int64_t w240 = cdiv(rt * cdiv(M, 240), sms) * 240;
-    // the narrower tile dequantizes 7 % more weight per FLOP: switch only for a clear gain
-    p.bn = w240 * 100 < w256 * 92 ? 240 : 256;
-  }
-  const int64_t tiles = cdiv(rows, 128) * cdiv(M, p.bn);
+  p.bn = M <= 32 ? 32 : 256;
+  p.pair = M > 32 && pair_slots > 0;
+  p.ntt = p.pair && M >= kTwoSubtileTokens ? 2 : 1;
+  p.slots = p.pair ? pair_slots : sms;
+  const int64_t tile_rows = p.pair ? 256 : 128;
+  const int64_t tile_cols = static_cast<int64_t>(p.bn) * p.ntt;
+  const int64_t tiles = cdiv(rows, tile_rows) * cdiv(M, tile_cols);
   int64_t splits = 1;
-  if (tiles < sms) {
-    splits = sms / tiles;
+  if (tiles < p.slots) {
+    splits = p.slots / tiles;
     if (splits > kblocks) splits = kblocks;
     if (splits < 1) splits = 1;
   }
   p.splits = static_cast<int>(splits);
-  p.part_bytes = p.splits > 1 ? align256(static_cast<size_t>(p.splits) * cdiv(rows, 128) * 128 *
-                                         cdiv(M, p.bn) * cdiv(p.bn, 32) * 32 * 4)
+  p.part_bytes = p.splits > 1 ? align256(static_cast<size_t>(p.splits) * cdiv(rows, tile_rows) * tile_rows *
+                                         cdiv(M, tile_cols) * p.ntt * cdiv(p.bn, 32) * 32 * 4)
                               : 0;
   return p;
 }
 
+// Partials bytes that any plan of this shape can need (the workspace size
+// must not depend on whether the pair variant turns out to be resident).
+size_t fused_part_bound(int64_t M, int64_t rows, int64_t kblocks, int sms) {
+  return std::max(plan_fused(M, rows, kblocks, sms, sms / 2).part_bytes,
+                  plan_fused(M, rows, kblocks, sms, 0).part_bytes);
+}
+
 template <int BN, int AS, int L2>
 qlora_status run_fused_bn(const GemmArgs &a, int sms, cudaStream_t st) {
-  // rings: activation tiles (SB), dequantized weight tiles (SA), packed codes + constants (SP);
+  // rings: token stages (SB), dequantized weight tiles (SA), packed codes + constants (SP);
   // a few tokens leave the tensor core idle, so that variant runs 12 dequant warps
   // (P slots hold 4 K blocks each; the few-token variant streams the packed
   // weight from DRAM, so its P ring is deeper)
-  constexpr int SB = BN > 64 ? 4 : 8, SA = BN > 64 ? 3 : 6, SP = BN > 64 ? 2 : 4, NPW = BN > 64 ? 8 : 12;
-  return launch_gemm<GemmCfg<BN, AS, B_TMA_K, L2, SB, SA, SP, NPW>>(a, sms, st);
+  constexpr int SB = BN > 64 ? 4 : 2, SA = BN > 64 ? 3 : 6, SP = BN > 64 ? 2 : 4, NPW = BN > 64 ? 8 : 12;
+  return launch_gemm<GemmCfg<BN, AS, L2, single_bkb(BN), SB, SA, SP, NPW, false>>(a, sms, 0, st);
+}
+
+template <class C>
+qlora_status run_fused_pair(const GemmArgs &a, int sms, int slots, cudaStream_t st) {
+  return launch_gemm<C>(a, sms, slots, st);
 }
 
 // ---------------------------------------------------- few-token forward --
@@ -660,11 +780,11 @@ WsLayout ws_layout(const Shape &s, int sms, bool backward) {
   w.cprime = cprime_bytes(s.N, s.K);
   if (!backward) {
     w.part = s.M <= kSmallmMaxTokens ? plan_smallm(s.M, s.N, s.K, sms, 0).part_bytes
-                                     : plan_fused(s.M, s.N, s.K / 64, sms).part_bytes;
+                                     : fused_part_bound(s.M, s.N, s.K / 64, sms);
     w.total = w.counters + w.mr + w.cprime + w.part;
   } else {
     // the skinny GEMMs reduce their split-K partials in shared memory
-    const size_t part = plan_fused(s.M, s.K, s.N / 64, sms).part_bytes;   // dX split-K
+    const size_t part = fused_part_bound(s.M, s.K, s.N / 64, sms);   // dX split-K
     w.part = part;
     w.total = w.counters + 2 * w.mr + w.cprime + w.part;
   }
@@ -756,6 +876,33 @@ void qlora_nf4_levels(float out[16]) {
 void qlora_dq_levels(float out[256]) {
   if (out == nullptr) return;
   for (int k = 0; k < 256; ++k) out[k] = static_cast<float>(k) / 255.0f;
+}
+
+void qlora_int4_levels(float out[16]) {
+  if (out == nullptr) return;
+  for (int i = 0; i < 16; ++i) out[i] = static_cast<float>(static_cast<double>(i - 8) / 7.0);
+}
+
+void qlora_fp4_levels(float out[16]) {
+  if (out == nullptr) return;
+  // E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit; +0 once; 8 pads the table
+  static const double v[16] = {-6.0, -4.0, -3.0, -2.0, -1.5, -1.0, -0.5, 0.0,
+                               0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, 8.0};
+  for (int i = 0; i < 16; ++i) out[i] = static_cast<float>(v[i] / 6.0);
+}
+
+void qlora_dq_signed_levels(float out[256]) {
+  if (out == nullptr) return;
+  for (int k = 0; k < 256; ++k) out[k] = static_cast<float>((2.0 * k - 255.0) / 255.0);
+}
+
+void qlora_dq_dynamic_levels(float out[256]) {
+  if (out == nullptr) return;
+  out[0] = 0.0f;
+  for (int k = 1; k < 256; ++k) {
+    const int j = 255 - k;  // j = 0 is the largest level, 1
+    out[k] = static_cast<float>(std::ldexp(1.0 - (j % 32) / 64.0, -(j / 32)));
+  }
 }
 
 size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
@@ -907,16 +1054,16 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   }
 
   // 2) Y^T[n, m] = W'[n, :] . X[m, :] + B^T[n, :] . xas[m, :]
-  const FusedPlan fp = plan_fused(M, N, K / 64, d.sms);
+  const FusedPlan fp = plan_fused(M, N, K / 64, d.sms, fused_pair_slots(d.sms));
+  const uint32_t b_rows = fp.cta_tokens();
+  const uint32_t bkb = static_cast<uint32_t>(!fp.pair ? single_bkb(fp.bn) : fp.ntt == 2 ? kPair2Bkb : kPairBkb);
   GemmArgs a;
   std::memset(&a, 0, sizeof a);
-  if (!map_kmajor(&a.tm_b, X, K, M, fp.bn) ||
+  if (!map_tokens_3d(&a.tm_b, X, M, K, b_rows, bkb) ||
       !make_map(&a.tm_pk, packed, MAP_U8, K / 2, N, K / 2, 128, 128, SW_128B) ||
       !make_map(&a.tm_cp, cprime, MAP_F32, N, K / 64, N * 4, 128, 4, SW_NONE) ||
-      !map_mnmajor(&a.tm_a2, B, N, r) || !map_kmajor(&a.tm_b2, xas, r, M, fp.bn))
+      !map_mnmajor(&a.tm_a2, B, N, r) || !map_kmajor(&a.tm_b2, xas, r, M, b_rows))
     return QLORA_ERR_CUDA;
-  a.w_kblocks = K / 64;
-  a.w_rows = static_cast<int>(N);
   a.rows = static_cast<int>(N);
   a.cols = static_cast<int>(M);
   a.kblocks = static_cast<int>(K / 64);
@@ -924,15 +1071,14 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   a.lora_kblocks = static_cast<int>(cdiv(r, 64));
   a.out = Y;
   a.out_ld = N;
-  a.out_scale = 1.0f;
-  a.transpose = 1;
   a.part = part;
   a.counters = counters;
   std::memcpy(a.nf4, nf4, sizeof a.nf4);
   trace_begin(cs);
-  st = fp.bn == 32    ? run_fused_bn<32, A_DEQ_K, L2_A_MN>(a, d.sms, cs)
-       : fp.bn == 240 ? run_fused_bn<240, A_DEQ_K, L2_A_MN>(a, d.sms, cs)
-                      : run_fused_bn<256, A_DEQ_K, L2_A_MN>(a, d.sms, cs);
+  st = fp.pair ? (fp.ntt == 2 ? run_fused_pair<FwdPair2Cfg>(a, d.sms, fp.slots, cs)
+                              : run_fused_pair<FwdPairCfg>(a, d.sms, fp.slots, cs))
+       : fp.bn == 32 ? run_fused_bn<32, A_DEQ_K, L2_A_MN>(a, d.sms, cs)
+                     : run_fused_bn<256, A_DEQ_K, L2_A_MN>(a, d.sms, cs);
   trace_end(cs);
   return st;
 }
@@ -983,16 +1129,16 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   }
 
   // 2) dX^T[k, m] = W'^T[k, :] . dY[m, :] + A[k, :] . Gs[m, :]
-  const FusedPlan fp = plan_fused(M, K, N / 64, d.sms);
+  const FusedPlan fp = plan_fused(M, K, N / 64, d.sms, fused_pair_slots(d.sms));
+  const uint32_t b_rows = fp.cta_tokens();
+  const uint32_t bkb = static_cast<uint32_t>(!fp.pair ? single_bkb(fp.bn) : fp.ntt == 2 ? kPair2Bkb : kPairBkb);
   GemmArgs a;
   std::memset(&a, 0, sizeof a);
-  if (!map_kmajor(&a.tm_b, dY, N, M, fp.bn) ||
+  if (!map_tokens_3d(&a.tm_b, dY, M, N, b_rows, bkb) ||
       !make_map(&a.tm_pk, packed, MAP_U8, K / 2, N, K / 2, 64, 256, SW_64B) ||
       !make_map(&a.tm_cp, cprime, MAP_F32, N, K / 64, N * 4, 256, 2, SW_NONE) ||
-      !map_kmajor(&a.tm_a2, A, r, K, 128) || !map_kmajor(&a.tm_b2, gs, r, M, fp.bn))
+      !map_kmajor(&a.tm_a2, A, r, K, 128) || !map_kmajor(&a.tm_b2, gs, r, M, b_rows))
     return QLORA_ERR_CUDA;
-  a.w_kblocks = K / 64;
-  a.w_rows = static_cast<int>(N);
   a.rows = static_cast<int>(K);
   a.cols = static_cast<int>(M);
   a.kblocks = static_cast<int>(N / 64);
@@ -1000,15 +1146,14 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   a.lora_kblocks = static_cast<int>(cdiv(r, 64));
   a.out = dX;
   a.out_ld = K;
-  a.out_scale = 1.0f;
-  a.transpose = 1;
   a.part = part;
   a.counters = counters;
   std::memcpy(a.nf4, nf4, sizeof a.nf4);
   trace_begin(cs);
-  st = fp.bn == 32    ? run_fused_bn<32, A_DEQ_MN, L2_A_K>(a, d.sms, cs)
-       : fp.bn == 240 ? run_fused_bn<240, A_DEQ_MN, L2_A_K>(a, d.sms, cs)
-                      : run_fused_bn<256, A_DEQ_MN, L2_A_K>(a, d.sms, cs);
+  st = fp.pair ? (fp.ntt == 2 ? run_fused_pair<BwdPair2Cfg>(a, d.sms, fp.slots, cs)
+                              : run_fused_pair<BwdPairCfg>(a, d.sms, fp.slots, cs))
+       : fp.bn == 32 ? run_fused_bn<32, A_DEQ_MN, L2_A_K>(a, d.sms, cs)
+                     : run_fused_bn<256, A_DEQ_MN, L2_A_K>(a, d.sms, cs);
   trace_end(cs);
   if (st != QLORA_OK) return st;
 

@@ -90,6 +90,26 @@ QLORA_API void qlora_nf4_levels(float out[16]);
 QLORA_API void qlora_dq_levels(float out[256]);
 
 /*
+ * Alternative code tables (host, no device work) for the comparison the
+ * pages make: 4-bit NormalFloat against the uniform 4-bit types it
+ * outperforms (promptingindex.com "Finetuning 65B Models on a Single GPU",
+ * section "4-bit NormalFloat"; intvml.com "DL0087 QLoRA", component 1).
+ * Each is an ordinary input of the calls below (a table swap):
+ *   qlora_int4_levels        i / 7 for i = -8..7 (absmax 4-bit integers; -8/7
+ *                            lies below -1 and is never the nearest level)
+ *   qlora_fp4_levels         the E2M1 values (0, 0.5, 1, 1.5, 2, 3, 4, 6 and
+ *                            negatives) / 6, +0 once, plus an unused 8/6
+ *   qlora_dq_signed_levels   (2k - 255) / 255: a signed linear 8-bit map
+ *   qlora_dq_dynamic_levels  0, then 2^-e (1 - m/64) for (e, m) = divmod(j, 32),
+ *                            j = 0..254, ascending: 8 octaves of 32 levels
+ * Every value is computed in double precision and rounded once to float.
+ */
+QLORA_API void qlora_int4_levels(float out[16]);
+QLORA_API void qlora_fp4_levels(float out[16]);
+QLORA_API void qlora_dq_signed_levels(float out[256]);
+QLORA_API void qlora_dq_dynamic_levels(float out[256]);
+
+/*
  * Bytes of scratch that qlora_linear_fwd / qlora_linear_bwd need for this
  * shape (the larger of the two). Returns 0 for shapes the calls reject.
  */

@@ -54,8 +54,14 @@ def test_status_strings(lib):
 
 def test_host_tables_match_oracle(lib):
     import oracle
+    from oracle import codebooks as cb
     assert np.array_equal(binding.nf4_levels(), oracle.nf4_levels())
     assert np.array_equal(binding.dq_levels(), oracle.dq_levels())
+    # the alternative tables, bit for bit (the +0 of FP4 included)
+    for got, want in ((binding.int4_levels(), cb.int4_levels()), (binding.fp4_levels(), cb.fp4_levels()),
+                      (binding.dq_signed_levels(), cb.dq_signed_levels()),
+                      (binding.dq_dynamic_levels(), cb.dq_dynamic_levels())):
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
 
 
 def _fake(addr=0x10000):

@@ -72,8 +72,10 @@ class Layer:
     (520, 384, 256, 16),     # three row tiles, K = 256
     (64, 128, 128, 128),     # rank 128
     (40, 256, 192, 256),     # rank 256 (four low-rank K blocks)
-    (2048, 4096, 512, 16),   # forward on 240-token tiles, 9 column tiles, no split
-    (2048, 512, 4096, 16),   # backward on 240-token tiles, no split
+    (2048, 4096, 512, 16),   # forward without split (512-token tiles of two sub-tiles)
+    (2048, 512, 4096, 16),   # backward without split
+    (1300, 768, 640, 32),    # two sub-tiles with a ragged last tile (276 tokens: the peer's half partly empty), split K
+    (1030, 256, 1536, 64),   # two sub-tiles, last tile of 6 tokens, split K
 ])
 def test_fwd_bwd_parity(M, N, K, r):
     L = Layer(M, N, K, r, seed=M * 7 + N + K + r)
