@@ -74,12 +74,19 @@ struct GemmArgs {
   // Output: bf16 out[col * out_ld + row] (the transposed tile).
   void *out;
   int64_t out_ld;
-  float *part;             // fp32 split-K partials [splits][rows_pad][cols_pad] (splits > 1)
-  unsigned int *counters;  // one per output tile; zero on entry, left zero (splits > 1)
+  float *part;             // fp32 partials of split tiles [tail_splits][tail tiles][tile columns][TILE_ROWS]
+  unsigned int *counters;  // one per split output tile; zero on entry, left zero
   int rows;               // extent of the weight-row MMA dimension
   int cols;               // extent of the token MMA dimension
   int kblocks;            // 64-deep K blocks of the main product
-  int splits;             // split-K count (> 1: partials reduced by the last CTA of a tile)
+  // Work units: the first full_tiles tiles whole, then every remaining tile
+  // cut either into its NTT token sub-tiles (tail_subtiles = NTT: disjoint
+  // outputs, each over the whole K) or into tail_splits K ranges (partials
+  // reduced by the last split of a tile to finish, in split order), so that
+  // the last, partial round of a persistent grid is spread over more CTAs.
+  int full_tiles;
+  int tail_splits;
+  int tail_subtiles;
   int lora_kblocks;       // 64-deep K blocks of the low-rank product (last split only)
   float nf4[16];
 };
@@ -143,27 +150,47 @@ struct GemmCfg {
 };
 
 struct TileCoord {
-  int row0, col0, split, rc, kb_begin, nmain, nlora;  // rc: (128-row tile, col tile) index
+  int row0, col0, rc, kb_begin, nmain, nlora;  // rc: (128-row tile, col tile) index
+  int split, nsplit, tail;  // K range split of nsplit (1: the whole K); tail: index among the split tiles
+  int only;                 // the one token sub-tile this unit computes, or -1 for all
 };
 
 // Tile `tile` of a grid of row_tiles x col_tiles tiles of (128 ncta) rows x
 // BN columns per split; row0 is the first of this CTA's 128 rows (`rank` in
 // the pair).
-__device__ __forceinline__ TileCoord tile_coord(const GemmArgs &a, int tile, int row_tiles,
+__device__ __forceinline__ TileCoord tile_coord(const GemmArgs &a, int unit, int row_tiles,
                                                 int col_tiles, int tile_cols, int ncta, int rank) {
   TileCoord t;
-  const int per_split = row_tiles * col_tiles;
-  t.split = tile / per_split;
-  const int rem = tile - t.split * per_split;
-  const int rt = rem / col_tiles;
-  const int ct = rem - rt * col_tiles;
+  int id;  // output tile
+  t.only = -1;
+  if (unit < a.full_tiles) {
+    id = unit;
+    t.split = 0;
+    t.nsplit = 1;
+    t.tail = -1;
+  } else if (a.tail_subtiles > 1) {
+    const int v = unit - a.full_tiles;
+    t.tail = v / a.tail_subtiles;
+    t.only = v - t.tail * a.tail_subtiles;
+    t.split = 0;
+    t.nsplit = 1;
+    id = a.full_tiles + t.tail;
+  } else {
+    const int v = unit - a.full_tiles;
+    t.tail = v / a.tail_splits;
+    t.split = v - t.tail * a.tail_splits;
+    t.nsplit = a.tail_splits;
+    id = a.full_tiles + t.tail;
+  }
+  const int rt = id / col_tiles;
+  const int ct = id - rt * col_tiles;
   t.rc = (rt * ncta + rank) * col_tiles + ct;
   t.row0 = (rt * ncta + rank) * 128;
   t.col0 = ct * tile_cols;
-  t.kb_begin = static_cast<int>((static_cast<int64_t>(t.split) * a.kblocks) / a.splits);
-  const int kb_end = static_cast<int>((static_cast<int64_t>(t.split + 1) * a.kblocks) / a.splits);
+  t.kb_begin = static_cast<int>((static_cast<int64_t>(t.split) * a.kblocks) / t.nsplit);
+  const int kb_end = static_cast<int>((static_cast<int64_t>(t.split + 1) * a.kblocks) / t.nsplit);
   t.nmain = kb_end - t.kb_begin;
-  t.nlora = (t.split == a.splits - 1) ? a.lora_kblocks : 0;
+  t.nlora = (t.split == t.nsplit - 1) ? a.lora_kblocks : 0;
   return t;
 }
 
@@ -260,7 +287,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
   // (number of pairs)-th tile
   const int row_tiles = (args.rows + C::TILE_ROWS - 1) / C::TILE_ROWS;
   const int col_tiles = (args.cols + C::TILE_COLS - 1) / C::TILE_COLS;
-  const int num_tiles = row_tiles * col_tiles * args.splits;
+  const int num_tiles = args.full_tiles + (row_tiles * col_tiles - args.full_tiles) *
+                                             (args.tail_subtiles > 1 ? args.tail_subtiles : args.tail_splits);
   const int first_tile = static_cast<int>(blockIdx.x) / C::NCTA;
   const int tile_step = static_cast<int>(gridDim.x) / C::NCTA;
   auto coord = [&](int tile) { return tile_coord(args, tile, row_tiles, col_tiles, C::TILE_COLS, C::NCTA, rank); };
@@ -377,6 +405,12 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
               if (!wait_full(tmem_empty(u & 1u), ((u >> 1) & 1u) ^ 1u)) { ok = false; break; }
               tc_fence_after();
             }
+            if (t.only >= 0 && st != t.only) {
+              // a sub-tile this unit leaves to another: its accumulator's
+              // phases still advance (nothing to drain, nothing written)
+              if (jj == njobs - 1) commit(tmem_full(u & 1u));
+              continue;
+            }
             const uint32_t d_tmem = tmem_base + (u & 1u) * C::ACC_STRIDE;
             const uint64_t bst = bd + ((st * C::B_ROWS * 128) >> 4);  // sub-tile st's tokens of the stage
             mma(d_tmem, ad, bst, idesc, jj > 0 ? 1u : 0u);
@@ -405,17 +439,24 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     __syncwarp();
   } else if (warp < 4) {
     // ------------------------------------------------------- epilogue --
-    // splits == 1: TMEM -> bf16 output directly. splits > 1: TMEM -> fp32
+    auto qrow_of = [](int w, int l) { return w * 32 + l; };
+    // A whole tile: TMEM -> bf16 output directly. A split tile: TMEM -> fp32
     // partial in global memory; the last of the tile's splits to arrive
     // (atomic counter) sums the partials in split order (deterministic) and
     // writes the bf16 output.
     volatile int *s_last = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
-    const int64_t rows_pad = static_cast<int64_t>(row_tiles) * C::TILE_ROWS;
     // partial rows are padded to whole 32-column chunks per sub-tile
     constexpr int TILE_PCOLS = C::NTT * C::NCHUNK * 32;
-    const int64_t cols_pad = static_cast<int64_t>(col_tiles) * TILE_PCOLS;
+    const int ntail = row_tiles * col_tiles - args.full_tiles;
+    // Partial of split sp of tail tile ti, column-major ([column][row]) so
+    // that the 32 threads of a warp (32 consecutive rows) store and load 128
+    // contiguous bytes: this thread's element of column c is part_col(..)[c * TILE_ROWS].
+    auto part_col = [&](int sp, int ti) {
+      return args.part + (static_cast<int64_t>(sp) * ntail + ti) * TILE_PCOLS * C::TILE_ROWS + rank * 128 +
+             qrow_of(warp, lane);
+    };
     uint32_t iter = 0;
-    const int qrow = warp * 32 + lane;  // TMEM lane of this thread
+    const int qrow = qrow_of(warp, lane);  // TMEM lane of this thread
     // chunk ch of the accumulator row (32 columns; a 16-column tail is zero-padded)
     auto load_chunk = [&](uint32_t tcol, int ch, uint32_t (&u)[32]) {
       if (C::BN % 32 == 16 && ch == C::NCHUNK - 1) {
@@ -449,41 +490,44 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
         const int c0 = ch * 32;
         return t.col0 + (c0 / C::B_ROWS) * C::CTA_TOK + st * C::B_ROWS + c0 % C::B_ROWS;
       };
-      float *prow = args.part + (static_cast<int64_t>(t.split) * rows_pad + row) * cols_pad +
-                    static_cast<int64_t>(t.col0 / C::TILE_COLS) * TILE_PCOLS;
+      float *pcol = t.nsplit > 1 ? part_col(t.split, t.tail) : nullptr;
 #pragma unroll 1
       for (int st = 0; st < C::NTT; ++st) {
         const uint32_t u = iter * C::NTT + st;
         if (!wait_warp(tmem_full(u & 1u), (u >> 1) & 1u)) { ok = false; break; }
         tc_fence_after();
+        if (t.only >= 0 && st != t.only) {  // computed by another unit
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) arrive_leader(tmem_empty(u & 1u));
+          continue;
+        }
         const uint32_t tcol = tmem_base + ((uint32_t)(warp * 32) << 16) + (u & 1u) * C::ACC_STRIDE;
 #pragma unroll 1
         for (int ch = 0; ch < C::NCHUNK; ++ch) {
           uint32_t w[32];
           load_chunk(tcol, ch, w);
-          if (args.splits == 1) {
+          if (t.nsplit == 1) {
             float v[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(w[j]);
             store_out(row, tok0(st, ch), v);
           } else {
-            float4 *o = reinterpret_cast<float4 *>(prow + (st * C::NCHUNK + ch) * 32);
+            float *o = pcol + static_cast<int64_t>((st * C::NCHUNK + ch) * 32) * C::TILE_ROWS;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              o[j] = make_float4(__uint_as_float(w[4 * j]), __uint_as_float(w[4 * j + 1]),
-                                 __uint_as_float(w[4 * j + 2]), __uint_as_float(w[4 * j + 3]));
+            for (int j = 0; j < 32; ++j) __stcg(o + j * C::TILE_ROWS, __uint_as_float(w[j]));
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) arrive_leader(tmem_empty(u & 1u));  // accumulator free (its partial is in memory)
       }
-      if (!ok || args.splits == 1) continue;
+      if (!ok || t.nsplit == 1) continue;
       __threadfence();
       named_bar_sync(1, 128);
       if (warp == 0 && lane == 0) {
         const unsigned int prev = atomicAdd(args.counters + t.rc, 1u);
-        const int last = prev == static_cast<unsigned int>(args.splits - 1);
+        const int last = prev == static_cast<unsigned int>(t.nsplit - 1);
         if (last) args.counters[t.rc] = 0u;  // every split has arrived: reset for the next use
         *s_last = last;
       }
@@ -495,18 +539,10 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-          for (int sp = 0; sp < args.splits; ++sp) {
-            const float4 *src = reinterpret_cast<const float4 *>(
-                args.part + (static_cast<int64_t>(sp) * rows_pad + row) * cols_pad +
-                static_cast<int64_t>(t.col0 / C::TILE_COLS) * TILE_PCOLS + pc * 32);
+          for (int sp = 0; sp < t.nsplit; ++sp) {
+            const float *src = part_col(sp, t.tail) + static_cast<int64_t>(pc * 32) * C::TILE_ROWS;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float4 x = __ldcg(src + j);
-              v[4 * j] += x.x;
-              v[4 * j + 1] += x.y;
-              v[4 * j + 2] += x.z;
-              v[4 * j + 3] += x.w;
-            }
+            for (int j = 0; j < 32; ++j) v[j] += __ldcg(src + j * C::TILE_ROWS);
           }
           store_out(row, tok0(pc / C::NCHUNK, pc % C::NCHUNK), v);
         }

@@ -311,7 +311,7 @@ qlora_status launch_gemm(const GemmArgs &args, int sms, int pair_slots, cudaStre
   if (attr_err != cudaSuccess) return QLORA_ERR_CUDA;
   const int row_tiles = (args.rows + C::TILE_ROWS - 1) / C::TILE_ROWS;
   const int col_tiles = (args.cols + C::TILE_COLS - 1) / C::TILE_COLS;
-  const int tiles = row_tiles * col_tiles * args.splits;
+  const int tiles = args.full_tiles + (row_tiles * col_tiles - args.full_tiles) * args.tail_splits;
   if constexpr (!C::PAIR) {
     const int grid = tiles < sms ? tiles : sms;
     return launch_pdl(qgemm_kernel<C>, grid, C::THREADS, C::SMEM_BYTES, stream, args);
@@ -658,7 +658,8 @@ int fused_pair_slots(int sms) {
 }
 
 struct FusedPlan {
-  int bn, splits;
+  int bn;
+  int full_tiles, tail_splits, tail_subtiles;  // whole tiles first, then the rest split (see GemmArgs)
   bool pair;      // 256-row tiles over a cluster of two CTAs
   int ntt;        // token sub-tiles of bn tokens per tile (pairs: 1 or 2)
   int slots;      // persistent units: CTAs (one-CTA tiles) or clusters (pairs)
@@ -669,8 +670,13 @@ struct FusedPlan {
 
 // Token tile: 32 tokens (one CTA per 128 weight rows) for a few tokens;
 // otherwise 256 tokens on CTA pairs (256 weight rows), when the device can
-// hold them, else on single CTAs. K is split across CTAs (or pairs) when
-// there are fewer tiles than persistent units.
+// hold them, else on single CTAs; from kTwoSubtileTokens tokens on, two
+// 256-token sub-tiles per tile. The persistent units (CTAs or pairs) run
+// whole rounds of whole tiles; the tiles of a last, partial round are split
+// so that the round fills the grid: by token sub-tile (two units of 256
+// tokens over the whole K, disjoint outputs) when the tiles hold two and
+// half the grid or more is idle, else over K (fp32 partials summed by the
+// last split) when there are fewer tiles than units.
 FusedPlan plan_fused(int64_t M, int64_t rows, int64_t kblocks, int sms, int pair_slots) {
   FusedPlan p;
   p.bn = M <= 32 ? 32 : 256;
@@ -680,24 +686,33 @@ FusedPlan plan_fused(int64_t M, int64_t rows, int64_t kblocks, int sms, int pair
   const int64_t tile_rows = p.pair ? 256 : 128;
   const int64_t tile_cols = static_cast<int64_t>(p.bn) * p.ntt;
   const int64_t tiles = cdiv(rows, tile_rows) * cdiv(M, tile_cols);
-  int64_t splits = 1;
-  if (tiles < p.slots) {
-    splits = p.slots / tiles;
-    if (splits > kblocks) splits = kblocks;
-    if (splits < 1) splits = 1;
+  const int64_t full = (tiles / p.slots) * p.slots;  // whole rounds
+  const int64_t tail = tiles - full;
+  p.tail_subtiles = 1;
+  if (full > 0 && tail > 0 && p.ntt > 1 && tail * p.ntt <= p.slots) {
+    p.full_tiles = static_cast<int>(full);
+    p.tail_splits = 1;
+    p.tail_subtiles = p.ntt;
+    p.part_bytes = 0;
+    return p;
   }
-  p.splits = static_cast<int>(splits);
-  p.part_bytes = p.splits > 1 ? align256(static_cast<size_t>(p.splits) * cdiv(rows, tile_rows) * tile_rows *
-                                         cdiv(M, tile_cols) * p.ntt * cdiv(p.bn, 32) * 32 * 4)
-                              : 0;
+  // split K only when the tiles do not fill one round (the fp32 partials of
+  // whole rounds of large tiles cost more than the imbalance they remove)
+  int64_t splits = (tail > 0 && full == 0) ? p.slots / tail : 1;
+  // a split runs at least 4 K blocks (1 on the memory-bound 32-token tiles)
+  const int64_t min_kb = p.bn == 32 ? 1 : 4;
+  if (splits > kblocks / min_kb) splits = kblocks / min_kb;
+  if (splits < 2) splits = 1;
+  p.full_tiles = static_cast<int>(splits > 1 ? full : tiles);
+  p.tail_splits = static_cast<int>(splits);
+  p.part_bytes = splits > 1 ? align256(static_cast<size_t>(splits) * tail * tile_rows * p.ntt * cdiv(p.bn, 32) * 32 * 4)
+                            : 0;
   return p;
 }
 
-// Partials bytes that any plan of this shape can need (the workspace size
-// must not depend on whether the pair variant turns out to be resident).
+// Partial bytes of the plan the call will run on this device.
 size_t fused_part_bound(int64_t M, int64_t rows, int64_t kblocks, int sms) {
-  return std::max(plan_fused(M, rows, kblocks, sms, sms / 2).part_bytes,
-                  plan_fused(M, rows, kblocks, sms, 0).part_bytes);
+  return plan_fused(M, rows, kblocks, sms, fused_pair_slots(sms)).part_bytes;
 }
 
 template <int BN, int AS, int L2>
@@ -735,8 +750,8 @@ SmallmPlan plan_smallm(int64_t M, int64_t N, int64_t K, int sms, int busy_sms) {
   p.units = p.bands * p.kc;
   const int avail = std::max(1, sms - busy_sms);
   p.grid = std::min(p.units, avail);
-  // one partial slot per CTA: its piece of the band an earlier CTA started
-  p.part_bytes = align256(static_cast<size_t>(p.grid) * SmallmCfg<1>::WARPS * p.nt * 32 * 16);
+  // two partial slots per CTA: its pieces of the bands shared with other CTAs
+  p.part_bytes = align256(static_cast<size_t>(p.grid) * 2 * SmallmCfg<1>::WARPS * p.nt * 32 * 16);
   return p;
 }
 
@@ -1067,7 +1082,9 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   a.rows = static_cast<int>(N);
   a.cols = static_cast<int>(M);
   a.kblocks = static_cast<int>(K / 64);
-  a.splits = fp.splits;
+  a.full_tiles = fp.full_tiles;
+  a.tail_splits = fp.tail_splits;
+  a.tail_subtiles = fp.tail_subtiles;
   a.lora_kblocks = static_cast<int>(cdiv(r, 64));
   a.out = Y;
   a.out_ld = N;
@@ -1142,7 +1159,9 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   a.rows = static_cast<int>(K);
   a.cols = static_cast<int>(M);
   a.kblocks = static_cast<int>(N / 64);
-  a.splits = fp.splits;
+  a.full_tiles = fp.full_tiles;
+  a.tail_splits = fp.tail_splits;
+  a.tail_subtiles = fp.tail_subtiles;
   a.lora_kblocks = static_cast<int>(cdiv(r, 64));
   a.out = dX;
   a.out_ld = K;

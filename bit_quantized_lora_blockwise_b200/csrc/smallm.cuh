@@ -15,10 +15,12 @@
 // Work split. Rows of W come in bands of 256 (one 16-row tile per compute
 // warp), K in chunks of 256 (four quantization blocks). The (band, chunk)
 // units, band-major, are divided evenly among a persistent grid (stream-K):
-// a CTA runs a contiguous range of units, its 8 warps on the same chunks.
-// The pieces of a band computed by different CTAs meet in fp32 partial
-// slots; the CTA that completes a band last (tile counter) sums the slots
-// in CTA order, so the result does not depend on timing.
+// a CTA runs a contiguous range of units, its 16 warps on the same chunks.
+// The pieces of a band computed by different CTAs are parked in fp32 slots
+// (at most two per CTA: the band its range starts in and the one it ends
+// in); the CTA whose piece completes a band (band counter) sums the slots in
+// CTA order, so the result does not depend on timing, and no CTA ever waits
+// for another one to be scheduled.
 //
 // Register fragments. In an m16n8k16 MMA, lane (g, t) = (lane / 4, lane % 4)
 // holds A elements (rows g and g+8, logical k 2t, 2t+1, 2t+8, 2t+9) and B
@@ -43,8 +45,8 @@ struct SmallmArgs {
   const __nv_bfloat16 *B;    // [r, N]
   const __nv_bfloat16 *xas;  // [M, r] = bf16((alpha / r) X A)
   __nv_bfloat16 *Y;          // [M, N]
-  float *part;               // partial slots: [grid][16 warps][NT][32 lanes][4]
-  unsigned int *counters;    // one per band, zero on entry (left zero): slots handed over
+  float *part;               // partial slots: [grid][2][16 warps][NT][32 lanes][4]
+  unsigned int *counters;    // one per band, zero on entry (left zero): pieces parked
   int64_t N, K;
   int M, r;
   int kc;     // 256-deep K chunks (the last may hold fewer than 4 blocks)
@@ -63,7 +65,7 @@ struct SmallmCfg {
   static constexpr int SX = 8;                   // activation stages
   static constexpr int OFF_BAR = SX * STAGE;
   static constexpr int OFF_T8 = OFF_BAR + 2 * SX * 8;
-  static constexpr int OFF_MISC = OFF_T8 + 256 * 4;
+  static constexpr int OFF_MISC = OFF_T8 + 256 * 4;  // abort flag, two completed-band flags
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SLOT_FLOATS = WARPS * NT * 32 * 4;
   static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
@@ -313,15 +315,17 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
     }
     store_y(n0);
   };
-  // Partial slot of CTA `cta`: the piece of the band its range starts in,
-  // when that band started in an earlier CTA.
-  auto slot_ptr = [&](int cta) {
-    return reinterpret_cast<float4 *>(a.part + static_cast<size_t>(cta) * C::SLOT_FLOATS) + warp * NT * 32 + lane;
+  // Partial slots of CTA `cta`: 0 holds the piece of the band its range
+  // starts in (when an earlier CTA started that band), 1 the piece of the
+  // band its range ends in (when later CTAs finish that band).
+  auto slot_ptr = [&](int cta, int which) {
+    return reinterpret_cast<float4 *>(a.part + (static_cast<size_t>(cta) * 2 + which) * C::SLOT_FLOATS) +
+           warp * NT * 32 + lane;
   };
 
   bool waited = false;
-  int reduce_band = -1;  // band this CTA completes from other CTAs' slots
-  int contrib_band = -1; // band whose slot this CTA fills for an earlier CTA
+  int first_band = -1;  // band whose later piece this CTA parked in slot 0
+  int last_band = -1;   // band whose first piece this CTA parked in slot 1
 
   const uint32_t swz16 = swz << 4;
   const uint32_t xrow = sbase + static_cast<uint32_t>((4 * g + t) * 128);
@@ -369,17 +373,14 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
           waited = true;
         }
         epilogue_lean(band);
-      } else if (piece0 == first_u) {
-        // the band starts here and continues in later CTAs: this CTA sums it
-        // (always its last piece, so acc stays live to the end)
-        reduce_band = band;
-        return true;
       } else {
-        // a later piece of a band started by an earlier CTA
-        float4 *dst = slot_ptr(blockIdx.x);
+        // a piece of a band shared with other CTAs: park it; the CTA whose
+        // piece completes the band sums them all (after the stream)
+        const int which = piece0 == first_u ? 1 : 0;
+        float4 *dst = slot_ptr(blockIdx.x, which);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) __stcg(dst + nt * 32, make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]));
-        contrib_band = band;
+        (which ? last_band : first_band) = band;
       }
       piece0 = u + 1;
 #pragma unroll
@@ -411,66 +412,70 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
     }
   }
   grid_dep_launch();
-  if (contrib_band < 0 && reduce_band < 0) return;
+  if (first_band < 0 && last_band < 0) return;
   if (!waited) grid_dep_wait();  // X A ready, band counters zeroed
 
-  // Hand the slot over: all warps' stores, then one release increment.
-  if (contrib_band >= 0) {
-    named_bar_sync(1, C::WARPS * 32);
-    if (threadIdx.x == 0) {
-      __threadfence();
-      atomicAdd(&a.counters[contrib_band], 1u);
-    }
-  }
-  if (reduce_band < 0) return;
-
-  // Sum the band: own piece (first in CTA order), then the slots of CTAs
-  // c0+1 .. c1 in order, once all of them have been handed over.
-  const int band = reduce_band;
-  const int64_t first_u = static_cast<int64_t>(band) * a.kc;
-  const int c0 = blockIdx.x;
-  const int c1 = smallm_cta_of(first_u + a.kc - 1, a.units, grid);
-  LoraFrag L0;  // loads in flight while the slots are awaited
-  if (band_row0(band) < a.N) lora_load(band_row0(band), 0, L0);
+  // For each parked piece: one release increment of the band's counter once
+  // every warp's stores are done; the CTA that brings the count to the
+  // band's number of pieces sums the slots of CTAs c0 .. c1 in CTA order
+  // (so the result does not depend on which CTA finishes last), applies the
+  // low-rank term and stores Y. No CTA waits for another.
+  named_bar_sync(1, C::WARPS * 32);  // every warp's parked pieces are stored
+  volatile int *s_last = s_abort + 1;  // [0]: first_band completed here, [1]: last_band
   if (threadIdx.x == 0) {
-    const unsigned int want = static_cast<unsigned int>(c1 - c0);
-    const unsigned long long tw = globaltimer_ns();
-    while (true) {
-      unsigned int v;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a.counters + band) : "memory");
-      if (v >= want) break;
-      if (globaltimer_ns() - tw > kWaitTimeoutNs) {
-        *s_abort = 1;
-        atomicOr(&g_error_word, kErrWaitTimeout);
-        break;
+    __threadfence();
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int band = k == 0 ? first_band : last_band;
+      int last = 0;
+      if (band >= 0) {
+        const int64_t first_u = static_cast<int64_t>(band) * a.kc;
+        const int npieces = smallm_cta_of(first_u + a.kc - 1, a.units, grid) - smallm_cta_of(first_u, a.units, grid) + 1;
+        const unsigned int prev = atomicAdd(&a.counters[band], 1u);
+        last = prev == static_cast<unsigned int>(npieces - 1);
+        if (last) a.counters[band] = 0u;  // every piece is in: left zero for the next call
       }
+      s_last[k] = last;
     }
-    a.counters[band] = 0u;  // left zero for the next call
   }
   named_bar_sync(1, C::WARPS * 32);
-  if (*s_abort) return;
-  for (int cta = c0 + 1; cta <= c1; cta += 8) {
-    float4 v[8][NT];
+#pragma unroll 1
+  for (int k = 0; k < 2; ++k) {
+    const int band = k == 0 ? first_band : last_band;
+    if (band < 0 || !s_last[k]) continue;
+    __threadfence();
+    const int64_t first_u = static_cast<int64_t>(band) * a.kc;
+    const int c0 = smallm_cta_of(first_u, a.units, grid);
+    const int c1 = smallm_cta_of(first_u + a.kc - 1, a.units, grid);
+    LoraFrag L0;  // its loads overlap the slot loads below
+    if (band_row0(band) < a.N) lora_load(band_row0(band), 0, L0);
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (cta + j <= c1) {
-        const float4 *src = slot_ptr(cta + j);
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) v[j][nt] = __ldcg(src + nt * 32);
-      }
+      for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
+    for (int cta = c0; cta <= c1; cta += 4) {
+      float4 v[4][NT];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (cta + j <= c1) {
+      for (int j = 0; j < 4; ++j)
+        if (cta + j <= c1) {
+          const float4 *src = slot_ptr(cta + j, cta + j == c0 ? 1 : 0);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          acc[nt][0] += v[j][nt].x;
-          acc[nt][1] += v[j][nt].y;
-          acc[nt][2] += v[j][nt].z;
-          acc[nt][3] += v[j][nt].w;
+          for (int nt = 0; nt < NT; ++nt) v[j][nt] = __ldcg(src + nt * 32);
         }
-      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (cta + j <= c1) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            acc[nt][0] += v[j][nt].x;
+            acc[nt][1] += v[j][nt].y;
+            acc[nt][2] += v[j][nt].z;
+            acc[nt][3] += v[j][nt].w;
+          }
+        }
+    }
+    epilogue(band, L0);
   }
-  epilogue(band, L0);
 }
 
 }  // namespace qlora
