@@ -761,7 +761,7 @@ int skinny_ctas(int64_t rows, int64_t kdim, int r) {
   return static_cast<int>(cdiv(rows, 128)) * p.splits;
 }
 
-template <int NT, bool V8>
+template <int NT>
 qlora_status run_smallm_nt(const SmallmArgs &a, int grid, cudaStream_t st) {
   using C = SmallmCfg<NT>;
   static std::once_flag once[kMaxDevices];
@@ -769,16 +769,14 @@ qlora_status run_smallm_nt(const SmallmArgs &a, int grid, cudaStream_t st) {
   cudaGetDevice(&dev);
   cudaError_t attr_err = cudaSuccess;
   std::call_once(once[dev], [&] {
-    attr_err = cudaFuncSetAttribute(smallm_kernel<NT, V8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    C::SMEM_BYTES);
+    attr_err = cudaFuncSetAttribute(smallm_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return QLORA_ERR_CUDA;
-  return launch_pdl(smallm_kernel<NT, V8>, grid, C::THREADS, C::SMEM_BYTES, st, a);
+  return launch_pdl(smallm_kernel<NT>, grid, C::THREADS, C::SMEM_BYTES, st, a);
 }
 
-qlora_status run_smallm(const SmallmArgs &a, const SmallmPlan &p, bool v8, cudaStream_t st) {
-  if (p.nt == 1) return v8 ? run_smallm_nt<1, true>(a, p.grid, st) : run_smallm_nt<1, false>(a, p.grid, st);
-  return v8 ? run_smallm_nt<2, true>(a, p.grid, st) : run_smallm_nt<2, false>(a, p.grid, st);
+qlora_status run_smallm(const SmallmArgs &a, const SmallmPlan &p, cudaStream_t st) {
+  return p.nt == 1 ? run_smallm_nt<1>(a, p.grid, st) : run_smallm_nt<2>(a, p.grid, st);
 }
 
 // Workspace carve-up: [tile counters][bf16 M x r][bf16 M x r (backward)][c'][fp32 partials]
@@ -1034,8 +1032,9 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
     if (st != QLORA_OK) return st;
     SmallmArgs a;
     std::memset(&a, 0, sizeof a);
-    if (!map_x_blocks(&a.tm_x, X, M, K, static_cast<uint32_t>(8 * sp.nt))) return QLORA_ERR_CUDA;
-    a.packed = packed;
+    if (!map_x_blocks(&a.tm_x, X, M, K, static_cast<uint32_t>(8 * sp.nt)) ||
+        !make_map(&a.tm_w, packed, MAP_U8, K / 2, N, K / 2, 128, SmallmCfg<1>::BAND, SW_128B))
+      return QLORA_ERR_CUDA;
     a.q = q;
     a.scale2 = scale2;
     a.B = reinterpret_cast<const __nv_bfloat16 *>(B);
@@ -1050,9 +1049,8 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
     a.kc = sp.kc;
     a.units = sp.units;
     a.tabs = make_tables(nf4, t8);
-    const bool v8 = (reinterpret_cast<uintptr_t>(packed) & 31u) == 0;
     trace_begin(cs);
-    st = run_smallm(a, sp, v8, cs);
+    st = run_smallm(a, sp, cs);
     trace_end(cs);
     return st;
   }

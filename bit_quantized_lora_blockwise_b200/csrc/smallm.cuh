@@ -4,23 +4,30 @@
 // The forward of one QLoRA linear (intvml.com "DL0087 QLoRA: 4-bit Quantized
 // LoRA", opening paragraph and Figure 1): the base weight is stored as NF4
 // codes with double-quantized block constants and is dequantized to bf16
-// just before it is multiplied. With a few
-// tokens the layer reads 0.516 bytes of packed weight per parameter and does
-// 2 M flops with it, so it is bound by HBM. This kernel therefore never
-// stages the weight in shared memory: every packed byte is loaded once, by
-// the thread that decodes it, straight into the register fragment of a
-// warp-level 16x8x16 tensor-core MMA. Only the activations (at most 16
-// tokens, L2-resident) go through shared memory, brought in by TMA.
+// just before it is multiplied. With a few tokens the layer reads 0.516
+// bytes of packed weight per parameter and does 2 M flops with it; what
+// bounds it is the HBM stream and the integer work of the decode (about 21
+// byte-permute and logic operations per 8 codes), not the tensor cores.
 //
-// Work split. Rows of W come in bands of 256 (one 16-row tile per compute
-// warp), K in chunks of 256 (four quantization blocks). The (band, chunk)
-// units, band-major, are divided evenly among a persistent grid (stream-K):
-// a CTA runs a contiguous range of units, its 16 warps on the same chunks.
-// The pieces of a band computed by different CTAs are parked in fp32 slots
-// (at most two per CTA: the band its range starts in and the one it ends
-// in); the CTA whose piece completes a band (band counter) sums the slots in
-// CTA order, so the result does not depend on timing, and no CTA ever waits
-// for another one to be scheduled.
+// Data path. One producer warp keeps a ring of shared-memory stages full
+// with TMA: a stage is one unit's packed codes (256 rows x 128 bytes, one
+// 32 KB box, 128-byte swizzle) plus the matching activations (X for the
+// unit's 256 K, at most 16 tokens). Sixteen compute warps (one 16-row tile
+// each) read their codes from the stage with 16-byte shared loads, decode
+// them in registers with a per-block bf16 table and feed warp-level
+// 16x8x16 tensor-core MMAs. The block constants (8-bit code and
+// second-level scale) are loaded by the compute threads two units ahead.
+// Decoupling the stream from the decode keeps five or six units (160-200 KB
+// per SM) in flight, so the integer pipe, not memory latency, sets the rate.
+//
+// Work split. Rows of W come in bands of 256, K in chunks of 256 (four
+// quantization blocks). The (band, chunk) units, band-major, are divided
+// evenly among a persistent grid (stream-K): a CTA runs a contiguous range
+// of units. The pieces of a band computed by different CTAs are parked in
+// fp32 slots (at most two per CTA: the band its range starts in and the one
+// it ends in); the CTA whose piece completes a band (band counter) sums the
+// slots in CTA order, so the result does not depend on timing, and no CTA
+// ever waits for another one to be scheduled.
 //
 // Register fragments. In an m16n8k16 MMA, lane (g, t) = (lane / 4, lane % 4)
 // holds A elements (rows g and g+8, logical k 2t, 2t+1, 2t+8, 2t+9) and B
@@ -39,7 +46,7 @@ namespace qlora {
 
 struct SmallmArgs {
   CUtensorMap tm_x;          // X [M, K] bf16 viewed as {64, K/64, M}; box {64, 4, 8 NT}, 128B swizzle
-  const uint8_t *packed;     // [N, K/2], element 2j in the low nibble
+  CUtensorMap tm_w;          // packed [N, K/2] u8; box {128, 256}, 128B swizzle
   const uint8_t *q;          // [N K / 64] 8-bit block-constant codes
   const float *scale2;       // [ceil(N K / 64 / 256)] second-level scales
   const __nv_bfloat16 *B;    // [r, N]
@@ -59,16 +66,19 @@ struct SmallmCfg {
   static constexpr int NT = NT_;                 // 8-token MMA column tiles
   static constexpr int WARPS = 16;               // compute warps, one 16-row tile each
   static constexpr int BAND = 16 * WARPS;        // rows of W per band
-  static constexpr int THREADS = WARPS * 32;     // lane 0 of warp 0 also issues the X copies
+  static constexpr int THREADS = WARPS * 32;     // lane 0 of warp 0 also issues the stage copies
   static constexpr int XR = 8 * NT;              // token rows per stage
-  static constexpr int STAGE = 4 * XR * 128;     // [XR tokens][4 blocks][64 bf16]
-  static constexpr int SX = 8;                   // activation stages
+  static constexpr int W_BYTES = BAND * 128;     // [256 rows][128 bytes = 256 codes]
+  static constexpr int X_BYTES = 4 * XR * 128;   // [XR tokens][4 blocks][64 bf16]
+  static constexpr int STAGE = W_BYTES + X_BYTES;
+  static constexpr int SX = NT == 1 ? 6 : 5;     // stages
   static constexpr int OFF_BAR = SX * STAGE;
   static constexpr int OFF_T8 = OFF_BAR + 2 * SX * 8;
   static constexpr int OFF_MISC = OFF_T8 + 256 * 4;  // abort flag, two completed-band flags
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SLOT_FLOATS = WARPS * NT * 32 * 4;
-  static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+  static_assert(W_BYTES % 1024 == 0 && X_BYTES % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
 // CTA that owns unit u when `units` units are split evenly over `grid` CTAs
@@ -80,7 +90,7 @@ __host__ __device__ __forceinline__ int smallm_unit_begin(int64_t cta, int64_t u
   return static_cast<int>(cta * units / grid);
 }
 
-template <int NT, bool V8>
+template <int NT>
 __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const __grid_constant__ SmallmArgs a) {
   using C = SmallmCfg<NT>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -88,143 +98,83 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float *s_t8 = reinterpret_cast<float *>(smem + C::OFF_T8);
   volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC);
-  auto x_full = [&](int s) { return sbase + C::OFF_BAR + 8u * s; };
-  auto x_empty = [&](int s) { return sbase + C::OFF_BAR + 8u * (C::SX + s); };
+  auto full_bar = [&](int s) { return sbase + C::OFF_BAR + 8u * s; };
+  auto empty_bar = [&](int s) { return sbase + C::OFF_BAR + 8u * (C::SX + s); };
 
   const int grid = gridDim.x;
   const int u_begin = smallm_unit_begin(blockIdx.x, a.units, grid);
   const int u_end = smallm_unit_begin(blockIdx.x + 1, a.units, grid);
   const int nunits = u_end - u_begin;
 
-  // X copies (lane 0 of warp 0): unit j goes to stage j % SX once every warp
-  // has released unit j - SX. Before unit i is consumed its copy must be
-  // issued (waiting for the slowest warp if needed); later ones are issued
-  // when their stage is already free. The first SX go out before anything
-  // else, ahead of the weight stream.
-  int x_issued = 0;
-  auto issue_x = [&](int i) {
-    while (x_issued < nunits && x_issued < i + C::SX) {
-      const int j = x_issued, st = j % C::SX;
+  // Stage copies (lane 0 of warp 0): unit j goes to stage j % SX once every
+  // warp has released unit j - SX; its codes (one box) and activations (one
+  // box) are counted on the stage's full barrier. Before unit i is consumed
+  // its copy must be issued (waiting for the slowest warp if needed); later
+  // ones are issued when their stage is already free. X and the packed
+  // weight are inputs of this call, so the copies need no wait on the launch
+  // before.
+  int issued = 0, is_band = u_begin / a.kc, is_c = u_begin - (u_begin / a.kc) * a.kc;
+  auto issue = [&](int i) {
+    while (issued < nunits && issued < i + C::SX) {
+      const int j = issued, st = j % C::SX;
       if (j >= C::SX) {
         const uint32_t par = ((j / C::SX) - 1) & 1u;
         if (j == i) {
-          if (!mbar_wait_spin(x_empty(st), par, s_abort)) return;
-        } else if (!mbar_try_wait(x_empty(st), par)) {
+          if (!mbar_wait_spin(empty_bar(st), par, s_abort)) return;
+        } else if (!mbar_try_wait(empty_bar(st), par)) {
           return;
         }
       }
-      const int c = (j + u_begin) % a.kc;
-      mbar_arrive_expect_tx(x_full(st), C::STAGE);
-      tma_load_3d(sbase + st * C::STAGE, &a.tm_x, x_full(st), 0, c * 4, 0);
-      ++x_issued;
+      const uint32_t dst = sbase + st * C::STAGE;
+      mbar_arrive_expect_tx(full_bar(st), C::STAGE);
+      tma_load_2d(dst, &a.tm_w, full_bar(st), is_c * 128, is_band * C::BAND);
+      tma_load_3d(dst + C::W_BYTES, &a.tm_x, full_bar(st), 0, is_c * 4, 0);
+      if (++is_c == a.kc) {
+        is_c = 0;
+        ++is_band;
+      }
+      ++issued;
     }
   };
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::SX; ++s) {
-      mbar_init(x_full(s), 1);
-      mbar_init(x_empty(s), C::WARPS);
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), C::WARPS);
     }
     *s_abort = 0;
     fence_barrier_init();
+    tma_prefetch_desc(&a.tm_w);
     tma_prefetch_desc(&a.tm_x);
-    issue_x(0);
+    issue(0);  // the first SX stages go out before anything else
   }
   for (int i = threadIdx.x; i < 256; i += blockDim.x) s_t8[i] = a.tabs.t8[i];
   __syncthreads();
 
   // ------------------------------------------------------ compute warps --
   const int g = lane >> 2, t = lane & 3;
-  const uint32_t swz = static_cast<uint32_t>((4 * g + t) & 7);
   const int64_t kb_total = a.K / 64;
-  const int64_t row_bytes = a.K / 2;
 
-  // This lane's packed bytes, constant codes and scales for one unit. The
-  // loader walks the CTA's units in order (chunk by chunk, band by band),
-  // so addresses advance by a fixed step inside a band.
-  struct Frag {
-    uint32_t w[2][8];
+  // This lane's block constants for one unit (rows g and g + 8 of the warp's
+  // tile, block t of the chunk), loaded two units ahead of their use.
+  struct Consts {
     uint32_t q[2];
     float s[2];
   };
-  // L2 prefetch: a second walk over the same units, kPfAhead units ahead of
-  // the register loads, so that those loads hit L2 rather than DRAM
-  constexpr int kPfAhead = 4;
-  int pf_band = u_begin / a.kc, pf_c = u_begin - (u_begin / a.kc) * a.kc, pf_idx = 0;
-  const uint8_t *pf_p = nullptr, *pf_q = nullptr;
-  bool pf_row_ok = false;
-  auto pf_setup = [&]() {
-    const int64_t row = static_cast<int64_t>(pf_band) * C::BAND + warp * 16 + g;
-    pf_row_ok = row < a.N;
-    const int64_t bi = row * kb_total + static_cast<int64_t>(pf_c) * 4 + t;
-    pf_p = a.packed + bi * 32;
-    pf_q = a.q + bi;
-  };
-  auto pf_step = [&]() {  // prefetch the walk's unit (rows g and g + 8), then advance
-    if (pf_idx >= nunits) return;
-    if (pf_row_ok && static_cast<int64_t>(pf_c) * 4 + t < kb_total) {
-      prefetch_l2(pf_p);
-      prefetch_l2(pf_p + 8 * row_bytes);
-      prefetch_l2(pf_q);
-      prefetch_l2(pf_q + 8 * kb_total);
-    }
-    ++pf_idx;
-    if (++pf_c == a.kc) {
-      pf_c = 0;
-      ++pf_band;
-      pf_setup();
-    } else {
-      pf_p += 128;
-      pf_q += 4;
-    }
-  };
-  pf_setup();
-  for (int k = 0; k < kPfAhead; ++k) pf_step();  // units 0 .. kPfAhead - 1 up front
   int ld_band = u_begin / a.kc, ld_c = u_begin - (u_begin / a.kc) * a.kc;
-  const uint8_t *ld_p = nullptr;  // row g of the band, chunk ld_c, block t
-  int64_t ld_bi = 0;              // block index of that row and block
-  bool ld_row_ok = false;
-  auto band_setup = [&]() {
+  auto load_consts = [&](Consts &f) {
     const int64_t row = static_cast<int64_t>(ld_band) * C::BAND + warp * 16 + g;
-    ld_row_ok = row < a.N;
-    ld_bi = row * kb_total + static_cast<int64_t>(ld_c) * 4 + t;
-    ld_p = a.packed + ld_bi * 32;
-  };
-  band_setup();
-  auto load_next = [&](Frag &f) {
-    const bool ok = ld_row_ok && static_cast<int64_t>(ld_c) * 4 + t < kb_total;
-    if (ok) {
+    const int64_t kb = static_cast<int64_t>(ld_c) * 4 + t;
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const uint8_t *p = ld_p + rr * 8 * row_bytes;
-        if (V8) {
-          ld_stream_32B(p, f.w[rr]);
-        } else {
-          const uint4 lo = ld_stream_16B(p), hi = ld_stream_16B(p + 16);
-          f.w[rr][0] = lo.x; f.w[rr][1] = lo.y; f.w[rr][2] = lo.z; f.w[rr][3] = lo.w;
-          f.w[rr][4] = hi.x; f.w[rr][5] = hi.y; f.w[rr][6] = hi.z; f.w[rr][7] = hi.w;
-        }
-        const int64_t bi = ld_bi + rr * 8 * kb_total;
-        f.q[rr] = __ldg(a.q + bi);
-        f.s[rr] = __ldg(a.scale2 + (bi >> 8));
-      }
-    } else {
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) f.w[rr][j] = 0u;
-        f.q[rr] = 0u;
-        f.s[rr] = 0.0f;  // c' = 0: the block contributes zeros
-      }
+    for (int rr = 0; rr < 2; ++rr) {
+      const bool ok = row + 8 * rr < a.N && kb < kb_total;
+      const int64_t bi = (row + 8 * rr) * kb_total + kb;
+      f.q[rr] = ok ? __ldg(a.q + bi) : 0u;
+      f.s[rr] = ok ? __ldg(a.scale2 + (bi >> 8)) : 0.0f;  // c' = 0: the block contributes zeros
     }
     if (++ld_c == a.kc) {
       ld_c = 0;
       ++ld_band;
-      band_setup();
-    } else {
-      ld_p += 128;
-      ld_bi += 4;
     }
-    pf_step();
   };
 
   float acc[NT][4];
@@ -327,37 +277,51 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
   int first_band = -1;  // band whose later piece this CTA parked in slot 0
   int last_band = -1;   // band whose first piece this CTA parked in slot 1
 
-  const uint32_t swz16 = swz << 4;
-  const uint32_t xrow = sbase + static_cast<uint32_t>((4 * g + t) * 128);
-  int cur_band = ld_band, cur_c = ld_c, piece0 = u_begin;
+  // Shared-memory addresses of this lane's data in stage 0. Codes: rows g
+  // and g + 8 of the warp's tile, 16-byte chunks 2t and 2t + 1 of the row's
+  // 128 bytes, at chunk ^ (row & 7) (row & 7 = g) under the 128-byte
+  // swizzle. Activations: token g, block t, 16-byte chunk u at u ^ (4g + t) & 7.
+  const uint32_t wrow = sbase + static_cast<uint32_t>((warp * 16 + g) * 128);
+  const uint32_t wc0 = static_cast<uint32_t>(((2 * t) ^ g) << 4);
+  const uint32_t wc1 = static_cast<uint32_t>(((2 * t + 1) ^ g) << 4);
+  const uint32_t swz16 = static_cast<uint32_t>(((4 * g + t) & 7) << 4);
+  const uint32_t xrow = sbase + C::W_BYTES + static_cast<uint32_t>((4 * g + t) * 128);
+  int cur_band = u_begin / a.kc, cur_c = u_begin - (u_begin / a.kc) * a.kc, piece0 = u_begin;
   // Decode one unit's codes into MMA fragments and accumulate; then
-  // release its activation stage and close the piece if a band ends.
-  auto run_unit = [&](int i, const Frag &f) -> bool {
+  // release its stage and close the piece if a band ends.
+  auto run_unit = [&](int i, const Consts &f) -> bool {
     const float cp0 = __fmul_rn(s_t8[f.q[0]], f.s[0]);
     const float cp1 = __fmul_rn(s_t8[f.q[1]], f.s[1]);
-    const Nf4Planes P0 = make_planes(a.tabs.nf4, cp0);
-    const Nf4Planes P1 = make_planes(a.tabs.nf4, cp1);
     const int s = i % C::SX;
-    if (warp == 0 && lane == 0) issue_x(i);
+    if (warp == 0 && lane == 0) issue(i);
     __syncwarp();
-    if (!__all_sync(0xFFFFFFFFu, mbar_wait_spin(x_full(s), (i / C::SX) & 1u, s_abort))) return false;
-    const uint32_t xs = xrow + s * C::STAGE;
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait_spin(full_bar(s), (i / C::SX) & 1u, s_abort))) return false;
     const bool rows_here = static_cast<int64_t>(cur_band) * C::BAND + warp * 16 < a.N;
+    if (rows_here) {
+      const Nf4Planes P0 = make_planes(a.tabs.nf4, cp0);
+      const Nf4Planes P1 = make_planes(a.tabs.nf4, cp1);
+      const uint32_t ws = wrow + s * C::STAGE;
+      const uint4 r0a = lds_16B(ws + wc0), r0b = lds_16B(ws + wc1);
+      const uint4 r1a = lds_16B(ws + 8 * 128 + wc0), r1b = lds_16B(ws + 8 * 128 + wc1);
+      const uint32_t w0[8] = {r0a.x, r0a.y, r0a.z, r0a.w, r0b.x, r0b.y, r0b.z, r0b.w};
+      const uint32_t w1[8] = {r1a.x, r1a.y, r1a.z, r1a.w, r1b.x, r1b.y, r1b.z, r1b.w};
+      const uint32_t xs = xrow + s * C::STAGE;
 #pragma unroll
-    for (int uu = 0; uu < (rows_here ? 8 : 0); ++uu) {
-      uint32_t o0[4], o1[4];
-      nf4_lookup8(P0, f.w[0][uu], o0);
-      nf4_lookup8(P1, f.w[1][uu], o1);
-      const uint32_t xa = xs | ((static_cast<uint32_t>(uu) << 4) ^ swz16);
+      for (int uu = 0; uu < 8; ++uu) {
+        uint32_t o0[4], o1[4];
+        nf4_lookup8(P0, w0[uu], o0);
+        nf4_lookup8(P1, w1[uu], o1);
+        const uint32_t xa = xs | ((static_cast<uint32_t>(uu) << 4) ^ swz16);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const uint4 xv = lds_16B(xa + nt * (8 * 4 * 128));
-        mma_16816_bf16(acc[nt], o0[0], o1[0], o0[1], o1[1], xv.x, xv.y);
-        mma_16816_bf16(acc[nt], o0[2], o1[2], o0[3], o1[3], xv.z, xv.w);
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint4 xv = lds_16B(xa + nt * (8 * 4 * 128));
+          mma_16816_bf16(acc[nt], o0[0], o1[0], o0[1], o1[1], xv.x, xv.y);
+          mma_16816_bf16(acc[nt], o0[2], o1[2], o0[3], o1[3], xv.z, xv.w);
+        }
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(x_empty(s));
+    if (lane == 0) mbar_arrive(empty_bar(s));
     const int u = u_begin + i;
     const int band = cur_band;
     if (++cur_c == a.kc) {
@@ -391,22 +355,26 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
     return true;
   };
 
-  // two register buffers: the next unit's loads are in flight while one
-  // unit is decoded
-  Frag fa, fb;
-  if (nunits > 0) load_next(fa);
-  for (int i = 0; i < nunits; i += 2) {
-    if (i + 1 < nunits) load_next(fb);
-    if (!run_unit(i, fa)) break;
+  // constants of the next two units in registers: one unit's are in
+  // flight while another is decoded
+  Consts ca, cb, cc;
+  if (nunits > 0) load_consts(ca);
+  if (nunits > 1) load_consts(cb);
+  for (int i = 0; i < nunits; i += 3) {
+    if (i + 2 < nunits) load_consts(cc);
+    if (!run_unit(i, ca)) break;
     if (i + 1 >= nunits) break;
-    if (i + 2 < nunits) load_next(fa);
-    if (!run_unit(i + 1, fb)) break;
+    if (i + 3 < nunits) load_consts(ca);
+    if (!run_unit(i + 1, cb)) break;
+    if (i + 2 >= nunits) break;
+    if (i + 4 < nunits) load_consts(cb);
+    if (!run_unit(i + 2, cc)) break;
   }
   if (warp == 0 && lane == 0) {
-    // bounded wait for X copies still in flight (only after an abort)
-    for (int j = x_issued > C::SX ? x_issued - C::SX : 0; j < x_issued; ++j) {
+    // bounded wait for the copies still in flight (only after an abort)
+    for (int j = issued > C::SX ? issued - C::SX : 0; j < issued; ++j) {
       const unsigned long long t0 = globaltimer_ns();
-      while (!mbar_try_wait(x_full(j % C::SX), (j / C::SX) & 1u)) {
+      while (!mbar_try_wait(full_bar(j % C::SX), (j / C::SX) & 1u)) {
         if (globaltimer_ns() - t0 > kWaitTimeoutNs) break;
       }
     }
