@@ -373,6 +373,22 @@ class LinearState:
                 "dequant": n // 2 + n // 64 + ((n // 64 + 255) // 256) * 4 + n * 2}
 
 
+def dequant_then_library(packed, q, scale2, X, A, B, dY, alpha, N, K, Wq=None):
+    """The comparison design, dequantize then multiply: this library's
+    dequant writes W' (in X's 16-bit type) to HBM, then torch matmuls
+    (cuBLAS) compute the layer's forward and backward products.
+    Returns (Y, dX, dA, dB)."""
+    import torch
+    from bit_quantized_lora_blockwise_b200 import binding
+    s = alpha / A.shape[1]
+    Wq = binding.dequant(packed, q, scale2, N, K, out=Wq, dtype=X.dtype)
+    xas = (X @ A) * s
+    Y = torch.addmm(xas @ B, X, Wq.t())
+    g = (dY @ B.t()) * s
+    dX = torch.addmm(g @ A.t(), dY, Wq)
+    return Y, dX, X.t() @ g, xas.t() @ dY
+
+
 def compare_dequant_then_library_gemm(layers, ws, steps):
     """The design the pages describe, dequantize then multiply, timed against
     the fused calls (a comparison, not the product and not the headline).
@@ -391,14 +407,7 @@ def compare_dequant_then_library_gemm(layers, ws, steps):
                            dA=L.dA, dB=L.dB, workspace=ws)
 
     def library(L):
-        s = L.alpha / L.r
-        binding.dequant(L.packed, L.q, L.scale2, L.N, L.K, out=L.Wq)
-        xas = (L.X @ L.A) * s
-        torch.addmm(xas @ L.B, L.X, L.Wq.t())              # Y
-        g = (L.dY @ L.B.t()) * s
-        torch.addmm(g @ L.A.t(), L.dY, L.Wq)               # dX
-        L.X.t() @ g                                        # dA
-        xas.t() @ L.dY                                     # dB
+        dequant_then_library(L.packed, L.q, L.scale2, L.X, L.A, L.B, L.dY, L.alpha, L.N, L.K, Wq=L.Wq)
 
     out = {}
     for name, fn in (("fused_ms", fused), ("dequant_then_cublas_ms", library)):

@@ -33,7 +33,11 @@ EXPORTS = ("qlora_status_string", "qlora_abi_version", "qlora_nf4_levels", "qlor
            "qlora_int4_levels", "qlora_fp4_levels", "qlora_dq_signed_levels", "qlora_dq_dynamic_levels",
            "qlora_workspace_bytes", "qlora_quantize_nf4", "qlora_double_quant", "qlora_dequant",
            "qlora_linear_fwd", "qlora_linear_bwd", "qlora_device_error", "qlora_set_trace_events",
-           "qlora_launch_count", "qlora_linear_fwd_noalloc", "qlora_selftest_bounded_wait")
+           "qlora_launch_count", "qlora_linear_fwd_noalloc", "qlora_selftest_bounded_wait",
+           "qlora_dequant_dt", "qlora_linear_fwd_dt", "qlora_linear_bwd_dt")
+
+# qlora_dtype of the 16-bit tensors of a call
+_DTYPE = {torch.bfloat16: 0, torch.float16: 1}
 
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -74,6 +78,13 @@ def load(path: str | None = None):
         lib.qlora_linear_fwd_noalloc.restype = I32
         lib.qlora_linear_bwd.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, P, P, P, I32, F32, P, P, P,
                                          P, SZ, P]
+        lib.qlora_dequant_dt.argtypes = [P, P, P, I64, I64, P, P, I32, P, P]
+        lib.qlora_linear_fwd_dt.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P, I32, F32, P, P, P, SZ,
+                                            P]
+        lib.qlora_linear_bwd_dt.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P, P, P, I32, F32, P, P,
+                                            P, P, SZ, P]
+        for fn in ("qlora_dequant_dt", "qlora_linear_fwd_dt", "qlora_linear_bwd_dt"):
+            getattr(lib, fn).restype = I32
         lib.qlora_device_error.argtypes = [I32]
         lib.qlora_device_error.restype = ctypes.c_uint32
         lib.qlora_set_trace_events.argtypes = [P, P]
@@ -252,17 +263,30 @@ def double_quant(absmax: torch.Tensor, t8=None, q=None, scale2=None):
     return q, scale2
 
 
-def dequant(packed, q, scale2, N: int, K: int, nf4=None, t8=None, out=None) -> torch.Tensor:
-    """-> W' bf16 [N, K]."""
+def _dtype_of(t, name):
+    if t.dtype not in _DTYPE:
+        raise TypeError(f"{name} must be torch.bfloat16 or torch.float16, got {t.dtype}")
+    return t.dtype
+
+
+def dequant(packed, q, scale2, N: int, K: int, nf4=None, t8=None, out=None,
+            dtype=torch.bfloat16) -> torch.Tensor:
+    """-> W' [N, K] in `dtype` (bf16, or fp16 through qlora_dequant_dt)."""
     _req(packed, "packed", torch.uint8, (N * K // 2,))
     _req(q, "q", torch.uint8, (N * K // BLOCK,))
     _req(scale2, "scale2", torch.float32)
+    if dtype not in _DTYPE:
+        raise TypeError(f"dtype must be torch.bfloat16 or torch.float16, got {dtype}")
     if out is None:
-        out = torch.empty((N, K), dtype=torch.bfloat16, device=packed.device)
-    _req(out, "out", torch.bfloat16, (N, K))
+        out = torch.empty((N, K), dtype=dtype, device=packed.device)
+    _req(out, "out", dtype, (N, K))
     tb = _tables(nf4, t8)
-    _check(load().qlora_dequant(_ptr(packed), _ptr(q), _ptr(scale2), N, K, tb.nf4, tb.t8, _ptr(out),
-                                _stream()), "qlora_dequant")
+    if dtype == torch.bfloat16:
+        _check(load().qlora_dequant(_ptr(packed), _ptr(q), _ptr(scale2), N, K, tb.nf4, tb.t8, _ptr(out),
+                                    _stream()), "qlora_dequant")
+    else:
+        _check(load().qlora_dequant_dt(_ptr(packed), _ptr(q), _ptr(scale2), N, K, tb.nf4, tb.t8,
+                                       _DTYPE[dtype], _ptr(out), _stream()), "qlora_dequant_dt")
     return out
 
 
@@ -276,22 +300,32 @@ def _workspace(workspace, M, N, K, r, device):
 
 def linear_fwd(packed, q, scale2, X, A, B, alpha: float, N: int, K: int, nf4=None, t8=None,
                Y=None, XA_out=None, workspace=None):
-    """Y = X W'^T + (alpha/r) (X A) B  -> Y bf16 [M, N] (and XA_out if given)."""
+    """Y = X W'^T + (alpha/r) (X A) B  -> Y [M, N] (and XA_out if given).
+
+    The 16-bit tensors are all bf16 or all fp16 (X's dtype decides; fp16
+    goes through qlora_linear_fwd_dt)."""
     M = X.shape[0]
     r = A.shape[1]
-    _req(X, "X", torch.bfloat16, (M, K))
-    _req(A, "A", torch.bfloat16, (K, r))
-    _req(B, "B", torch.bfloat16, (r, N))
+    dt = _dtype_of(X, "X")
+    _req(X, "X", dt, (M, K))
+    _req(A, "A", dt, (K, r))
+    _req(B, "B", dt, (r, N))
     if Y is None:
-        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
-    _req(Y, "Y", torch.bfloat16, (M, N))
+        Y = torch.empty((M, N), dtype=dt, device=X.device)
+    _req(Y, "Y", dt, (M, N))
     if XA_out is not None:
-        _req(XA_out, "XA_out", torch.bfloat16, (M, r))
+        _req(XA_out, "XA_out", dt, (M, r))
     workspace = _workspace(workspace, M, N, K, r, X.device)
     tb = _tables(nf4, t8)
-    _check(load().qlora_linear_fwd(_ptr(packed), _ptr(q), _ptr(scale2), tb.nf4, tb.t8, M, N, K, _ptr(X),
-                                   _ptr(A), _ptr(B), r, float(alpha), _ptr(Y), _ptr(XA_out),
-                                   _ptr(workspace), workspace.numel(), _stream()), "qlora_linear_fwd")
+    if dt == torch.bfloat16:
+        _check(load().qlora_linear_fwd(_ptr(packed), _ptr(q), _ptr(scale2), tb.nf4, tb.t8, M, N, K, _ptr(X),
+                                       _ptr(A), _ptr(B), r, float(alpha), _ptr(Y), _ptr(XA_out),
+                                       _ptr(workspace), workspace.numel(), _stream()), "qlora_linear_fwd")
+    else:
+        _check(load().qlora_linear_fwd_dt(_ptr(packed), _ptr(q), _ptr(scale2), tb.nf4, tb.t8, _DTYPE[dt], M, N,
+                                          K, _ptr(X), _ptr(A), _ptr(B), r, float(alpha), _ptr(Y),
+                                          _ptr(XA_out), _ptr(workspace), workspace.numel(), _stream()),
+               "qlora_linear_fwd_dt")
     return Y
 
 
@@ -319,26 +353,34 @@ def linear_fwd_noalloc(packed, q, scale2, X, A, B, alpha: float, N: int, K: int,
 
 def linear_bwd(packed, q, scale2, X, dY, A, B, alpha: float, N: int, K: int, XA=None, nf4=None, t8=None,
                dX=None, dA=None, dB=None, workspace=None):
-    """-> (dX bf16 [M, K], dA bf16 [K, r], dB bf16 [r, N]); no dW (W is frozen)."""
+    """-> (dX [M, K], dA [K, r], dB [r, N]); no dW (W is frozen). The 16-bit
+    tensors are all bf16 or all fp16 (X's dtype decides)."""
     M = X.shape[0]
     r = A.shape[1]
-    _req(X, "X", torch.bfloat16, (M, K))
-    _req(dY, "dY", torch.bfloat16, (M, N))
-    _req(A, "A", torch.bfloat16, (K, r))
-    _req(B, "B", torch.bfloat16, (r, N))
+    dt = _dtype_of(X, "X")
+    _req(X, "X", dt, (M, K))
+    _req(dY, "dY", dt, (M, N))
+    _req(A, "A", dt, (K, r))
+    _req(B, "B", dt, (r, N))
     if XA is not None:
-        _req(XA, "XA", torch.bfloat16, (M, r))
+        _req(XA, "XA", dt, (M, r))
     dev = X.device
-    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev) if dX is None else dX
-    dA = torch.empty((K, r), dtype=torch.bfloat16, device=dev) if dA is None else dA
-    dB = torch.empty((r, N), dtype=torch.bfloat16, device=dev) if dB is None else dB
-    _req(dX, "dX", torch.bfloat16, (M, K))
-    _req(dA, "dA", torch.bfloat16, (K, r))
-    _req(dB, "dB", torch.bfloat16, (r, N))
+    dX = torch.empty((M, K), dtype=dt, device=dev) if dX is None else dX
+    dA = torch.empty((K, r), dtype=dt, device=dev) if dA is None else dA
+    dB = torch.empty((r, N), dtype=dt, device=dev) if dB is None else dB
+    _req(dX, "dX", dt, (M, K))
+    _req(dA, "dA", dt, (K, r))
+    _req(dB, "dB", dt, (r, N))
     workspace = _workspace(workspace, M, N, K, r, dev)
     tb = _tables(nf4, t8)
-    _check(load().qlora_linear_bwd(_ptr(packed), _ptr(q), _ptr(scale2), tb.nf4, tb.t8, M, N, K, _ptr(X),
-                                   _ptr(dY), _ptr(A), _ptr(B), _ptr(XA), r, float(alpha), _ptr(dX), _ptr(dA),
-                                   _ptr(dB), _ptr(workspace), workspace.numel(), _stream()),
-           "qlora_linear_bwd")
+    if dt == torch.bfloat16:
+        _check(load().qlora_linear_bwd(_ptr(packed), _ptr(q), _ptr(scale2), tb.nf4, tb.t8, M, N, K, _ptr(X),
+                                       _ptr(dY), _ptr(A), _ptr(B), _ptr(XA), r, float(alpha), _ptr(dX),
+                                       _ptr(dA), _ptr(dB), _ptr(workspace), workspace.numel(), _stream()),
+               "qlora_linear_bwd")
+    else:
+        _check(load().qlora_linear_bwd_dt(_ptr(packed), _ptr(q), _ptr(scale2), tb.nf4, tb.t8, _DTYPE[dt], M, N,
+                                          K, _ptr(X), _ptr(dY), _ptr(A), _ptr(B), _ptr(XA), r, float(alpha),
+                                          _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), workspace.numel(),
+                                          _stream()), "qlora_linear_bwd_dt")
     return dX, dA, dB

@@ -328,10 +328,10 @@ struct Nf4Planes {
   uint32_t alo0, alo1, ahi0, ahi1, blo0, blo1, bhi0, bhi1;
 };
 
-__device__ __forceinline__ Nf4Planes make_planes(const float (&L)[16], float cp) {
+__device__ __forceinline__ Nf4Planes make_planes(const float (&L)[16], float cp, bool f16 = false) {
   uint32_t t[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) t[j] = pack_bf16x2(__fmul_rn(L[2 * j], cp), __fmul_rn(L[2 * j + 1], cp));
+  for (int j = 0; j < 8; ++j) t[j] = pack_16x2(__fmul_rn(L[2 * j], cp), __fmul_rn(L[2 * j + 1], cp), f16);
   Nf4Planes p;
   p.alo0 = prmt(t[0], t[1], 0x6420u);
   p.alo1 = prmt(t[2], t[3], 0x6420u);
@@ -364,15 +364,17 @@ __device__ __forceinline__ void nf4_lookup8(const Nf4Planes &P, uint32_t w, uint
   }
 }
 
-// Standalone dequantization: one lane per 64-block (its bf16 table built
-// once), 32 consecutive blocks per warp. Each lane writes its 128 output
+// Standalone dequantization to bf16, or to fp16 when f16 is set (the pages'
+// compute types, systemoverflow.com "QLoRA ... at Extreme Scale": 16-bit
+// float or bfloat16): one lane per 64-block (its 16-bit table built once),
+// 32 consecutive blocks per warp. Each lane writes its 128 output
 // bytes into a padded shared-memory row, and the warp then stores the 4 KB
 // with fully coalesced 16-byte stores.
 __global__ void __launch_bounds__(256) dequant_kernel(const uint4 *__restrict__ packed,
                                                       const uint8_t *__restrict__ q,
                                                       const float *__restrict__ scale2,
                                                       int64_t nblocks, uint4 *__restrict__ out,
-                                                      const CodecTables tabs) {
+                                                      const CodecTables tabs, int f16) {
   __shared__ float s_t8[256];
   __shared__ uint4 s_stage[8][32 * 9];  // per warp: 32 rows of 128 B, padded to 144 B
   s_t8[threadIdx.x] = tabs.t8[threadIdx.x];
@@ -408,7 +410,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint4 *__restrict__ 
     const uint4 w0 = n0, w1 = n1;
     const float cp = __fmul_rn(s_t8[nq], ns);
     if (b0 + nwarps * 32 < nblocks) load(b0 + nwarps * 32 + lane);
-    const Nf4Planes P = make_planes(L, cp);
+    const Nf4Planes P = make_planes(L, cp, f16 != 0);
     const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
     for (int c = 0; c < 8; ++c) {

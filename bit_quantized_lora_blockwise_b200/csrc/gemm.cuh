@@ -71,7 +71,7 @@ struct GemmArgs {
   CUtensorMap tm_a2;  // low-rank A2
   CUtensorMap tm_b2;  // low-rank B2 [tokens, r]: box {64, B_ROWS}
   CUtensorMap tm_cp;  // decoded block constants c' [K/64][N] fp32
-  // Output: bf16 out[col * out_ld + row] (the transposed tile).
+  // Output: 16-bit (bf16, or fp16 when f16) out[col * out_ld + row] (the transposed tile).
   void *out;
   int64_t out_ld;
   float *part;             // fp32 partials of split tiles [tail_splits][tail tiles][tile columns][TILE_ROWS]
@@ -88,6 +88,7 @@ struct GemmArgs {
   int tail_splits;
   int tail_subtiles;
   int lora_kblocks;       // 64-deep K blocks of the low-rank product (last split only)
+  int f16;                // operands, decoded weight and output are fp16 (else bf16)
   float nf4[16];
 };
 
@@ -362,8 +363,9 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     if (lane == 0 && rank == 0) {
       constexpr uint64_t DK = smem_desc_const(16, 1024);    // K-major, 128B swizzle
       constexpr uint64_t DM = smem_desc_const(8192, 1024);  // MN-major, 128B swizzle
-      constexpr uint32_t ID_MAIN = make_idesc_bf16(C::TILE_ROWS, C::BN, C::A_MN ? 1 : 0, 0);
-      constexpr uint32_t ID_LORA = make_idesc_bf16(C::TILE_ROWS, C::BN, C::L2 == L2_A_MN ? 1 : 0, 0);
+      const uint32_t ID_MAIN = idesc_dtype(make_idesc_bf16(C::TILE_ROWS, C::BN, C::A_MN ? 1 : 0, 0), args.f16);
+      const uint32_t ID_LORA =
+          idesc_dtype(make_idesc_bf16(C::TILE_ROWS, C::BN, C::L2 == L2_A_MN ? 1 : 0, 0), args.f16);
       auto wait_full = [&](uint32_t bar, uint32_t par) -> bool {
         return mbar_try_wait(bar, par) || mbar_wait(bar, par, s_abort);
       };
@@ -476,10 +478,11 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     auto store_out = [&](int row, int tok, const float (&v)[32]) {
       if (row >= args.rows) return;
       const int ncol = args.cols - tok < 32 ? args.cols - tok : 32;
-      __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(args.out);
+      uint16_t *dst = reinterpret_cast<uint16_t *>(args.out);
+      const bool f16 = args.f16 != 0;
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        if (j < ncol) dst[static_cast<int64_t>(tok + j) * args.out_ld + row] = __float2bfloat16_rn(v[j]);
+        if (j < ncol) dst[static_cast<int64_t>(tok + j) * args.out_ld + row] = to_16(v[j], f16);
     };
     bool ok = true;
     for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step, ++iter) {
@@ -647,7 +650,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
             L[4 * i + 2] = l4.z;
             L[4 * i + 3] = l4.w;
           }
-          const Nf4Planes P = make_planes(L, cp);
+          const Nf4Planes P = make_planes(L, cp, args.f16 != 0);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             uint32_t o[4];

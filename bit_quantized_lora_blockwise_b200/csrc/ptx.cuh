@@ -8,6 +8,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace qlora {
@@ -245,6 +246,22 @@ __device__ __forceinline__ void mma_16816_bf16(float (&d)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// The same with fp16 operands.
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+template <bool F16>
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  if constexpr (F16) mma_16816_f16(d, a0, a1, a2, a3, b0, b1);
+  else mma_16816_bf16(d, a0, a1, a2, a3, b0, b1);
+}
+
 // 4-byte asynchronous global -> shared copy (cache-all), grouped by
 // cp.async.commit_group / cp.async.wait_group.
 __device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src) {
@@ -388,6 +405,14 @@ __host__ __device__ constexpr uint64_t smem_desc_const(uint32_t lbo, uint32_t sb
          (1ull << 46) | (2ull << 61);
 }
 
+// The A/B format fields of a kind::f16 instruction descriptor (bits 7-9
+// and 10-12: 0 = f16, 1 = bf16); clearing them turns a bf16 descriptor into
+// the fp16 one.
+constexpr uint32_t kIdescAbFormat = (7u << 7) | (7u << 10);
+__host__ __device__ constexpr uint32_t idesc_dtype(uint32_t id_bf16, bool f16) {
+  return f16 ? (id_bf16 & ~kIdescAbFormat) : id_bf16;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B, fp32 accumulator.
 __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, int a_mn_major,
                                                       int b_mn_major) {
@@ -432,6 +457,20 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), RNE
   return *reinterpret_cast<uint32_t *>(&v);
+}
+// IEEE binary16 pair, round to nearest even (out of range -> +-inf).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);  // .x = lo (low half)
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+// 16-bit operand pair in the compute type (fp16 when f16, else bf16).
+__device__ __forceinline__ uint32_t pack_16x2(float lo, float hi, bool f16) {
+  return f16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+}
+// One output element in the compute type.
+__device__ __forceinline__ uint16_t to_16(float v, bool f16) {
+  if (f16) return __half_as_ushort(__float2half_rn(v));
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 
 }  // namespace qlora

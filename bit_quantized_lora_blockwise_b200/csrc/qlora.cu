@@ -41,6 +41,16 @@ DeviceInfo g_dev[kMaxDevices];
 std::atomic<uint64_t> g_launches{0};
 thread_local cudaEvent_t t_trace_start = nullptr;
 thread_local cudaEvent_t t_trace_stop = nullptr;
+// Compute type of the call in progress on this thread (set by the entry
+// points for the duration of one call): fp16 operands and outputs when true,
+// else bf16. Every launch of the call reads it.
+thread_local bool t_f16 = false;
+struct DtypeScope {
+  explicit DtypeScope(bool f16) { t_f16 = f16; }
+  ~DtypeScope() { t_f16 = false; }
+  DtypeScope(const DtypeScope &) = delete;
+  DtypeScope &operator=(const DtypeScope &) = delete;
+};
 
 
 qlora_status device_info(DeviceInfo *out) {
@@ -597,6 +607,7 @@ qlora_status skinny_launch(SkinnyKind kind, const SkinnyOperands *ops, int nprob
   a.nzero = nzero;
   a.early = early ? 1 : 0;
   a.late = late ? 1 : 0;
+  a.f16 = t_f16 ? 1 : 0;
   a.gemm_ctas = (row_tiles[0] + row_tiles[1]) * p.splits;
   int grid = a.gemm_ctas;
   if (dc != nullptr) {
@@ -761,7 +772,7 @@ int skinny_ctas(int64_t rows, int64_t kdim, int r) {
   return static_cast<int>(cdiv(rows, 128)) * p.splits;
 }
 
-template <int NT>
+template <int NT, bool F16>
 qlora_status run_smallm_nt(const SmallmArgs &a, int grid, cudaStream_t st) {
   using C = SmallmCfg<NT>;
   static std::once_flag once[kMaxDevices];
@@ -769,14 +780,16 @@ qlora_status run_smallm_nt(const SmallmArgs &a, int grid, cudaStream_t st) {
   cudaGetDevice(&dev);
   cudaError_t attr_err = cudaSuccess;
   std::call_once(once[dev], [&] {
-    attr_err = cudaFuncSetAttribute(smallm_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    attr_err =
+        cudaFuncSetAttribute(smallm_kernel<NT, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return QLORA_ERR_CUDA;
-  return launch_pdl(smallm_kernel<NT>, grid, C::THREADS, C::SMEM_BYTES, st, a);
+  return launch_pdl(smallm_kernel<NT, F16>, grid, C::THREADS, C::SMEM_BYTES, st, a);
 }
 
 qlora_status run_smallm(const SmallmArgs &a, const SmallmPlan &p, cudaStream_t st) {
-  return p.nt == 1 ? run_smallm_nt<1>(a, p.grid, st) : run_smallm_nt<2>(a, p.grid, st);
+  if (t_f16) return p.nt == 1 ? run_smallm_nt<1, true>(a, p.grid, st) : run_smallm_nt<2, true>(a, p.grid, st);
+  return p.nt == 1 ? run_smallm_nt<1, false>(a, p.grid, st) : run_smallm_nt<2, false>(a, p.grid, st);
 }
 
 // Workspace carve-up: [tile counters][bf16 M x r][bf16 M x r (backward)][c'][fp32 partials]
@@ -995,7 +1008,7 @@ qlora_status qlora_dequant(const uint8_t *packed, const uint8_t *q, const float 
   const int grid = grid_for(nblocks, 256, d.sms, resident_per_sm<dequant_kernel>(256));
   return launch_pdl(dequant_kernel, grid, 256, 0, static_cast<cudaStream_t>(stream),
                     reinterpret_cast<const uint4 *>(packed), q, scale2, nblocks, reinterpret_cast<uint4 *>(W_out),
-                    make_tables(nf4, t8));
+                    make_tables(nf4, t8), t_f16 ? 1 : 0);
 }
 
 qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const float *scale2, const float nf4[16],
@@ -1037,9 +1050,9 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
       return QLORA_ERR_CUDA;
     a.q = q;
     a.scale2 = scale2;
-    a.B = reinterpret_cast<const __nv_bfloat16 *>(B);
-    a.xas = reinterpret_cast<const __nv_bfloat16 *>(xas);
-    a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
+    a.B = B;
+    a.xas = xas;
+    a.Y = Y;
     a.part = part;
     a.counters = counters;
     a.N = N;
@@ -1089,6 +1102,7 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   a.part = part;
   a.counters = counters;
   std::memcpy(a.nf4, nf4, sizeof a.nf4);
+  a.f16 = t_f16 ? 1 : 0;
   trace_begin(cs);
   st = fp.pair ? (fp.ntt == 2 ? run_fused_pair<FwdPair2Cfg>(a, d.sms, fp.slots, cs)
                               : run_fused_pair<FwdPairCfg>(a, d.sms, fp.slots, cs))
@@ -1166,6 +1180,7 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   a.part = part;
   a.counters = counters;
   std::memcpy(a.nf4, nf4, sizeof a.nf4);
+  a.f16 = t_f16 ? 1 : 0;
   trace_begin(cs);
   st = fp.pair ? (fp.ntt == 2 ? run_fused_pair<BwdPair2Cfg>(a, d.sms, fp.slots, cs)
                               : run_fused_pair<BwdPairCfg>(a, d.sms, fp.slots, cs))
@@ -1185,6 +1200,40 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
       {X, K, M, gs, r, M, K, M, OutSpec{dA, r, 1.0f, nullptr, 0, 0.0f, false}},
       {dY, N, M, xa, r, M, N, M, OutSpec{dB, N, scl, nullptr, 0, 0.0f, true}}};
   return skinny_launch(SK_DA, ops, 2, r, d.sms, cs, nullptr, 0, true, nullptr, true);
+}
+
+qlora_status qlora_dequant_dt(const uint8_t *packed, const uint8_t *q, const float *scale2, int64_t N, int64_t K,
+                              const float nf4[16], const float t8[256], qlora_dtype dtype, void *W_out,
+                              qlora_stream_t stream) {
+  if (dtype != QLORA_BF16 && dtype != QLORA_F16) return QLORA_ERR_RANGE;
+  DtypeScope scope(dtype == QLORA_F16);
+  return qlora_dequant(packed, q, scale2, N, K, nf4, t8, static_cast<qlora_bf16 *>(W_out), stream);
+}
+
+qlora_status qlora_linear_fwd_dt(const uint8_t *packed, const uint8_t *q, const float *scale2, const float nf4[16],
+                                 const float t8[256], qlora_dtype dtype, int64_t M, int64_t N, int64_t K,
+                                 const void *X, const void *A, const void *B, int r, float alpha, void *Y,
+                                 void *XA_out, void *workspace, size_t workspace_bytes, qlora_stream_t stream) {
+  if (dtype != QLORA_BF16 && dtype != QLORA_F16) return QLORA_ERR_RANGE;
+  DtypeScope scope(dtype == QLORA_F16);
+  return qlora_linear_fwd(packed, q, scale2, nf4, t8, M, N, K, static_cast<const qlora_bf16 *>(X),
+                          static_cast<const qlora_bf16 *>(A), static_cast<const qlora_bf16 *>(B), r, alpha,
+                          static_cast<qlora_bf16 *>(Y), static_cast<qlora_bf16 *>(XA_out), workspace,
+                          workspace_bytes, stream);
+}
+
+qlora_status qlora_linear_bwd_dt(const uint8_t *packed, const uint8_t *q, const float *scale2, const float nf4[16],
+                                 const float t8[256], qlora_dtype dtype, int64_t M, int64_t N, int64_t K,
+                                 const void *X, const void *dY, const void *A, const void *B, const void *XA, int r,
+                                 float alpha, void *dX, void *dA, void *dB, void *workspace, size_t workspace_bytes,
+                                 qlora_stream_t stream) {
+  if (dtype != QLORA_BF16 && dtype != QLORA_F16) return QLORA_ERR_RANGE;
+  DtypeScope scope(dtype == QLORA_F16);
+  return qlora_linear_bwd(packed, q, scale2, nf4, t8, M, N, K, static_cast<const qlora_bf16 *>(X),
+                          static_cast<const qlora_bf16 *>(dY), static_cast<const qlora_bf16 *>(A),
+                          static_cast<const qlora_bf16 *>(B), static_cast<const qlora_bf16 *>(XA), r, alpha,
+                          static_cast<qlora_bf16 *>(dX), static_cast<qlora_bf16 *>(dA), static_cast<qlora_bf16 *>(dB),
+                          workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

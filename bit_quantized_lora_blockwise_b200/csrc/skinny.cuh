@@ -50,6 +50,7 @@ struct SkinnyArgs {
   int late;   // 1: every operand is complete when this launch starts and nothing it writes is touched by
               // the kernel before it, so the whole product runs without waiting for that kernel; each
               // thread waits for it only before exiting, so this grid still completes after it
+  int f16;   // operands and outputs are fp16 (else bf16)
   // Optional constants pass for the fused GEMM that follows, run by the CTAs
   // from gemm_ctas on (whole clusters): cprime[kb * dc_N + n] = t8[q] * S.
   int gemm_ctas;
@@ -189,7 +190,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_cons
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = make_idesc_bf16(128, C::BN, C::A_MN ? 1 : 0, C::B_MN ? 1 : 0);
+      const uint32_t idesc = idesc_dtype(make_idesc_bf16(128, C::BN, C::A_MN ? 1 : 0, C::B_MN ? 1 : 0), args.f16);
       bool ok = true;
       for (int j = 0; j < nk; ++j) {
         const int s = j % C::STAGES;
@@ -282,7 +283,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_cons
       if (row >= P.rows) continue;
       const float vv[4] = {v.x, v.y, v.z, v.w};
       for (int o = 0; o < 2; ++o) {
-        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(o ? P.out2 : P.out);
+        uint16_t *dst = reinterpret_cast<uint16_t *>(o ? P.out2 : P.out);
         if (dst == nullptr) continue;
         const float sc = o ? P.out2_scale : P.out_scale;
         const int64_t ld = o ? P.out2_ld : P.out_ld;
@@ -292,7 +293,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_cons
           if (col >= P.cols) continue;
           const int64_t idx = P.transpose ? static_cast<int64_t>(col) * ld + row
                                              : static_cast<int64_t>(row) * ld + col;
-          dst[idx] = __float2bfloat16_rn(vv[e] * sc);
+          dst[idx] = to_16(vv[e] * sc, args.f16 != 0);
         }
       }
     }

@@ -49,9 +49,9 @@ struct SmallmArgs {
   CUtensorMap tm_w;          // packed [N, K/2] u8; box {128, 256}, 128B swizzle
   const uint8_t *q;          // [N K / 64] 8-bit block-constant codes
   const float *scale2;       // [ceil(N K / 64 / 256)] second-level scales
-  const __nv_bfloat16 *B;    // [r, N]
-  const __nv_bfloat16 *xas;  // [M, r] = bf16((alpha / r) X A)
-  __nv_bfloat16 *Y;          // [M, N]
+  const uint16_t *B;         // [r, N] (16-bit: bf16, or fp16 in the fp16 build)
+  const uint16_t *xas;       // [M, r] = 16-bit((alpha / r) X A)
+  uint16_t *Y;               // [M, N]
   float *part;               // partial slots: [grid][2][16 warps][NT][32 lanes][4]
   unsigned int *counters;    // one per band, zero on entry (left zero): pieces parked
   int64_t N, K;
@@ -90,7 +90,7 @@ __host__ __device__ __forceinline__ int smallm_unit_begin(int64_t cta, int64_t u
   return static_cast<int>(cta * units / grid);
 }
 
-template <int NT>
+template <int NT, bool F16>
 __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const __grid_constant__ SmallmArgs a) {
   using C = SmallmCfg<NT>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
     for (int q = 0; q < 4; ++q)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
-        mma_16816_bf16(acc[nt], L.af[q][0], L.af[q][1], L.af[q][2], L.af[q][3], L.bf[q][nt][0], L.bf[q][nt][1]);
+        mma_16816<F16>(acc[nt], L.af[q][0], L.af[q][1], L.af[q][2], L.af[q][3], L.bf[q][nt][0], L.bf[q][nt][1]);
   };
   auto band_row0 = [&](int band) { return static_cast<int64_t>(band) * C::BAND + warp * 16; };
   auto store_y = [&](int64_t n0) {
@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
       for (int e = 0; e < 4; ++e) {
         const int m = 8 * nt + 2 * t + (e & 1);
         const int64_t n = n0 + g + 8 * (e >> 1);
-        if (m < a.M) a.Y[static_cast<int64_t>(m) * a.N + n] = __float2bfloat16_rn(acc[nt][e]);
+        if (m < a.M) a.Y[static_cast<int64_t>(m) * a.N + n] = to_16(acc[nt][e], F16);
       }
   };
   // after the stream (registers free): first 64 ranks preloaded
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
         const uint32_t *xr = reinterpret_cast<const uint32_t *>(a.xas + static_cast<int64_t>(m) * a.r);
         const uint32_t b0 = (m < a.M && ja < a.r) ? xr[ja >> 1] : 0u;
         const uint32_t b1 = (m < a.M && jb < a.r) ? xr[jb >> 1] : 0u;
-        mma_16816_bf16(acc[nt], a0, a1, a2, a3, b0, b1);
+        mma_16816<F16>(acc[nt], a0, a1, a2, a3, b0, b1);
       }
     }
     store_y(n0);
@@ -298,8 +298,8 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
     if (!__all_sync(0xFFFFFFFFu, mbar_wait_spin(full_bar(s), (i / C::SX) & 1u, s_abort))) return false;
     const bool rows_here = static_cast<int64_t>(cur_band) * C::BAND + warp * 16 < a.N;
     if (rows_here) {
-      const Nf4Planes P0 = make_planes(a.tabs.nf4, cp0);
-      const Nf4Planes P1 = make_planes(a.tabs.nf4, cp1);
+      const Nf4Planes P0 = make_planes(a.tabs.nf4, cp0, F16);
+      const Nf4Planes P1 = make_planes(a.tabs.nf4, cp1, F16);
       const uint32_t ws = wrow + s * C::STAGE;
       const uint4 r0a = lds_16B(ws + wc0), r0b = lds_16B(ws + wc1);
       const uint4 r1a = lds_16B(ws + 8 * 128 + wc0), r1b = lds_16B(ws + 8 * 128 + wc1);
@@ -315,8 +315,8 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const uint4 xv = lds_16B(xa + nt * (8 * 4 * 128));
-          mma_16816_bf16(acc[nt], o0[0], o1[0], o0[1], o1[1], xv.x, xv.y);
-          mma_16816_bf16(acc[nt], o0[2], o1[2], o0[3], o1[3], xv.z, xv.w);
+          mma_16816<F16>(acc[nt], o0[0], o1[0], o0[1], o1[1], xv.x, xv.y);
+          mma_16816<F16>(acc[nt], o0[2], o1[2], o0[3], o1[3], xv.z, xv.w);
         }
       }
     }

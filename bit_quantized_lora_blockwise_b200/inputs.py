@@ -90,6 +90,15 @@ def normal_bf16(shape, std: float, seed: int, device="cpu") -> torch.Tensor:
     return x.to(torch.bfloat16)
 
 
+def normal_f16(shape, std: float, seed: int, device="cpu") -> torch.Tensor:
+    """N(0, std^2) samples drawn in fp32 and rounded to fp16."""
+    g = _gen(seed, device)
+    x = torch.randn(tuple(shape), generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(torch.float16)
+
+
 def weight_bf16(N: int, K: int, std: float, seed: int, outlier_frac: float = 0.0,
                 outlier_sigma: float = 10.0, device="cpu") -> torch.Tensor:
     """Frozen base weight [N, K]: N(0, std^2), with a fraction of entries at
@@ -122,4 +131,9 @@ def layer_inputs(wl: Workload, li: int, M: int, device="cpu", layer: int = 0,
 
 def bf16_bits(t: torch.Tensor):
     """uint16 numpy view of a bf16 tensor's bit patterns (host copy)."""
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view("uint16")
+
+
+def f16_bits(t: torch.Tensor):
+    """uint16 numpy view of an fp16 tensor's bit patterns (host copy)."""
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view("uint16")

@@ -45,7 +45,7 @@ extern "C" {
 #define QLORA_API
 #endif
 
-#define QLORA_ABI_VERSION 1
+#define QLORA_ABI_VERSION 2
 #define QLORA_BLOCK 64          /* weights per absmax constant (DL0087 component 2)        */
 #define QLORA_DQ_BLOCK 256      /* constants per second-level fp32 scale (DL0087 comp. 3) */
 #define QLORA_NF4_LEVELS 16     /* 4-bit code -> level table                              */
@@ -203,6 +203,42 @@ QLORA_API qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q,
                               const qlora_bf16 *X, const qlora_bf16 *dY,
                               const qlora_bf16 *A, const qlora_bf16 *B, const qlora_bf16 *XA,
                               int r, float alpha, qlora_bf16 *dX, qlora_bf16 *dA, qlora_bf16 *dB,
+                              void *workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/*
+ * Compute type of the 16-bit tensors of a call (systemoverflow.com "QLoRA:
+ * Efficient Finetuning of Quantized LLMs at Extreme Scale": the adapters and
+ * the computation run in 16-bit float or bfloat16). With QLORA_F16 every
+ * 16-bit operand and output is IEEE binary16 instead of bf16: the
+ * dequantized weight is W'[e] = f16_rne(nf4[code_e] * c'_b) (fp32 product;
+ * magnitudes beyond 65504 round to +-inf, small ones to fp16 subnormals),
+ * the tensor-core MMAs take fp16 A and B, accumulation stays fp32 and every
+ * output (including X A and the scaled s X A the low-rank step uses) is
+ * rounded to fp16. The packed codes and constants are the same for both.
+ */
+typedef enum { QLORA_BF16 = 0, QLORA_F16 = 1 } qlora_dtype;
+
+/*
+ * qlora_dequant, qlora_linear_fwd and qlora_linear_bwd with the compute type
+ * as an argument; the 16-bit pointers are bf16 or fp16 bit patterns as
+ * `dtype` says. Same requirements, ownership and error behaviour as the bf16
+ * calls above (which are these with QLORA_BF16); a dtype other than the two
+ * values returns QLORA_ERR_RANGE and launches nothing.
+ */
+QLORA_API qlora_status qlora_dequant_dt(const uint8_t *packed, const uint8_t *q, const float *scale2,
+                              int64_t N, int64_t K, const float nf4[16], const float t8[256],
+                              qlora_dtype dtype, void *W_out, qlora_stream_t stream);
+QLORA_API qlora_status qlora_linear_fwd_dt(const uint8_t *packed, const uint8_t *q, const float *scale2,
+                              const float nf4[16], const float t8[256], qlora_dtype dtype,
+                              int64_t M, int64_t N, int64_t K,
+                              const void *X, const void *A, const void *B,
+                              int r, float alpha, void *Y, void *XA_out,
+                              void *workspace, size_t workspace_bytes, qlora_stream_t stream);
+QLORA_API qlora_status qlora_linear_bwd_dt(const uint8_t *packed, const uint8_t *q, const float *scale2,
+                              const float nf4[16], const float t8[256], qlora_dtype dtype,
+                              int64_t M, int64_t N, int64_t K,
+                              const void *X, const void *dY, const void *A, const void *B, const void *XA,
+                              int r, float alpha, void *dX, void *dA, void *dB,
                               void *workspace, size_t workspace_bytes, qlora_stream_t stream);
 
 /*

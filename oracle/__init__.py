@@ -32,7 +32,7 @@ from .linear import (linear_fwd, linear_bwd, linear_fwd_rows, linear_bwd_rows,
 
 __all__ = [
     "BLOCK", "DQ_BLOCK", "nf4_levels", "dq_levels", "nearest_level",
-    "absmax", "encode_nf4", "quantize_nf4", "double_quant", "dequant",
+    "absmax", "encode_nf4", "quantize_nf4", "double_quant", "dequant", "dequant_f16", "f32_to_f16",
     "dq_constants", "bf16_to_f32", "f32_to_bf16", "linear_fwd", "linear_bwd",
     "linear_fwd_rows", "linear_bwd_rows", "bf16_bits_to_f64", "build",
 ]
@@ -77,6 +77,8 @@ def _load():
             lib.oracle_dq_constants.argtypes = [P, P, I64, P, P]
             lib.oracle_bf16_to_f32.argtypes = [P, I64, P]
             lib.oracle_f32_to_bf16.argtypes = [P, I64, P]
+            lib.oracle_dequant_f16.argtypes = [P, P, P, I64, P, P, P]
+            lib.oracle_f32_to_f16.argtypes = [P, I64, P]
             _lib = lib
     return _lib
 
@@ -160,6 +162,28 @@ def dequant(packed: np.ndarray, q: np.ndarray, scale2: np.ndarray, n_elems: int,
     out = np.zeros(n_elems, np.uint16)
     _load().oracle_dequant(_ptr(packed), _ptr(q), _ptr(scale2), n_elems, _ptr(lv),
                            _ptr(t8), _ptr(out))
+    return out
+
+
+def dequant_f16(packed: np.ndarray, q: np.ndarray, scale2: np.ndarray, n_elems: int,
+                levels: np.ndarray | None = None, t8: np.ndarray | None = None) -> np.ndarray:
+    """fp16 bit patterns of the dequantized weight (flat, n_elems)."""
+    lv = nf4_levels() if levels is None else np.ascontiguousarray(levels, np.float32)
+    t8 = dq_levels() if t8 is None else np.ascontiguousarray(t8, np.float32)
+    packed = np.ascontiguousarray(packed, np.uint8).reshape(-1)
+    q = np.ascontiguousarray(q, np.uint8).reshape(-1)
+    scale2 = np.ascontiguousarray(scale2, np.float32).reshape(-1)
+    out = np.zeros(n_elems, np.uint16)
+    _load().oracle_dequant_f16(_ptr(packed), _ptr(q), _ptr(scale2), n_elems, _ptr(lv),
+                               _ptr(t8), _ptr(out))
+    return out
+
+
+def f32_to_f16(x: np.ndarray) -> np.ndarray:
+    """fp16 bit patterns of x (round to nearest even)."""
+    x = np.ascontiguousarray(x, np.float32)
+    out = np.zeros(x.shape, np.uint16)
+    _load().oracle_f32_to_f16(_ptr(x), x.size, _ptr(out))
     return out
 
 

@@ -53,6 +53,40 @@ static uint16_t float_to_bf16_rne(float f) {
     return (uint16_t)(u >> 16);
 }
 
+/* binary32 -> IEEE 754 binary16 (1 sign, 5 exponent bits of bias 15, 10
+ * fraction bits) with round-to-nearest-even, on the bit patterns:
+ *   |f| >= 65520 (half-way above the largest finite 65504) -> inf;
+ *   2^-14 <= |f|: normal, the 23-bit fraction rounded to 10 bits (a carry
+ *                 out of the fraction correctly bumps the exponent);
+ *   |f| <  2^-14: subnormal, |f| / 2^-24 rounded to an integer (2^-24 is
+ *                 the subnormal unit; 1024 units become the least normal).
+ * NaN maps to the quiet NaN 0x7E00 with the input's sign. */
+static uint16_t float_to_f16_rne(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+    uint32_t a = u & 0x7FFFFFFFu;
+    if (a > 0x7F800000u) return (uint16_t)(sign | 0x7E00u);
+    if (a >= 0x477FF000u) return (uint16_t)(sign | 0x7C00u);
+    if (a >= 0x38800000u) {
+        uint32_t e = (a >> 23) - 127u + 15u;
+        uint32_t frac = a & 0x7FFFFFu;
+        uint32_t h = (e << 10) | (frac >> 13);
+        uint32_t rem = frac & 0x1FFFu;
+        if (rem > 0x1000u || (rem == 0x1000u && (h & 1u))) h += 1u;
+        return (uint16_t)(sign | h);
+    }
+    uint32_t E = a >> 23;             /* biased binary32 exponent, <= 112 here */
+    if (E < 102u) return sign;        /* |f| < 2^-25: rounds to (signed) zero */
+    uint32_t sig = (a & 0x7FFFFFu) | 0x800000u;  /* |f| = sig * 2^(E - 150)  */
+    uint32_t shift = 126u - E;        /* |f| / 2^-24 = sig / 2^shift, 14..24 */
+    uint32_t h = sig >> shift;
+    uint32_t rem = sig & ((1u << shift) - 1u);
+    uint32_t half = 1u << (shift - 1u);
+    if (rem > half || (rem == half && (h & 1u))) h += 1u;
+    return (uint16_t)(sign | h);
+}
+
 /* -------------------------------------------------------- NF4 levels ---- */
 
 /* Standard normal CDF in long double. */
@@ -214,6 +248,25 @@ void oracle_dequant(const uint8_t *packed, const uint8_t *q, const float *scale2
         float v = levels[code] * cprime;
         w_out[e] = float_to_bf16_rne(v);
     }
+}
+
+/* The same dequantization with an fp16 result (the pages' other 16-bit
+ * compute type, systemoverflow.com "QLoRA ... at Extreme Scale"):
+ * W'[e] = f16_rne( L[code_e] * c'_b ), the products as above. */
+void oracle_dequant_f16(const uint8_t *packed, const uint8_t *q, const float *scale2,
+                        int64_t n_elems, const float levels[16], const float t8[256],
+                        uint16_t *w_out) {
+    for (int64_t e = 0; e < n_elems; ++e) {
+        int64_t b = e / ORACLE_BLOCK;
+        float cprime = t8[q[b]] * scale2[b / ORACLE_DQ_BLOCK];
+        int code = (e & 1) ? (packed[e / 2] >> 4) : (packed[e / 2] & 0x0F);
+        float v = levels[code] * cprime;
+        w_out[e] = float_to_f16_rne(v);
+    }
+}
+
+void oracle_f32_to_f16(const float *f, int64_t n, uint16_t *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = float_to_f16_rne(f[i]);
 }
 
 /* The double-quantized constants c'_b alone (used by the round-trip pins). */

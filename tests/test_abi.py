@@ -38,7 +38,7 @@ def test_header_declares_the_five_calls():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_symbols():
         assert hasattr(lib, name), name
-    assert lib.qlora_abi_version() == 1
+    assert lib.qlora_abi_version() == 2
 
 
 def test_library_has_sm100a_code():
@@ -113,3 +113,21 @@ def test_argument_checks_before_any_launch(lib):
                                     _fake(), _fake(), _fake(), _fake(), None, a["r"], a["alpha"],
                                     _fake(), _fake(), _fake(), _fake(), 1 << 30, s)
     assert bwd(r=0) == 4 and bwd(r=257) == 4 and bwd(N=100) == 2 and bwd(alpha=float("nan")) == 4
+
+
+def test_dtype_argument_is_checked_first(lib):
+    """A compute type other than bf16 (0) and fp16 (1) is refused before any
+    other check or launch."""
+    tb = binding._tables(None, None)
+    s = ctypes.c_void_p(0)
+    for bad in (2, -1, 7):
+        assert lib.qlora_dequant_dt(_fake(), _fake(), _fake(), 64, 64, tb.nf4, tb.t8, bad, _fake(), s) == 4
+        assert lib.qlora_linear_fwd_dt(_fake(), _fake(), _fake(), tb.nf4, tb.t8, bad, 16, 128, 128, _fake(),
+                                       _fake(), _fake(), 8, 16.0, _fake(), None, _fake(), 1 << 30, s) == 4
+        assert lib.qlora_linear_bwd_dt(_fake(), _fake(), _fake(), tb.nf4, tb.t8, bad, 16, 128, 128, _fake(),
+                                       _fake(), _fake(), _fake(), None, 8, 16.0, _fake(), _fake(), _fake(),
+                                       _fake(), 1 << 30, s) == 4
+    # with a valid type the ordinary checks follow (r out of range)
+    assert lib.qlora_linear_fwd_dt(_fake(), _fake(), _fake(), tb.nf4, tb.t8, 1, 16, 128, 128, _fake(), _fake(),
+                                   _fake(), 0, 16.0, _fake(), None, _fake(), 1 << 30, s) == 4
+    assert lib.qlora_dequant_dt(None, _fake(), _fake(), 64, 64, tb.nf4, tb.t8, 1, _fake(), s) == 1
