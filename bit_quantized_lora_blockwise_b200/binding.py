@@ -34,7 +34,10 @@ EXPORTS = ("qlora_status_string", "qlora_abi_version", "qlora_nf4_levels", "qlor
            "qlora_workspace_bytes", "qlora_quantize_nf4", "qlora_double_quant", "qlora_dequant",
            "qlora_linear_fwd", "qlora_linear_bwd", "qlora_device_error", "qlora_set_trace_events",
            "qlora_launch_count", "qlora_linear_fwd_noalloc", "qlora_selftest_bounded_wait",
-           "qlora_dequant_dt", "qlora_linear_fwd_dt", "qlora_linear_bwd_dt")
+           "qlora_dequant_dt", "qlora_linear_fwd_dt", "qlora_linear_bwd_dt",
+           "qlora_paged_adamw_create", "qlora_paged_adamw_destroy", "qlora_paged_adamw_init",
+           "qlora_paged_adamw_step", "qlora_paged_adamw_set_reserve", "qlora_paged_adamw_placement",
+           "qlora_paged_adamw_location", "qlora_paged_adamw_state_bytes", "qlora_paged_adamw_state")
 
 # qlora_dtype of the 16-bit tensors of a call
 _DTYPE = {torch.bfloat16: 0, torch.float16: 1}
@@ -85,6 +88,25 @@ def load(path: str | None = None):
                                             P, P, SZ, P]
         for fn in ("qlora_dequant_dt", "qlora_linear_fwd_dt", "qlora_linear_bwd_dt"):
             getattr(lib, fn).restype = I32
+        PP = ctypes.POINTER(ctypes.c_void_p)
+        lib.qlora_paged_adamw_create.argtypes = [I32, ctypes.POINTER(I64), ctypes.POINTER(P)]
+        lib.qlora_paged_adamw_create.restype = I32
+        lib.qlora_paged_adamw_destroy.argtypes = [P]
+        lib.qlora_paged_adamw_destroy.restype = None
+        lib.qlora_paged_adamw_init.argtypes = [P, PP, I32, P]
+        lib.qlora_paged_adamw_init.restype = I32
+        lib.qlora_paged_adamw_step.argtypes = [P, PP, PP, I32, I64, F32, F32, F32, F32, F32, P]
+        lib.qlora_paged_adamw_step.restype = I32
+        lib.qlora_paged_adamw_set_reserve.argtypes = [P, SZ]
+        lib.qlora_paged_adamw_set_reserve.restype = I32
+        lib.qlora_paged_adamw_placement.argtypes = [SZ, SZ, SZ, I32]
+        lib.qlora_paged_adamw_placement.restype = I32
+        lib.qlora_paged_adamw_location.argtypes = [P]
+        lib.qlora_paged_adamw_location.restype = I32
+        lib.qlora_paged_adamw_state_bytes.argtypes = [P]
+        lib.qlora_paged_adamw_state_bytes.restype = SZ
+        lib.qlora_paged_adamw_state.argtypes = [P, PP, PP, PP]
+        lib.qlora_paged_adamw_state.restype = I32
         lib.qlora_device_error.argtypes = [I32]
         lib.qlora_device_error.restype = ctypes.c_uint32
         lib.qlora_set_trace_events.argtypes = [P, P]
@@ -384,3 +406,80 @@ def linear_bwd(packed, q, scale2, X, dY, A, B, alpha: float, N: int, K: int, XA=
                                           _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), workspace.numel(),
                                           _stream()), "qlora_linear_bwd_dt")
     return dX, dA, dB
+
+
+def paged_adamw_placement(free_bytes: int, state_bytes: int, reserve_bytes: int, current: int) -> int:
+    """The library's placement policy: 1 (state on the host) or 0 (device)."""
+    return int(load().qlora_paged_adamw_placement(free_bytes, state_bytes, reserve_bytes, current))
+
+
+class PagedAdamW:
+    """AdamW over 16-bit adapter tensors with its fp32 state (master copy and
+    moments) in unified memory that the library pages between device and
+    host by free device memory (qlora_paged_adamw_*)."""
+
+    def __init__(self, params, lr=1e-3, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.0):
+        self.params = list(params)
+        if not self.params:
+            raise ValueError("no parameters")
+        self.dtype = _dtype_of(self.params[0], "params[0]")
+        for i, p in enumerate(self.params):
+            _req(p, f"params[{i}]", self.dtype)
+        self.lr, self.betas, self.eps, self.weight_decay = lr, betas, eps, weight_decay
+        self.t = 0
+        lib = load()
+        counts = (ctypes.c_int64 * len(self.params))(*[p.numel() for p in self.params])
+        h = ctypes.c_void_p()
+        _check(lib.qlora_paged_adamw_create(len(self.params), counts, ctypes.byref(h)), "qlora_paged_adamw_create")
+        self._h = h
+        self._pp = (ctypes.c_void_p * len(self.params))(*[p.data_ptr() for p in self.params])
+        _check(lib.qlora_paged_adamw_init(self._h, self._pp, _DTYPE[self.dtype], _stream()), "qlora_paged_adamw_init")
+
+    def step(self, grads):
+        grads = list(grads)
+        if len(grads) != len(self.params):
+            raise ValueError("one gradient per parameter")
+        for i, (g, p) in enumerate(zip(grads, self.params)):
+            _req(g, f"grads[{i}]", self.dtype, tuple(p.shape))
+        gp = (ctypes.c_void_p * len(grads))(*[g.data_ptr() for g in grads])
+        self.t += 1
+        _check(load().qlora_paged_adamw_step(self._h, self._pp, gp, _DTYPE[self.dtype], self.t, float(self.lr),
+                                             float(self.betas[0]), float(self.betas[1]), float(self.eps),
+                                             float(self.weight_decay), _stream()), "qlora_paged_adamw_step")
+
+    def set_reserve(self, reserve_bytes: int):
+        _check(load().qlora_paged_adamw_set_reserve(self._h, int(reserve_bytes)), "qlora_paged_adamw_set_reserve")
+
+    @property
+    def location(self) -> str:
+        return "host" if load().qlora_paged_adamw_location(self._h) == 1 else "device"
+
+    @property
+    def state_bytes(self) -> int:
+        return int(load().qlora_paged_adamw_state_bytes(self._h))
+
+    def state(self):
+        """Host copies (numpy float32) of the master copy and the moments,
+        concatenated over the tensors in order; synchronizes the device."""
+        torch.cuda.synchronize()
+        pm, pm1, pv = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
+        _check(load().qlora_paged_adamw_state(self._h, ctypes.byref(pm), ctypes.byref(pm1), ctypes.byref(pv)),
+               "qlora_paged_adamw_state")
+        n = sum(p.numel() for p in self.params)
+        out = []
+        for ptr in (pm, pm1, pv):
+            a = np.empty(n, np.float32)
+            ctypes.memmove(a.ctypes.data, ptr.value, n * 4)
+            out.append(a)
+        return tuple(out)
+
+    def close(self):
+        if getattr(self, "_h", None):
+            load().qlora_paged_adamw_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

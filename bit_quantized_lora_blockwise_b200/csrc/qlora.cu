@@ -12,12 +12,14 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "qlora.h"
 #include "codec.cuh"
 #include "gemm.cuh"
 #include "skinny.cuh"
 #include "smallm.cuh"
+#include "adamw.cuh"
 #include "ptx.cuh"
 
 using namespace qlora;
@@ -1305,6 +1307,192 @@ uint32_t qlora_device_error(int clear) {
     if (cudaMemcpyToSymbol(g_error_word, &z, sizeof z) != cudaSuccess) return 0xFFFFFFFFu;
   }
   return v;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------- paged AdamW --
+struct qlora_paged_adamw {
+  int device = 0;
+  std::vector<int64_t> offset;  // nseg + 1 element offsets
+  int64_t total = 0;            // elements (each of master, m, v holds `total` floats)
+  int64_t stride = 0;           // floats between master, m and v (total rounded up to 64)
+  float *state = nullptr;       // managed: master | m | v
+  size_t bytes = 0;
+  size_t reserve = 0;
+  int where = 0;                // 0: device, 1: host
+  bool hints = false;           // the device takes prefetch and placement hints
+};
+
+namespace {
+
+// Page the state to `to` (0: device, 1: host) with placement hints and an
+// asynchronous prefetch on `st`.
+qlora_status adamw_place(qlora_paged_adamw *o, int to, cudaStream_t st) {
+  if (o->hints) {
+    const int loc = to == 1 ? cudaCpuDeviceId : o->device;
+    if (cudaMemAdvise(o->state, o->bytes, cudaMemAdviseSetPreferredLocation, loc) != cudaSuccess ||
+        (to == 1 && cudaMemAdvise(o->state, o->bytes, cudaMemAdviseSetAccessedBy, o->device) != cudaSuccess) ||
+        cudaMemPrefetchAsync(o->state, o->bytes, loc, st) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+  }
+  o->where = to;
+  return QLORA_OK;
+}
+
+// One launch per kAdamwMaxSegs segments; `init` selects the start kernel.
+qlora_status adamw_launch(qlora_paged_adamw *o, void *const *params, const void *const *grads, bool init,
+                          const AdamwHyper &h, cudaStream_t st) {
+  DeviceInfo d;
+  qlora_status status = device_info(&d);
+  if (status != QLORA_OK) return status;
+  const int nseg = static_cast<int>(o->offset.size()) - 1;
+  for (int s0 = 0; s0 < nseg; s0 += kAdamwMaxSegs) {
+    const int n = std::min(kAdamwMaxSegs, nseg - s0);
+    AdamwSegs segs;
+    std::memset(&segs, 0, sizeof segs);
+    for (int i = 0; i < n; ++i) {
+      segs.param[i] = params[s0 + i];
+      segs.grad[i] = grads ? grads[s0 + i] : nullptr;
+      segs.offset[i] = o->offset[s0 + i] - o->offset[s0];
+    }
+    segs.offset[n] = o->offset[s0 + n] - o->offset[s0];
+    segs.nseg = n;
+    const int64_t base = o->offset[s0];
+    float *master = o->state + base, *m = o->state + o->stride + base, *v = o->state + 2 * o->stride + base;
+    const int grid = grid_for(segs.offset[n], 256 * 4, d.sms, 8);
+    status = init ? launch_pdl(adamw_init_kernel, grid, 256, 0, st, segs, master, m, v, h.f16)
+                  : launch_pdl(adamw_kernel, grid, 256, 0, st, segs, master, m, v, h);
+    if (status != QLORA_OK) return status;
+  }
+  return QLORA_OK;
+}
+
+bool finite_nonneg(float x) { return std::isfinite(x) && x >= 0.0f; }
+
+}  // namespace
+
+extern "C" {
+
+int qlora_paged_adamw_placement(size_t free_bytes, size_t state_bytes, size_t reserve_bytes, int current) {
+  if (current == 0) return free_bytes < reserve_bytes ? 1 : 0;
+  return free_bytes >= state_bytes + reserve_bytes ? 0 : 1;
+}
+
+qlora_status qlora_paged_adamw_create(int nseg, const int64_t *counts, qlora_paged_adamw **out) {
+  if (!counts || !out) return QLORA_ERR_NULL;
+  *out = nullptr;
+  if (nseg < 1) return QLORA_ERR_SHAPE;
+  auto *o = new qlora_paged_adamw();
+  o->offset.resize(static_cast<size_t>(nseg) + 1);
+  o->offset[0] = 0;
+  for (int i = 0; i < nseg; ++i) {
+    if (counts[i] < 1) {
+      delete o;
+      return QLORA_ERR_SHAPE;
+    }
+    o->offset[i + 1] = o->offset[i] + counts[i];
+  }
+  o->total = o->offset[nseg];
+  o->stride = (o->total + 63) / 64 * 64;
+  o->bytes = static_cast<size_t>(o->stride) * 3 * sizeof(float);
+  DeviceInfo d;
+  const qlora_status st = device_info(&d);
+  if (st != QLORA_OK) {
+    delete o;
+    return st;
+  }
+  cudaGetDevice(&o->device);
+  int cma = 0;
+  cudaDeviceGetAttribute(&cma, cudaDevAttrConcurrentManagedAccess, o->device);
+  o->hints = cma != 0;
+  void *p = nullptr;
+  if (cudaMallocManaged(&p, o->bytes, cudaMemAttachGlobal) != cudaSuccess) {
+    cudaGetLastError();
+    delete o;
+    return QLORA_ERR_CUDA;
+  }
+  o->state = static_cast<float *>(p);
+  *out = o;
+  return QLORA_OK;
+}
+
+void qlora_paged_adamw_destroy(qlora_paged_adamw *opt) {
+  if (!opt) return;
+  if (opt->state) {
+    cudaDeviceSynchronize();
+    cudaFree(opt->state);
+  }
+  delete opt;
+}
+
+qlora_status qlora_paged_adamw_set_reserve(qlora_paged_adamw *opt, size_t reserve_bytes) {
+  if (!opt) return QLORA_ERR_NULL;
+  opt->reserve = reserve_bytes;
+  return QLORA_OK;
+}
+
+int qlora_paged_adamw_location(const qlora_paged_adamw *opt) { return opt ? opt->where : -1; }
+
+size_t qlora_paged_adamw_state_bytes(const qlora_paged_adamw *opt) { return opt ? opt->bytes : 0; }
+
+qlora_status qlora_paged_adamw_state(const qlora_paged_adamw *opt, float **master, float **m, float **v) {
+  if (!opt || !master || !m || !v) return QLORA_ERR_NULL;
+  *master = opt->state;
+  *m = opt->state + opt->stride;
+  *v = opt->state + 2 * opt->stride;
+  return QLORA_OK;
+}
+
+qlora_status qlora_paged_adamw_init(qlora_paged_adamw *opt, void *const *params, qlora_dtype dtype,
+                                    qlora_stream_t stream) {
+  if (!opt || !params) return QLORA_ERR_NULL;
+  if (dtype != QLORA_BF16 && dtype != QLORA_F16) return QLORA_ERR_RANGE;
+  const size_t nseg = opt->offset.size() - 1;
+  for (size_t i = 0; i < nseg; ++i) {
+    if (!params[i]) return QLORA_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(params[i]) & 1u) return QLORA_ERR_ALIGN;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  qlora_status status = adamw_place(opt, 0, st);
+  if (status != QLORA_OK) return status;
+  AdamwHyper h;
+  std::memset(&h, 0, sizeof h);
+  h.f16 = dtype == QLORA_F16 ? 1 : 0;
+  return adamw_launch(opt, params, nullptr, true, h, st);
+}
+
+qlora_status qlora_paged_adamw_step(qlora_paged_adamw *opt, void *const *params, const void *const *grads,
+                                    qlora_dtype dtype, int64_t t, float lr, float beta1, float beta2, float eps,
+                                    float weight_decay, qlora_stream_t stream) {
+  if (!opt || !params || !grads) return QLORA_ERR_NULL;
+  if (dtype != QLORA_BF16 && dtype != QLORA_F16) return QLORA_ERR_RANGE;
+  if (t < 1 || !finite_nonneg(lr) || !finite_nonneg(beta1) || beta1 >= 1.0f || !finite_nonneg(beta2) ||
+      beta2 >= 1.0f || !(std::isfinite(eps) && eps > 0.0f) || !finite_nonneg(weight_decay))
+    return QLORA_ERR_RANGE;
+  const size_t nseg = opt->offset.size() - 1;
+  for (size_t i = 0; i < nseg; ++i) {
+    if (!params[i] || !grads[i]) return QLORA_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(params[i]) | reinterpret_cast<uintptr_t>(grads[i])) & 1u)
+      return QLORA_ERR_ALIGN;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  size_t free_b = 0, total_b = 0;
+  if (cudaMemGetInfo(&free_b, &total_b) != cudaSuccess) return QLORA_ERR_CUDA;
+  const int to = qlora_paged_adamw_placement(free_b, opt->bytes, opt->reserve, opt->where);
+  qlora_status status = QLORA_OK;
+  if (to != opt->where && (status = adamw_place(opt, to, st)) != QLORA_OK) return status;
+  AdamwHyper h;
+  h.lr = lr;
+  h.b1 = beta1;
+  h.b2 = beta2;
+  h.eps = eps;
+  h.wd = weight_decay;
+  h.bc1 = static_cast<float>(1.0 - std::pow(static_cast<double>(beta1), static_cast<double>(t)));
+  h.bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(beta2), static_cast<double>(t)));
+  h.f16 = dtype == QLORA_F16 ? 1 : 0;
+  if (!(h.bc1 > 0.0f) || !(h.bc2 > 0.0f)) return QLORA_ERR_RANGE;  // beta^t rounds to 1 only for beta = 1
+  return adamw_launch(opt, params, grads, false, h, st);
 }
 
 }  // extern "C"

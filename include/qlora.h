@@ -289,6 +289,71 @@ QLORA_API qlora_status qlora_linear_fwd_noalloc(const uint8_t *packed, const uin
                                                 qlora_bf16 *XA_out, qlora_stream_t stream);
 
 /*
+ * Paged AdamW for the adapters (intvml.com "DL0087 QLoRA: 4-bit Quantized
+ * LoRA", component (5) "Paged Optimizers"; promptingindex.com "QLoRA:
+ * Finetuning 65B Models on a Single GPU", "Double Quantization and Paged
+ * Optimizers"): the optimizer state sits in CUDA unified (managed) memory,
+ * so it can be paged out to host RAM when device memory runs short and
+ * back when it frees up, instead of failing the step.
+ *
+ * State per adapter element: an fp32 master copy of the 16-bit parameter and
+ * the two fp32 moments m, v (12 bytes), in one managed allocation that the
+ * handle owns. The update is AdamW with decoupled weight decay (Loshchilov
+ * and Hutter, ICLR 2019, Algorithm 2) in fp32:
+ *   p <- p (1 - lr wd); m <- b1 m + (1 - b1) g; v <- b2 v + (1 - b2) g^2;
+ *   p <- p - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
+ * and the 16-bit parameter is then p rounded to nearest even.
+ *
+ * Placement: before each step the library reads the device's free memory
+ * (cudaMemGetInfo) and calls qlora_paged_adamw_placement. Paging out sets
+ * the preferred location to the host, lets the device map the pages, and
+ * prefetches them to the host; the step then reads and writes the state
+ * across the host link. Paging in sets the preferred location to the
+ * device and prefetches the pages back. Where the device does not support
+ * concurrent managed access the hints are skipped and the driver migrates
+ * on demand.
+ *
+ * create:  nseg tensors (1 <= nseg), counts[s] >= 1 elements each (host
+ *          array); *out receives the handle. QLORA_ERR_CUDA if the managed
+ *          allocation fails.
+ * init:    params[s]: device 16-bit tensors (host array of nseg pointers);
+ *          master <- params, m = v = 0. Asynchronous on `stream`.
+ * step:    grads[s]: device 16-bit gradients, same shapes; t >= 1 the step
+ *          number; lr >= 0, 0 <= beta1, beta2 < 1, eps > 0, wd >= 0, all
+ *          finite (else QLORA_ERR_RANGE). Writes params[s] and the state.
+ *          Asynchronous on `stream`; the state must not be read by the host
+ *          until the stream is synchronized.
+ * set_reserve: device bytes the placement keeps free for other work
+ *          (default 0).
+ * placement: pure policy, exported for tests: 1 (host) or 0 (device) for a
+ *          state of state_bytes given free device bytes and the reserve;
+ *          `current` is the present location (0 or 1). On the device it
+ *          stays until free < reserve; on the host it comes back once
+ *          free >= state_bytes + reserve.
+ * location: 0 or 1, where the last step placed the state.
+ * state:   the managed pointers of the master copy and the moments (fp32,
+ *          concatenated over the segments in order); host-readable once the
+ *          stream is synchronized. Owned by the handle.
+ * destroy: frees the state (synchronizes the device first); NULL is a no-op.
+ */
+typedef struct qlora_paged_adamw qlora_paged_adamw;
+QLORA_API qlora_status qlora_paged_adamw_create(int nseg, const int64_t *counts, qlora_paged_adamw **out);
+QLORA_API void qlora_paged_adamw_destroy(qlora_paged_adamw *opt);
+QLORA_API qlora_status qlora_paged_adamw_init(qlora_paged_adamw *opt, void *const *params, qlora_dtype dtype,
+                                              qlora_stream_t stream);
+QLORA_API qlora_status qlora_paged_adamw_step(qlora_paged_adamw *opt, void *const *params,
+                                              const void *const *grads, qlora_dtype dtype, int64_t t, float lr,
+                                              float beta1, float beta2, float eps, float weight_decay,
+                                              qlora_stream_t stream);
+QLORA_API qlora_status qlora_paged_adamw_set_reserve(qlora_paged_adamw *opt, size_t reserve_bytes);
+QLORA_API int qlora_paged_adamw_placement(size_t free_bytes, size_t state_bytes, size_t reserve_bytes,
+                                          int current);
+QLORA_API int qlora_paged_adamw_location(const qlora_paged_adamw *opt);
+QLORA_API size_t qlora_paged_adamw_state_bytes(const qlora_paged_adamw *opt);
+QLORA_API qlora_status qlora_paged_adamw_state(const qlora_paged_adamw *opt, float **master, float **m,
+                                               float **v);
+
+/*
  * Measurement instrumentation (no counterpart on the pages).
  *
  * qlora_set_trace_events: when both are non-NULL, the next qlora_linear_fwd
