@@ -452,7 +452,7 @@ def workload_phases(dev, hbm_gbs, tc_tflops, quick=False):
       single_1024          one 1024x1024 linear, M = 16, r = 8: fwd + bwd latency
       llama13b_quant_sweep quantize + double quant, and dequant, over 40 layers x 7 linears
       llama65b_fwd         7 linears: few-token forwards (M = 1, 4, 16) and M = 4096
-      llama33b_block       7 linears, M = 2048: fwd (saving XA) + bwd recomputing XA
+      llama33b_block       7 linears, M = 2048: block fwd + block bwd recomputing XA (and one by one)
     Rates are against the measured peaks and the spec ones (8 TB/s HBM,
     2.25 PFLOP/s dense bf16)."""
     import torch
@@ -593,13 +593,27 @@ def workload_phases(dev, hbm_gbs, tc_tflops, quick=False):
         for lin, pk, q, s2, inp, Y, XA, dX, dA, dB in reversed(state):
             binding.linear_bwd(pk, q, s2, inp["X"], inp["dY"], inp["A"], inp["B"], wl.alpha, lin.N, lin.K, XA=None,
                                dX=dX, dA=dA, dB=dB, workspace=ws)
-    ms = device_ms(block, 3)
+    ms_seq = device_ms(block, 3)
+    # the same work through the block executor (qlora_block_fwd/bwd: one call
+    # per pass, linears over two streams), checkpoint schedule: the forward
+    # saves nothing and the backward recomputes X A
+    lins = [{"packed": pk, "q": q, "scale2": s2, "N": lin.N, "K": lin.K, "X": inp["X"], "A": inp["A"],
+             "B": inp["B"], "Y": Y, "XA": XA, "dY": inp["dY"], "dX": dX, "dA": dA, "dB": dB}
+            for lin, pk, q, s2, inp, Y, XA, dX, dA, dB in state]
+    bws = torch.empty(binding.block_workspace_bytes(lins, M, wl.r), dtype=torch.uint8, device=dev)
+    rev = lins[::-1]
+
+    def block_exec():
+        binding.block_fwd(lins, M, wl.r, wl.alpha, save_xa=False, workspace=bws)
+        binding.block_bwd(rev, M, wl.r, wl.alpha, save_xa=False, workspace=bws)
+    ms = device_ms(block_exec, 3)
     flops = sum(linear_flops(M, lin.N, lin.K, wl.r) + 2 * M * lin.K * wl.r for lin, *_ in state)
-    out["llama33b_block"] = {"what": "7 linears (d=6656, ffn=17920), M=2048, r=64: fwd saving XA, then bwd "
-                                     "recomputing XA and re-dequantizing W",
-                             "ms": round(ms, 4), "GFLOP": round(flops / 1e9, 1),
-                             **frac_tc(flops / (ms * 1e-3) / 1e12)}
-    del state, ws
+    out["llama33b_block"] = {"what": "7 linears (d=6656, ffn=17920), M=2048, r=64: block forward saving nothing, "
+                                     "block backward recomputing XA and re-dequantizing W (qlora_block_fwd/bwd, "
+                                     "2 streams)",
+                             "ms": round(ms, 4), "ms_linears_one_by_one": round(ms_seq, 4),
+                             "GFLOP": round(flops / 1e9, 1), **frac_tc(flops / (ms * 1e-3) / 1e12)}
+    del state, ws, bws, lins, rev
     torch.cuda.empty_cache()
     return out
 

@@ -37,7 +37,18 @@ EXPORTS = ("qlora_status_string", "qlora_abi_version", "qlora_nf4_levels", "qlor
            "qlora_dequant_dt", "qlora_linear_fwd_dt", "qlora_linear_bwd_dt",
            "qlora_paged_adamw_create", "qlora_paged_adamw_destroy", "qlora_paged_adamw_init",
            "qlora_paged_adamw_step", "qlora_paged_adamw_set_reserve", "qlora_paged_adamw_placement",
-           "qlora_paged_adamw_location", "qlora_paged_adamw_state_bytes", "qlora_paged_adamw_state")
+           "qlora_paged_adamw_location", "qlora_paged_adamw_state_bytes", "qlora_paged_adamw_state",
+           "qlora_block_workspace_bytes", "qlora_block_fwd", "qlora_block_bwd")
+
+BLOCK_STREAMS = 2
+
+
+class LinearDesc(ctypes.Structure):
+    """qlora_linear_desc: one linear of a decoder block (device pointers)."""
+    _fields_ = [("packed", ctypes.c_void_p), ("q", ctypes.c_void_p), ("scale2", ctypes.c_void_p),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("X", ctypes.c_void_p), ("A", ctypes.c_void_p),
+                ("B", ctypes.c_void_p), ("Y", ctypes.c_void_p), ("XA", ctypes.c_void_p), ("dY", ctypes.c_void_p),
+                ("dX", ctypes.c_void_p), ("dA", ctypes.c_void_p), ("dB", ctypes.c_void_p)]
 
 # qlora_dtype of the 16-bit tensors of a call
 _DTYPE = {torch.bfloat16: 0, torch.float16: 1}
@@ -107,6 +118,12 @@ def load(path: str | None = None):
         lib.qlora_paged_adamw_state_bytes.restype = SZ
         lib.qlora_paged_adamw_state.argtypes = [P, PP, PP, PP]
         lib.qlora_paged_adamw_state.restype = I32
+        DP = ctypes.POINTER(LinearDesc)
+        lib.qlora_block_workspace_bytes.argtypes = [I32, DP, I64, I32]
+        lib.qlora_block_workspace_bytes.restype = SZ
+        for fn in ("qlora_block_fwd", "qlora_block_bwd"):
+            getattr(lib, fn).argtypes = [I32, DP, P, P, I32, I64, I32, F32, I32, P, SZ, P]
+            getattr(lib, fn).restype = I32
         lib.qlora_device_error.argtypes = [I32]
         lib.qlora_device_error.restype = ctypes.c_uint32
         lib.qlora_set_trace_events.argtypes = [P, P]
@@ -483,3 +500,60 @@ class PagedAdamW:
             self.close()
         except Exception:
             pass
+
+
+_DESC_TENSORS = ("X", "A", "B", "Y", "XA", "dY", "dX", "dA", "dB")
+
+
+def _descs(linears, M: int, r: int, need):
+    """ctypes array of qlora_linear_desc from dicts of tensors; `need` names
+    the tensors the pass reads or writes (checked for type and shape)."""
+    arr = (LinearDesc * len(linears))()
+    dt = None
+    for i, L in enumerate(linears):
+        N, K = int(L["N"]), int(L["K"])
+        shapes = {"X": (M, K), "A": (K, r), "B": (r, N), "Y": (M, N), "XA": (M, r), "dY": (M, N), "dX": (M, K),
+                  "dA": (K, r), "dB": (r, N)}
+        d = arr[i]
+        d.packed, d.q, d.scale2 = (L[k].data_ptr() for k in ("packed", "q", "scale2"))
+        d.N, d.K = N, K
+        for k in _DESC_TENSORS:
+            t = L.get(k)
+            if k in need:
+                if t is None:
+                    raise ValueError(f"linear {i}: {k} is required")
+                dt = dt or _dtype_of(t, k)
+                _req(t, f"linear {i} {k}", dt, shapes[k])
+            setattr(d, k, None if t is None else t.data_ptr())
+    return arr, dt
+
+
+def block_workspace_bytes(linears, M: int, r: int) -> int:
+    arr, _ = _descs(linears, M, r, ())
+    return int(load().qlora_block_workspace_bytes(len(linears), arr, M, r))
+
+
+def _block(fn, linears, M, r, alpha, save_xa, workspace, nf4, t8, need):
+    arr, dt = _descs(linears, M, r, need)
+    need_ws = int(load().qlora_block_workspace_bytes(len(linears), arr, M, r))
+    if workspace is None:
+        workspace = torch.empty(max(need_ws, 256), dtype=torch.uint8, device=linears[0]["X"].device)
+    _req(workspace, "workspace", torch.uint8)
+    tb = _tables(nf4, t8)
+    _check(getattr(load(), fn)(len(linears), arr, tb.nf4, tb.t8, _DTYPE[dt], M, r, float(alpha), 1 if save_xa else 0,
+                               _ptr(workspace), workspace.numel(), _stream()), fn)
+    return workspace
+
+
+def block_fwd(linears, M: int, r: int, alpha: float, save_xa: bool = True, workspace=None, nf4=None, t8=None):
+    """Forward of every linear of a decoder block in one call (qlora_block_fwd):
+    each dict holds packed, q, scale2, N, K, X, A, B, Y and, with save_xa, XA."""
+    need = ("X", "A", "B", "Y") + (("XA",) if save_xa else ())
+    return _block("qlora_block_fwd", linears, M, r, alpha, save_xa, workspace, nf4, t8, need)
+
+
+def block_bwd(linears, M: int, r: int, alpha: float, save_xa: bool = True, workspace=None, nf4=None, t8=None):
+    """Backward of every linear of a decoder block in one call (qlora_block_bwd):
+    each dict also holds dY, dX, dA, dB (and XA when the forward saved it)."""
+    need = ("X", "A", "B", "dY", "dX", "dA", "dB") + (("XA",) if save_xa else ())
+    return _block("qlora_block_bwd", linears, M, r, alpha, save_xa, workspace, nf4, t8, need)

@@ -1311,6 +1311,106 @@ uint32_t qlora_device_error(int clear) {
 
 }  // extern "C"
 
+// ------------------------------------------------ decoder-block chains --
+namespace {
+
+// The library's extra streams and fork/join events of this host thread on
+// one device (created on first use, kept for the thread's life).
+struct BlockStreams {
+  bool init = false;
+  cudaStream_t side[QLORA_BLOCK_STREAMS - 1] = {};
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join[QLORA_BLOCK_STREAMS - 1] = {};
+};
+thread_local BlockStreams t_block[kMaxDevices];
+
+qlora_status block_streams(BlockStreams **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ERR_CUDA;
+  BlockStreams &b = t_block[dev];
+  if (!b.init) {
+    if (cudaEventCreateWithFlags(&b.fork, cudaEventDisableTiming) != cudaSuccess) return QLORA_ERR_CUDA;
+    for (int i = 0; i < QLORA_BLOCK_STREAMS - 1; ++i)
+      if (cudaStreamCreateWithFlags(&b.side[i], cudaStreamNonBlocking) != cudaSuccess ||
+          cudaEventCreateWithFlags(&b.join[i], cudaEventDisableTiming) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    b.init = true;
+  }
+  *out = &b;
+  return QLORA_OK;
+}
+
+size_t block_slice_bytes(int n, const qlora_linear_desc *desc, int64_t M, int r) {
+  size_t m = 0;
+  for (int i = 0; i < n; ++i) m = std::max(m, align256(qlora_workspace_bytes(M, desc[i].N, desc[i].K, r)));
+  return m;
+}
+
+template <class Fn>
+qlora_status run_block(int n, const qlora_linear_desc *desc, int64_t M, int r, void *workspace,
+                       size_t workspace_bytes, cudaStream_t main, Fn &&one) {
+  if (n < 1 || !desc) return n < 1 ? QLORA_ERR_SHAPE : QLORA_ERR_NULL;
+  const size_t slice = block_slice_bytes(n, desc, M, r);
+  if (slice == 0) return QLORA_ERR_SHAPE;
+  const int ns = std::min(n, QLORA_BLOCK_STREAMS);
+  if (!workspace || workspace_bytes < slice * ns) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QLORA_ERR_ALIGN;
+  BlockStreams *b = nullptr;
+  qlora_status st = block_streams(&b);
+  if (st != QLORA_OK) return st;
+  // fork: the side streams start after everything queued on `main`
+  if (cudaEventRecord(b->fork, main) != cudaSuccess) return QLORA_ERR_CUDA;
+  for (int j = 1; j < ns; ++j)
+    if (cudaStreamWaitEvent(b->side[j - 1], b->fork, 0) != cudaSuccess) return QLORA_ERR_CUDA;
+  qlora_status first_err = QLORA_OK;
+  for (int i = 0; i < n && first_err == QLORA_OK; ++i) {
+    const int j = i % ns;
+    cudaStream_t s = j == 0 ? main : b->side[j - 1];
+    first_err = one(desc[i], static_cast<uint8_t *>(workspace) + slice * j, slice, s);
+  }
+  // join: `main` continues after every side stream's work (also on error,
+  // so nothing launched is left outside the caller's stream order)
+  for (int j = 1; j < ns; ++j)
+    if (cudaEventRecord(b->join[j - 1], b->side[j - 1]) != cudaSuccess ||
+        cudaStreamWaitEvent(main, b->join[j - 1], 0) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+  return first_err;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t qlora_block_workspace_bytes(int n, const qlora_linear_desc *desc, int64_t M, int r) {
+  if (n < 1 || !desc) return 0;
+  return block_slice_bytes(n, desc, M, r) * static_cast<size_t>(std::min(n, QLORA_BLOCK_STREAMS));
+}
+
+qlora_status qlora_block_fwd(int n, const qlora_linear_desc *desc, const float nf4[16], const float t8[256],
+                             qlora_dtype dtype, int64_t M, int r, float alpha, int save_xa, void *workspace,
+                             size_t workspace_bytes, qlora_stream_t stream) {
+  if (dtype != QLORA_BF16 && dtype != QLORA_F16) return QLORA_ERR_RANGE;
+  return run_block(n, desc, M, r, workspace, workspace_bytes, static_cast<cudaStream_t>(stream),
+                   [&](const qlora_linear_desc &d, void *ws, size_t wsb, cudaStream_t s) {
+                     return qlora_linear_fwd_dt(d.packed, d.q, d.scale2, nf4, t8, dtype, M, d.N, d.K, d.X, d.A,
+                                                d.B, r, alpha, d.Y, save_xa ? d.XA : nullptr, ws, wsb, s);
+                   });
+}
+
+qlora_status qlora_block_bwd(int n, const qlora_linear_desc *desc, const float nf4[16], const float t8[256],
+                             qlora_dtype dtype, int64_t M, int r, float alpha, int save_xa, void *workspace,
+                             size_t workspace_bytes, qlora_stream_t stream) {
+  if (dtype != QLORA_BF16 && dtype != QLORA_F16) return QLORA_ERR_RANGE;
+  return run_block(n, desc, M, r, workspace, workspace_bytes, static_cast<cudaStream_t>(stream),
+                   [&](const qlora_linear_desc &d, void *ws, size_t wsb, cudaStream_t s) {
+                     return qlora_linear_bwd_dt(d.packed, d.q, d.scale2, nf4, t8, dtype, M, d.N, d.K, d.X, d.dY,
+                                                d.A, d.B, save_xa ? d.XA : nullptr, r, alpha, d.dX, d.dA, d.dB,
+                                                ws, wsb, s);
+                   });
+}
+
+}  // extern "C"
+
 // ------------------------------------------------------- paged AdamW --
 struct qlora_paged_adamw {
   int device = 0;

@@ -289,6 +289,55 @@ QLORA_API qlora_status qlora_linear_fwd_noalloc(const uint8_t *packed, const uin
                                                 qlora_bf16 *XA_out, qlora_stream_t stream);
 
 /*
+ * Decoder-block chaining (promptingindex.com "QLoRA: Finetuning 65B Models on
+ * a Single GPU", "LoRA placement": adapters on every linear of the block;
+ * systemoverflow.com "QLoRA ... at Extreme Scale": gradient checkpointing
+ * trades recomputation for memory). One call runs all linears of a decoder
+ * block (for LLaMA: q, k, v, o, gate, up, down), each a qlora_linear_fwd or
+ * qlora_linear_bwd, spread round-robin over QLORA_BLOCK_STREAMS streams (the
+ * caller's stream and library-owned ones that fork from it and join back
+ * into it with events), so that one linear's low-rank (skinny) kernels and
+ * GEMM tail overlap the next linear's GEMM. The call is asynchronous on
+ * `stream`, ordered after earlier work on it, and everything it launches is
+ * complete, in stream order, before later work on `stream`; it can be
+ * captured into a CUDA graph (after one uncaptured call, which sets up the
+ * library's kernels and streams).
+ *
+ * Recompute schedule (`save_xa`): 1 = the forward writes X A of every linear
+ * to desc.XA and the backward reads it; 0 = the forward saves nothing and
+ * the backward recomputes X A. The base weight is dequantized again in the
+ * backward in both (it is never stored in 16-bit form).
+ *
+ * desc[i]: packed, q, scale2 (the quantized base), N, K, X [M, K], A [K, r],
+ *   B [r, N], Y [M, N] (forward output), XA [M, r] (save_xa = 1), dY
+ *   [M, N], dX [M, K], dA [K, r], dB [r, N] (backward). Pointers a pass does
+ *   not use may be NULL. The linears must not share any output buffer.
+ * workspace: at least qlora_block_workspace_bytes(n, desc, M, r) bytes.
+ * Errors: as the per-linear calls (the first failing linear's status is
+ * returned; linears before it have been launched).
+ */
+#define QLORA_BLOCK_STREAMS 2
+typedef struct {
+  const uint8_t *packed;
+  const uint8_t *q;
+  const float *scale2;
+  int64_t N, K;
+  const void *X, *A, *B;
+  void *Y, *XA;
+  const void *dY;
+  void *dX, *dA, *dB;
+} qlora_linear_desc;
+QLORA_API size_t qlora_block_workspace_bytes(int n, const qlora_linear_desc *desc, int64_t M, int r);
+QLORA_API qlora_status qlora_block_fwd(int n, const qlora_linear_desc *desc, const float nf4[16],
+                                       const float t8[256], qlora_dtype dtype, int64_t M, int r, float alpha,
+                                       int save_xa, void *workspace, size_t workspace_bytes,
+                                       qlora_stream_t stream);
+QLORA_API qlora_status qlora_block_bwd(int n, const qlora_linear_desc *desc, const float nf4[16],
+                                       const float t8[256], qlora_dtype dtype, int64_t M, int r, float alpha,
+                                       int save_xa, void *workspace, size_t workspace_bytes,
+                                       qlora_stream_t stream);
+
+/*
  * Paged AdamW for the adapters (intvml.com "DL0087 QLoRA: 4-bit Quantized
  * LoRA", component (5) "Paged Optimizers"; promptingindex.com "QLoRA:
  * Finetuning 65B Models on a Single GPU", "Double Quantization and Paged
