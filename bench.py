@@ -8,8 +8,8 @@ Workload: the 7B-shaped linear set (q, k, v, o 4096x4096; gate, up
 alpha = 16, W ~ N(0, 0.02) with 0.1 % outliers at +-10 sigma; synthetic
 seeded inputs, generated on the device before timing.
 
-One step = for every linear: qlora_quantize_nf4, qlora_double_quant,
-qlora_dequant, qlora_linear_fwd (saving XA), qlora_linear_bwd, and a
+One step = for every linear: qlora_quantize_dq (quantize and double
+quantization in one pass), qlora_dequant, qlora_linear_fwd (saving XA), qlora_linear_bwd, and a
 few-token qlora_linear_fwd (the first 16 tokens: the memory-bound small-M
 path) — every row of the hot path once. Under torchrun each rank runs its own batch (weak
 scaling, data parallel over tokens) and the adapter gradients dA, dB of
@@ -368,8 +368,10 @@ class LinearState:
 
     def codec_bytes(self):
         n = self.N * self.K
-        return {"quantize": n * 2 + n // 2 + n // 64 * 4,
-                "double_quant": n // 64 * 4 + n // 64 + ((n // 64 + 255) // 256) * 4,
+        ng = (n // 64 + 255) // 256
+        return {"quantize_dq": n * 2 + n // 2 + n // 64 + ng * 4,
+                "quantize": n * 2 + n // 2 + n // 64 * 4,
+                "double_quant": n // 64 * 4 + n // 64 + ng * 4,
                 "dequant": n // 2 + n // 64 + ((n // 64 + 255) // 256) * 4 + n * 2}
 
 
@@ -504,7 +506,7 @@ def workload_phases(dev, hbm_gbs, tc_tflops, quick=False):
                      "s2": torch.empty((n // 64 + 255) // 256, dtype=torch.float32, device=dev),
                      "Wq": torch.empty((lin.N, lin.K), dtype=torch.bfloat16, device=dev)})
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 2x L2: written between timed calls
-    t_q = t_dq = t_d = 0.0
+    t_q = t_dq = t_d = t_qdq = 0.0
     params = 0
     for layer in range(layers):
         for li, b in enumerate(bufs):
@@ -513,6 +515,9 @@ def workload_phases(dev, hbm_gbs, tc_tflops, quick=False):
         t_q += device_ms(lambda: [binding.quantize_nf4(b["W"], packed=b["pk"], absmax=b["am"]) for b in bufs], 1, 0)
         flush.zero_()
         t_dq += device_ms(lambda: [binding.double_quant(b["am"], q=b["q"], scale2=b["s2"]) for b in bufs], 1, 0)
+        flush.zero_()
+        t_qdq += device_ms(lambda: [binding.quantize_dq(b["W"], packed=b["pk"], q=b["q"], scale2=b["s2"])
+                                    for b in bufs], 1, 0)
         flush.zero_()
         t_d += device_ms(lambda: [binding.dequant(b["pk"], b["q"], b["s2"], b["N"], b["K"], out=b["Wq"])
                                   for b in bufs], 1, 0)
@@ -528,6 +533,9 @@ def workload_phases(dev, hbm_gbs, tc_tflops, quick=False):
         "double_quant": {"ms": round(t_dq, 3), **frac_hbm((dq_in + dq_out) / (t_dq * 1e-3) / 1e9)},
         "quantize_plus_double_quant": {"ms": round(t_q + t_dq, 3),
                                        **frac_hbm((q_in + q_out + dq_in + dq_out) / ((t_q + t_dq) * 1e-3) / 1e9)},
+        "quantize_dq_one_pass": {"ms": round(t_qdq, 3), "GB_in": round(q_in / 1e9, 3),
+                                 "GB_out": round((n // 2 + n // 64 + n // 16384 * 4) / 1e9, 3),
+                                 **frac_hbm((q_in + n // 2 + n // 64 + n // 16384 * 4) / (t_qdq * 1e-3) / 1e9)},
         "dequant": {"ms": round(t_d, 3), "GB_in": round(d_in / 1e9, 3), "GB_out": round(d_out / 1e9, 3),
                     **frac_hbm((d_in + d_out) / (t_d * 1e-3) / 1e9)}}
     del bufs, flush
@@ -648,7 +656,7 @@ def run_native(args, rank, world, local_rank):
 
     # per step, per linear: events around the codec calls and the fused GEMMs
     def make_events():
-        return [{k: (ev(), ev()) for k in ("quantize", "double_quant", "dequant", "fwd_gemm", "bwd_gemm",
+        return [{k: (ev(), ev()) for k in ("quantize_dq", "dequant", "fwd_gemm", "bwd_gemm",
                                             "fwd_call", "bwd_call", "smallm_fwd")}
                 for _ in range(nl)]
 
@@ -658,8 +666,7 @@ def run_native(args, rank, world, local_rank):
         the library on its stream (headline pass)."""
         if tr is not None and e is None:
             binding.set_trace_events(*tr[0])
-            binding.quantize_nf4(L.W, packed=L.packed, absmax=L.absmax)
-            binding.double_quant(L.absmax, q=L.q, scale2=L.scale2)
+            binding.quantize_dq(L.W, packed=L.packed, q=L.q, scale2=L.scale2)
             binding.dequant(L.packed, L.q, L.scale2, L.N, L.K, out=L.Wq)
             binding.linear_fwd(L.packed, L.q, L.scale2, L.X, L.A, L.B, L.alpha, L.N, L.K, Y=L.Y,
                                XA_out=L.XA, workspace=ws)
@@ -670,11 +677,9 @@ def run_native(args, rank, world, local_rank):
             binding.linear_fwd(L.packed, L.q, L.scale2, L.Xs, L.A, L.B, L.alpha, L.N, L.K, Y=L.Ys,
                                XA_out=L.XAs, workspace=ws)
             return
-        if e: e["quantize"][0].record()
-        binding.quantize_nf4(L.W, packed=L.packed, absmax=L.absmax)
-        if e: e["quantize"][1].record(); e["double_quant"][0].record()
-        binding.double_quant(L.absmax, q=L.q, scale2=L.scale2)
-        if e: e["double_quant"][1].record(); e["dequant"][0].record()
+        if e: e["quantize_dq"][0].record()
+        binding.quantize_dq(L.W, packed=L.packed, q=L.q, scale2=L.scale2)
+        if e: e["quantize_dq"][1].record(); e["dequant"][0].record()
         binding.dequant(L.packed, L.q, L.scale2, L.N, L.K, out=L.Wq)
         if e: e["dequant"][1].record(); binding.set_trace_events(*e["fwd_gemm"]); e["fwd_call"][0].record()
         binding.linear_fwd(L.packed, L.q, L.scale2, L.X, L.A, L.B, L.alpha, L.N, L.K, Y=L.Y,
@@ -740,6 +745,7 @@ def run_native(args, rank, world, local_rank):
     # in a row, one event pair, queued the same way): their device throughput
     # without the per-call event gaps of the breakdown pass
     codec_calls = {
+        "quantize_dq": lambda L: binding.quantize_dq(L.W, packed=L.packed, q=L.q, scale2=L.scale2),
         "quantize": lambda L: binding.quantize_nf4(L.W, packed=L.packed, absmax=L.absmax),
         "double_quant": lambda L: binding.double_quant(L.absmax, q=L.q, scale2=L.scale2),
         "dequant": lambda L: binding.dequant(L.packed, L.q, L.scale2, L.N, L.K, out=L.Wq),
@@ -768,13 +774,14 @@ def run_native(args, rank, world, local_rank):
     value = step_flops * world / (ms * 1e-3) / 1e12
 
     # per-phase device times (mean over the timed steps)
-    phase = {k: [] for k in ("quantize", "double_quant", "dequant", "fwd_gemm", "bwd_gemm", "fwd_call",
+    phase = {k: [] for k in ("quantize_dq", "dequant", "fwd_gemm", "bwd_gemm", "fwd_call",
                              "bwd_call", "smallm_fwd")}
     for evs in evs_steps:
         for k in phase:
             phase[k].append(sum(evs[i][k][0].elapsed_time(evs[i][k][1]) for i in range(nl)))
     phase_ms = {k: sum(v) / len(v) for k, v in phase.items()}
-    codec_bytes = {k: sum(L.codec_bytes()[k] for L in layers) for k in ("quantize", "double_quant", "dequant")}
+    codec_bytes = {k: sum(L.codec_bytes()[k] for L in layers)
+                   for k in ("quantize_dq", "quantize", "double_quant", "dequant")}
     gemm_flops = {"fwd_gemm": sum(2 * M * L.N * L.K + 2 * M * L.r * L.N for L in layers),
                   "bwd_gemm": sum(2 * M * L.N * L.K + 2 * M * L.r * L.K for L in layers)}
     pk, pk_kind = peaks()
@@ -790,14 +797,17 @@ def run_native(args, rank, world, local_rank):
     if clocks.get("sm_mhz") and clocks.get("sm_max_mhz"):
         clock_ratio = min(1.0, clocks["sm_mhz"] / clocks["sm_max_mhz"])
     phases = {}
-    for k in ("quantize", "double_quant", "dequant"):
-        gbs = codec_bytes[k] / (phase_ms[k] * 1e-3) / 1e9
+    for k in ("quantize_dq", "quantize", "double_quant", "dequant"):
         gbs_run = codec_bytes[k] / (codec_run_ms[k] * 1e-3) / 1e9
-        phases[k] = {"ms": round(phase_ms[k], 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
-                     "frac_8tbs": round(gbs / SPEC_HBM_GBS, 3),
-                     "back_to_back": {"ms": round(codec_run_ms[k], 4), "GB/s": round(gbs_run, 1),
+        phases[k] = {"back_to_back": {"ms": round(codec_run_ms[k], 4), "GB/s": round(gbs_run, 1),
                                       "frac_hbm": round(gbs_run / hbm, 3),
                                       "frac_8tbs": round(gbs_run / SPEC_HBM_GBS, 3)}}
+        if k in phase_ms:  # in the step (per-call events)
+            gbs = codec_bytes[k] / (phase_ms[k] * 1e-3) / 1e9
+            phases[k].update({"ms": round(phase_ms[k], 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
+                              "frac_8tbs": round(gbs / SPEC_HBM_GBS, 3)})
+        else:
+            phases[k]["note"] = "not in the step (the step runs the one-pass quantize_dq); back to back only"
     for k in ("fwd_gemm", "bwd_gemm"):
         tf = gemm_flops[k] / (phase_ms[k] * 1e-3) / 1e12
         phases[k] = {"ms": round(phase_ms[k], 4), "TFLOP/s": round(tf, 1), "frac_tensor": round(tf / tc, 3),
@@ -917,7 +927,7 @@ def run_native(args, rank, world, local_rank):
                            "M": M, "r": wl.r, "alpha": wl.alpha, "per_rank_tokens": M,
                            "parallelism": f"dp{world}",
                            "l2": "inputs larger than L2 (405 MB of bf16 weights + 320 MB of activations per step)",
-                           "step": "per linear: quantize_nf4, double_quant, dequant, linear_fwd, linear_bwd, "
+                           "step": "per linear: quantize_dq (one pass), dequant, linear_fwd, linear_bwd, "
                                    f"linear_fwd on the first {SMALL_M} tokens"},
                 "phases": phases, "roofline": roofline, "gpu_launches": launches,
                 "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,

@@ -38,7 +38,7 @@ EXPORTS = ("qlora_status_string", "qlora_abi_version", "qlora_nf4_levels", "qlor
            "qlora_paged_adamw_create", "qlora_paged_adamw_destroy", "qlora_paged_adamw_init",
            "qlora_paged_adamw_step", "qlora_paged_adamw_set_reserve", "qlora_paged_adamw_placement",
            "qlora_paged_adamw_location", "qlora_paged_adamw_state_bytes", "qlora_paged_adamw_state",
-           "qlora_block_workspace_bytes", "qlora_block_fwd", "qlora_block_bwd")
+           "qlora_block_workspace_bytes", "qlora_block_fwd", "qlora_block_bwd", "qlora_quantize_dq")
 
 BLOCK_STREAMS = 2
 
@@ -86,6 +86,8 @@ def load(path: str | None = None):
         lib.qlora_workspace_bytes.restype = SZ
         lib.qlora_quantize_nf4.argtypes = [P, I64, I64, P, P, P, P]
         lib.qlora_double_quant.argtypes = [P, I64, P, P, P, P]
+        lib.qlora_quantize_dq.argtypes = [P, I64, I64, P, P, P, P, P, P, P]
+        lib.qlora_quantize_dq.restype = I32
         lib.qlora_dequant.argtypes = [P, P, P, I64, I64, P, P, P, P]
         lib.qlora_linear_fwd.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, P, I32, F32, P, P, P, SZ, P]
         lib.qlora_linear_fwd_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, P, I32, F32, P, P, P]
@@ -283,6 +285,31 @@ def quantize_nf4(W: torch.Tensor, nf4=None, packed=None, absmax=None):
     _check(load().qlora_quantize_nf4(_ptr(W), N, K, tb.nf4, _ptr(packed), _ptr(absmax), _stream()),
            "qlora_quantize_nf4")
     return packed, absmax
+
+
+def quantize_dq(W: torch.Tensor, nf4=None, t8=None, packed=None, q=None, scale2=None, absmax=None):
+    """W bf16 [N, K] -> (packed uint8 [N*K/2], q uint8 [nb], scale2 fp32
+    [ceil(nb/256)]) in one pass (qlora_quantize_dq); the fp32 block
+    constants are written to `absmax` only when it is given."""
+    N, K = W.shape
+    _req(W, "W", torch.bfloat16)
+    nb = N * K // BLOCK
+    ng = (nb + DQ_BLOCK - 1) // DQ_BLOCK
+    if packed is None:
+        packed = torch.empty(N * K // 2, dtype=torch.uint8, device=W.device)
+    if q is None:
+        q = torch.empty(nb, dtype=torch.uint8, device=W.device)
+    if scale2 is None:
+        scale2 = torch.empty(ng, dtype=torch.float32, device=W.device)
+    _req(packed, "packed", torch.uint8, (N * K // 2,))
+    _req(q, "q", torch.uint8, (nb,))
+    _req(scale2, "scale2", torch.float32, (ng,))
+    if absmax is not None:
+        _req(absmax, "absmax", torch.float32, (nb,))
+    tb = _tables(nf4, t8)
+    _check(load().qlora_quantize_dq(_ptr(W), N, K, tb.nf4, tb.t8, _ptr(packed), _ptr(q), _ptr(scale2), _ptr(absmax),
+                                    _stream()), "qlora_quantize_dq")
+    return packed, q, scale2
 
 
 def double_quant(absmax: torch.Tensor, t8=None, q=None, scale2=None):

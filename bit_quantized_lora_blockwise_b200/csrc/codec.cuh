@@ -320,6 +320,138 @@ __global__ void __launch_bounds__(256) double_quant_kernel(const float *__restri
 }
 
 // ------------------------------------------------------------------------
+// Quantize fused with the double quantization: one CTA owns whole groups of
+// 256 blocks (16384 weights, a second-level group), so the block constants
+// never leave the chip. Per group: the 256 threads load 4 units of 16
+// weights each (the next group's loads are issued before this one is
+// encoded), find every block's absmax across its 4 lanes, encode and store
+// the NF4 codes exactly as quantize_nf4_kernel does, and park the absmax in
+// shared memory; then thread i encodes constant i of the group as
+// double_quant_kernel does (S = the group's max, q = the 8-bit code of
+// RN(c / S)) and the CTA writes q and S (and the fp32 absmax only when the
+// caller asks for it). Bytes: 2 read + 0.5 + 1/64 + 4/16384 written per
+// weight.
+template <bool BUCKET>
+__device__ __forceinline__ uint32_t dq_code(float c, float s, float r, bool fast, const float2 *s_bk,
+                                            const float *s_mid) {
+  if constexpr (BUCKET) {
+    const float x = (s == 0.0f) ? 0.0f : (fast ? div_by_recip(c, s, r) : __fdiv_rn(c, s));
+    const float y = __fmaf_rn(x, 256.0f, kBucketMagic);
+    const uint32_t j = min(__float_as_uint(y) - __float_as_uint(kBucketMagic), 257u);
+    const float2 e = s_bk[j];
+    return __float_as_uint(e.y) + (x > e.x ? 1u : 0u);
+  } else {
+    const float x = (s == 0.0f) ? 0.0f : __fdiv_rn(c, s);
+    uint32_t k = 0;
+#pragma unroll
+    for (uint32_t step = 128; step > 0; step >>= 1)
+      if (x > s_mid[k + step - 1]) k += step;
+    return k;
+  }
+}
+
+template <bool BUCKET, bool V8, bool DQBUCKET>
+__global__ void __launch_bounds__(256) quantize_dq_kernel(const uint4 *__restrict__ W, int64_t nblocks,
+                                                          uint32_t *__restrict__ packed, uint8_t *__restrict__ q,
+                                                          float *__restrict__ scale2, float *__restrict__ absmax,
+                                                          const CodecTables tabs, const BucketTable bt,
+                                                          const DqBucketTable dbt) {
+  __shared__ float s_mid[16];
+  __shared__ float2 s_bk[64];
+  __shared__ float s_mid8[DQBUCKET ? 1 : 256];
+  __shared__ float2 s_bk8[DQBUCKET ? 258 : 1];
+  __shared__ float s_c[2][256];  // the group's constants (two buffers: no barrier between groups)
+  __shared__ float s_wmax[2][8];
+  const int tid = threadIdx.x;
+  if (tid < 15) s_mid[tid] = __fmul_rn(__fadd_rn(tabs.nf4[tid], tabs.nf4[tid + 1]), 0.5f);
+  if (tid < 64)
+    s_bk[tid] = tid < 33 ? make_float2(bt.thr[tid], __uint_as_float(bt.cand[tid])) : make_float2(2.0f, 0.0f);
+  if constexpr (DQBUCKET) {
+    for (int i = tid; i < 258; i += blockDim.x) s_bk8[i] = make_float2(dbt.thr[i], __uint_as_float(dbt.cand[i]));
+  } else {
+    if (tid < 255) s_mid8[tid] = __fmul_rn(__fadd_rn(tabs.t8[tid], tabs.t8[tid + 1]), 0.5f);
+  }
+  __syncthreads();
+  grid_dep_wait();
+  grid_dep_launch();
+  const float mid7 = s_mid[7];
+  const int64_t nunits = nblocks * 4;     // 32-byte units of 16 weights
+  const int64_t ng = (nblocks + 255) / 256;
+  constexpr int U = 4;                    // units per thread per group: 256 threads x 4 = 1024 units = 256 blocks
+  uint32_t vn[U][8];
+  auto load = [&](int64_t g) {
+#pragma unroll
+    for (int h = 0; h < U; ++h) {
+      const int64_t t = g * 1024 + h * 256 + tid;
+      if (t < nunits) {
+        if (V8) {
+          ld_stream_32B(W + 2 * t, vn[h]);
+        } else {
+          const uint4 lo = __ldg(W + 2 * t), hi = __ldg(W + 2 * t + 1);
+          vn[h][0] = lo.x; vn[h][1] = lo.y; vn[h][2] = lo.z; vn[h][3] = lo.w;
+          vn[h][4] = hi.x; vn[h][5] = hi.y; vn[h][6] = hi.z; vn[h][7] = hi.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) vn[h][i] = 0u;
+      }
+    }
+  };
+  int64_t g = blockIdx.x;
+  if (g < ng) load(g);
+  for (int buf = 0; g < ng; g += gridDim.x, buf ^= 1) {
+    uint32_t v[U][8];
+#pragma unroll
+    for (int h = 0; h < U; ++h)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[h][i] = vn[h][i];
+    if (g + gridDim.x < ng) load(g + gridDim.x);
+#pragma unroll
+    for (int h = 0; h < U; ++h) {
+      const int64_t t = g * 1024 + h * 256 + tid;
+      float f0[8], f1[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        f0[2 * i] = __uint_as_float(v[h][i] << 16);
+        f0[2 * i + 1] = __uint_as_float(v[h][i] & 0xFFFF0000u);
+        f1[2 * i] = __uint_as_float(v[h][4 + i] << 16);
+        f1[2 * i + 1] = __uint_as_float(v[h][4 + i] & 0xFFFF0000u);
+      }
+      float m = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fmaxf(fabsf(f0[i]), fabsf(f1[i])));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+      const uint32_t w0 = encode8<BUCKET>(f0, m, s_mid, mid7, s_bk);
+      const uint32_t w1 = encode8<BUCKET>(f1, m, s_mid, mid7, s_bk);
+      if (t < nunits) *reinterpret_cast<uint2 *>(packed + 2 * t) = make_uint2(w0, w1);
+      // block (h * 256 + tid) / 4 of the group; zeros past the last block
+      if ((tid & 3) == 0) s_c[buf][(h * 256 + tid) >> 2] = t < nunits ? m : 0.0f;
+    }
+    __syncthreads();
+    // second level: constant tid of the group
+    const int64_t b = g * 256 + tid;
+    const float c = s_c[buf][tid];
+    float s = c;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s = fmaxf(s, __shfl_xor_sync(0xFFFFFFFFu, s, o));
+    if ((tid & 31) == 0) s_wmax[buf][tid >> 5] = s;
+    __syncthreads();
+    s = s_wmax[buf][0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) s = fmaxf(s, s_wmax[buf][w]);
+    const bool fast = s >= 0x1p-125f && s <= 0x1p125f;
+    const float r = (DQBUCKET && fast) ? __frcp_rn(s) : 0.0f;
+    const uint32_t code = dq_code<DQBUCKET>(c, s, r, fast, s_bk8, s_mid8);
+    if (b < nblocks) {
+      q[b] = static_cast<uint8_t>(code);
+      if (absmax != nullptr) absmax[b] = c;
+    }
+    if (tid == 0) scale2[g] = s;
+  }
+}
+
+// ------------------------------------------------------------------------
 // NF4 decode of one block: the 16 products bf16(L_i * c') are formed once
 // (fp32 multiply, RNE to bf16) and split into four 8-byte planes (low and
 // high bytes of entries 0-7 and 8-15); each 4-bit code then picks its two

@@ -180,6 +180,21 @@ bool build_dq_buckets(const float *t8, DqBucketTable *bt) {
   return true;
 }
 
+// The 8-bit bucket table of t8 (rebuilt only when t8 differs from this
+// thread's last one); false when t8 needs the binary search instead.
+bool dq_buckets(const float *t8, const DqBucketTable **out) {
+  thread_local float last_t8[256];
+  thread_local DqBucketTable bt;
+  thread_local bool have_last = false, bucketed = false;
+  if (!have_last || std::memcmp(last_t8, t8, sizeof last_t8) != 0) {
+    std::memcpy(last_t8, t8, sizeof last_t8);
+    bucketed = build_dq_buckets(t8, &bt);
+    have_last = true;
+  }
+  *out = &bt;
+  return bucketed;
+}
+
 // Every kernel is launched with programmatic stream serialization: it may
 // start (prologue only) while the previous kernel in the stream finishes,
 // and waits for it (griddepcontrol.wait) before touching its outputs.
@@ -968,6 +983,38 @@ qlora_status qlora_quantize_nf4(const qlora_bf16 *W, int64_t N, int64_t K, const
                     reinterpret_cast<uint32_t *>(packed), absmax, make_tables(nf4, nullptr), bt);
 }
 
+qlora_status qlora_quantize_dq(const qlora_bf16 *W, int64_t N, int64_t K, const float nf4[16], const float t8[256],
+                               uint8_t *packed, uint8_t *q, float *scale2, float *absmax, qlora_stream_t stream) {
+  if (!W || !nf4 || !t8 || !packed || !q || !scale2) return QLORA_ERR_NULL;
+  if (N < 1 || K < 64 || K % 64) return QLORA_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(q) || !aligned16(scale2) || (absmax && !aligned16(absmax)))
+    return QLORA_ERR_ALIGN;
+  qlora_status st = check_tables(nf4, t8);
+  if (st != QLORA_OK) return st;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != QLORA_OK) return st;
+  const int64_t nblocks = N * (K / 64);
+  BucketTable bt;
+  const bool bucketed = build_buckets(nf4, &bt);
+  const DqBucketTable *dbt = nullptr;
+  const bool dq_bucketed = dq_buckets(t8, &dbt);
+  const bool v8 = (reinterpret_cast<uintptr_t>(W) & 31u) == 0;
+  using KFn = void (*)(const uint4 *, int64_t, uint32_t *, uint8_t *, float *, float *, const CodecTables,
+                       const BucketTable, const DqBucketTable);
+  static const KFn table[8] = {
+      quantize_dq_kernel<false, false, false>, quantize_dq_kernel<false, false, true>,
+      quantize_dq_kernel<false, true, false>,  quantize_dq_kernel<false, true, true>,
+      quantize_dq_kernel<true, false, false>,  quantize_dq_kernel<true, false, true>,
+      quantize_dq_kernel<true, true, false>,   quantize_dq_kernel<true, true, true>};
+  const KFn kernel = table[(bucketed ? 4 : 0) + (v8 ? 2 : 0) + (dq_bucketed ? 1 : 0)];
+  // one group (256 blocks) per CTA pass, one resident wave
+  const int64_t ng = cdiv(nblocks, 256);
+  const int grid = grid_for(ng, 1, d.sms, resident_per_sm<quantize_dq_kernel<true, true, true>>(256));
+  return launch_pdl(kernel, grid, 256, 0, static_cast<cudaStream_t>(stream), reinterpret_cast<const uint4 *>(W),
+                    nblocks, reinterpret_cast<uint32_t *>(packed), q, scale2, absmax, make_tables(nf4, t8), bt,
+                    *dbt);
+}
+
 qlora_status qlora_double_quant(const float *absmax, int64_t nb, const float t8[256], uint8_t *q, float *scale2,
                                 qlora_stream_t stream) {
   if (!absmax || !t8 || !q || !scale2) return QLORA_ERR_NULL;
@@ -977,16 +1024,10 @@ qlora_status qlora_double_quant(const float *absmax, int64_t nb, const float t8[
   if (st != QLORA_OK) return st;
   DeviceInfo d;
   if ((st = device_info(&d)) != QLORA_OK) return st;
-  // the table is rebuilt only when t8 differs from this thread's last one
+  const DqBucketTable *btp = nullptr;
+  const bool bucketed = dq_buckets(t8, &btp);
+  const DqBucketTable &bt = *btp;
   static DqBucketTable no_buckets;
-  thread_local float last_t8[256];
-  thread_local DqBucketTable bt;
-  thread_local bool have_last = false, bucketed = false;
-  if (!have_last || std::memcmp(last_t8, t8, sizeof last_t8) != 0) {
-    std::memcpy(last_t8, t8, sizeof last_t8);
-    bucketed = build_dq_buckets(t8, &bt);
-    have_last = true;
-  }
   // one group per warp; at most two CTAs per SM (each fills its own table),
   // warps with more groups load the next one ahead
   const int64_t ng = cdiv(nb, 256);

@@ -148,6 +148,18 @@ QLORA_API qlora_status qlora_double_quant(const float *absmax, int64_t nb, const
                                 uint8_t *q, float *scale2, qlora_stream_t stream);
 
 /*
+ * Quantize and double-quantize in one pass (DL0087 components (2) and (3)):
+ * the same packed codes, q and scale2 as qlora_quantize_nf4 followed by
+ * qlora_double_quant, bit for bit, from one kernel in which a CTA owns whole
+ * second-level groups (256 blocks), so the fp32 block constants stay on
+ * chip. absmax: device fp32 [N*K/64] receiving the block constants, or NULL
+ * (not written). Same requirements and errors as the two calls.
+ */
+QLORA_API qlora_status qlora_quantize_dq(const qlora_bf16 *W, int64_t N, int64_t K, const float nf4[16],
+                              const float t8[256], uint8_t *packed, uint8_t *q, float *scale2,
+                              float *absmax, qlora_stream_t stream);
+
+/*
  * Dequantization to bf16 (DL0087, opening paragraph and Figure 1):
  *   W_out[e] = bf16_rne( nf4[code_e] * c'_b ),  c'_b = t8[q_b] * scale2[b/256],
  * both products in fp32. Bit-identical to the bf16 weight the two linear
