@@ -350,8 +350,8 @@ __device__ __forceinline__ uint32_t dq_code(float c, float s, float r, bool fast
   }
 }
 
-template <bool BUCKET, bool V8, bool DQBUCKET>
-__global__ void __launch_bounds__(256) quantize_dq_kernel(const uint4 *__restrict__ W, int64_t nblocks,
+template <bool BUCKET, bool V8, bool DQBUCKET, int QT = 256>
+__global__ void __launch_bounds__(QT) quantize_dq_kernel(const uint4 *__restrict__ W, int64_t nblocks,
                                                           uint32_t *__restrict__ packed, uint8_t *__restrict__ q,
                                                           float *__restrict__ scale2, float *__restrict__ absmax,
                                                           const CodecTables tabs, const BucketTable bt,
@@ -362,6 +362,7 @@ __global__ void __launch_bounds__(256) quantize_dq_kernel(const uint4 *__restric
   __shared__ float2 s_bk8[DQBUCKET ? 258 : 1];
   __shared__ float s_c[2][256];  // the group's constants (two buffers: no barrier between groups)
   __shared__ float s_wmax[2][8];
+  static_assert(QT == 256 || QT == 512 || QT == 1024, "threads per CTA");
   const int tid = threadIdx.x;
   if (tid < 15) s_mid[tid] = __fmul_rn(__fadd_rn(tabs.nf4[tid], tabs.nf4[tid + 1]), 0.5f);
   if (tid < 64)
@@ -377,12 +378,12 @@ __global__ void __launch_bounds__(256) quantize_dq_kernel(const uint4 *__restric
   const float mid7 = s_mid[7];
   const int64_t nunits = nblocks * 4;     // 32-byte units of 16 weights
   const int64_t ng = (nblocks + 255) / 256;
-  constexpr int U = 4;                    // units per thread per group: 256 threads x 4 = 1024 units = 256 blocks
+  constexpr int U = 1024 / QT;             // units per thread per group: QT threads x U = 1024 units = 256 blocks
   uint32_t vn[U][8];
   auto load = [&](int64_t g) {
 #pragma unroll
     for (int h = 0; h < U; ++h) {
-      const int64_t t = g * 1024 + h * 256 + tid;
+      const int64_t t = g * 1024 + h * QT + tid;
       if (t < nunits) {
         if (V8) {
           ld_stream_32B(W + 2 * t, vn[h]);
@@ -408,7 +409,7 @@ __global__ void __launch_bounds__(256) quantize_dq_kernel(const uint4 *__restric
     if (g + gridDim.x < ng) load(g + gridDim.x);
 #pragma unroll
     for (int h = 0; h < U; ++h) {
-      const int64_t t = g * 1024 + h * 256 + tid;
+      const int64_t t = g * 1024 + h * QT + tid;
       float f0[8], f1[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -426,28 +427,32 @@ __global__ void __launch_bounds__(256) quantize_dq_kernel(const uint4 *__restric
       const uint32_t w1 = encode8<BUCKET>(f1, m, s_mid, mid7, s_bk);
       if (t < nunits) *reinterpret_cast<uint2 *>(packed + 2 * t) = make_uint2(w0, w1);
       // block (h * 256 + tid) / 4 of the group; zeros past the last block
-      if ((tid & 3) == 0) s_c[buf][(h * 256 + tid) >> 2] = t < nunits ? m : 0.0f;
+      if ((tid & 3) == 0) s_c[buf][(h * QT + tid) >> 2] = t < nunits ? m : 0.0f;
     }
     __syncthreads();
-    // second level: constant tid of the group
+    // second level: constant tid of the group (the first 256 threads)
     const int64_t b = g * 256 + tid;
-    const float c = s_c[buf][tid];
+    const float c = tid < 256 ? s_c[buf][tid] : 0.0f;
     float s = c;
+    if (tid < 256) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s = fmaxf(s, __shfl_xor_sync(0xFFFFFFFFu, s, o));
-    if ((tid & 31) == 0) s_wmax[buf][tid >> 5] = s;
-    __syncthreads();
-    s = s_wmax[buf][0];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) s = fmaxf(s, s_wmax[buf][w]);
-    const bool fast = s >= 0x1p-125f && s <= 0x1p125f;
-    const float r = (DQBUCKET && fast) ? __frcp_rn(s) : 0.0f;
-    const uint32_t code = dq_code<DQBUCKET>(c, s, r, fast, s_bk8, s_mid8);
-    if (b < nblocks) {
-      q[b] = static_cast<uint8_t>(code);
-      if (absmax != nullptr) absmax[b] = c;
+      for (int o = 16; o > 0; o >>= 1) s = fmaxf(s, __shfl_xor_sync(0xFFFFFFFFu, s, o));
+      if ((tid & 31) == 0) s_wmax[buf][tid >> 5] = s;
     }
-    if (tid == 0) scale2[g] = s;
+    __syncthreads();
+    if (tid < 256) {
+      s = s_wmax[buf][0];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) s = fmaxf(s, s_wmax[buf][w]);
+      const bool fast = s >= 0x1p-125f && s <= 0x1p125f;
+      const float r = (DQBUCKET && fast) ? __frcp_rn(s) : 0.0f;
+      const uint32_t code = dq_code<DQBUCKET>(c, s, r, fast, s_bk8, s_mid8);
+      if (b < nblocks) {
+        q[b] = static_cast<uint8_t>(code);
+        if (absmax != nullptr) absmax[b] = c;
+      }
+      if (tid == 0) scale2[g] = s;
+    }
   }
 }
 

@@ -338,7 +338,8 @@ qlora_status launch_gemm(const GemmArgs &args, int sms, int pair_slots, cudaStre
   if (attr_err != cudaSuccess) return QLORA_ERR_CUDA;
   const int row_tiles = (args.rows + C::TILE_ROWS - 1) / C::TILE_ROWS;
   const int col_tiles = (args.cols + C::TILE_COLS - 1) / C::TILE_COLS;
-  const int tiles = args.full_tiles + (row_tiles * col_tiles - args.full_tiles) * args.tail_splits;
+  const int tiles = args.full_tiles + (row_tiles * col_tiles - args.full_tiles) *
+                                          (args.tail_subtiles > 1 ? args.tail_subtiles : args.tail_splits);
   if constexpr (!C::PAIR) {
     const int grid = tiles < sms ? tiles : sms;
     return launch_pdl(qgemm_kernel<C>, grid, C::THREADS, C::SMEM_BYTES, stream, args);
@@ -983,6 +984,10 @@ qlora_status qlora_quantize_nf4(const qlora_bf16 *W, int64_t N, int64_t K, const
                     reinterpret_cast<uint32_t *>(packed), absmax, make_tables(nf4, nullptr), bt);
 }
 
+// threads per CTA of the one-pass quantize (each takes 1024 / this many
+// 16-weight units of a group)
+constexpr int kQuantizeDqThreads = 512;
+
 qlora_status qlora_quantize_dq(const qlora_bf16 *W, int64_t N, int64_t K, const float nf4[16], const float t8[256],
                                uint8_t *packed, uint8_t *q, float *scale2, float *absmax, qlora_stream_t stream) {
   if (!W || !nf4 || !t8 || !packed || !q || !scale2) return QLORA_ERR_NULL;
@@ -1001,16 +1006,17 @@ qlora_status qlora_quantize_dq(const qlora_bf16 *W, int64_t N, int64_t K, const 
   const bool v8 = (reinterpret_cast<uintptr_t>(W) & 31u) == 0;
   using KFn = void (*)(const uint4 *, int64_t, uint32_t *, uint8_t *, float *, float *, const CodecTables,
                        const BucketTable, const DqBucketTable);
+  constexpr int QT = kQuantizeDqThreads;
   static const KFn table[8] = {
-      quantize_dq_kernel<false, false, false>, quantize_dq_kernel<false, false, true>,
-      quantize_dq_kernel<false, true, false>,  quantize_dq_kernel<false, true, true>,
-      quantize_dq_kernel<true, false, false>,  quantize_dq_kernel<true, false, true>,
-      quantize_dq_kernel<true, true, false>,   quantize_dq_kernel<true, true, true>};
+      quantize_dq_kernel<false, false, false, QT>, quantize_dq_kernel<false, false, true, QT>,
+      quantize_dq_kernel<false, true, false, QT>,  quantize_dq_kernel<false, true, true, QT>,
+      quantize_dq_kernel<true, false, false, QT>,  quantize_dq_kernel<true, false, true, QT>,
+      quantize_dq_kernel<true, true, false, QT>,   quantize_dq_kernel<true, true, true, QT>};
   const KFn kernel = table[(bucketed ? 4 : 0) + (v8 ? 2 : 0) + (dq_bucketed ? 1 : 0)];
   // one group (256 blocks) per CTA pass, one resident wave
   const int64_t ng = cdiv(nblocks, 256);
-  const int grid = grid_for(ng, 1, d.sms, resident_per_sm<quantize_dq_kernel<true, true, true>>(256));
-  return launch_pdl(kernel, grid, 256, 0, static_cast<cudaStream_t>(stream), reinterpret_cast<const uint4 *>(W),
+  const int grid = grid_for(ng, 1, d.sms, resident_per_sm<quantize_dq_kernel<true, true, true, QT>>(QT));
+  return launch_pdl(kernel, grid, QT, 0, static_cast<cudaStream_t>(stream), reinterpret_cast<const uint4 *>(W),
                     nblocks, reinterpret_cast<uint32_t *>(packed), q, scale2, absmax, make_tables(nf4, t8), bt,
                     *dbt);
 }
