@@ -660,10 +660,10 @@ qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a
 
 // -------------------------------------------------------- fused GEMMs --
 // The pair variants of the fused GEMM (256 weight rows x 256 tokens per
-// cluster of two CTAs): token stages of kPairBkb K blocks of 128 tokens
-// (one TMA box each), dequantized-weight stages of one K block (16 KB) and
+// cluster of two CTAs): six token stages of one K block of 128 tokens (one
+// 16 KB TMA box each), dequantized-weight stages of one K block (16 KB) and
 // packed-code slots of 4 K blocks (18 KB).
-constexpr int kPairBkb = 2, kPairSb = 3, kPairSa = 4, kPairSp = 2, kPairNpw = 8;
+constexpr int kPairBkb = 1, kPairSb = 6, kPairSa = 4, kPairSp = 2, kPairNpw = 8;
 using FwdPairCfg = GemmCfg<256, A_DEQ_K, L2_A_MN, kPairBkb, kPairSb, kPairSa, kPairSp, kPairNpw, true>;
 using BwdPairCfg = GemmCfg<256, A_DEQ_MN, L2_A_K, kPairBkb, kPairSb, kPairSa, kPairSp, kPairNpw, true>;
 // Two 256-token sub-tiles per job (512 tokens per tile, each CTA loading 256
