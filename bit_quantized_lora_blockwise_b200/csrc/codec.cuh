@@ -567,47 +567,5 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint4 *__restrict__ 
   }
 }
 
-// ------------------------------------------------------------------------
-// Decoded block constants for the GEMMs, block-major: cprime[kb * N + n] =
-// t8[q_b] * scale2[b / 256] (fp32 product), b = n * KB + kb. One work item
-// is 16 consecutive blocks of one row n: its codes come in with one 16-byte
-// load (byte loads when KB is not a multiple of 16), its one or two
-// second-level scales with two loads, all issued before any is used, so a
-// thread waits for memory once per item rather than once per constant.
-// Consecutive threads take consecutive rows of the same 16 blocks, so every
-// one of the 16 stores is coalesced across the warp. Thread `first` of
-// `stride` threads takes every stride-th item. t8 is a 256-entry table in
-// shared memory.
-__device__ __forceinline__ void decode_constants_range(const uint8_t *__restrict__ q,
-                                                       const float *__restrict__ scale2, int64_t N, int64_t KB,
-                                                       float *__restrict__ cprime, const float *t8,
-                                                       int64_t first, int64_t stride) {
-  const int64_t items = N * ((KB + 15) / 16);
-  const bool vec = (KB & 15) == 0;  // every row's 16-block groups are 16-byte aligned
-  for (int64_t w = first; w < items; w += stride) {
-    const int64_t g = w / N;
-    const int64_t n = w - g * N;
-    const int64_t kb0 = g * 16;
-    const int nv = static_cast<int>(KB - kb0 < 16 ? KB - kb0 : 16);
-    const int64_t b0 = n * KB + kb0;
-    uint32_t code[16];
-    if (vec) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(q + b0));
-      const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int i = 0; i < 16; ++i) code[i] = (wd[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) code[i] = i < nv ? __ldg(q + b0 + i) : 0u;
-    }
-    const int64_t grp0 = b0 >> 8;  // 16 consecutive blocks span at most two 256-groups
-    const float s0 = __ldg(scale2 + grp0);
-    const float s1 = __ldg(scale2 + ((b0 + nv - 1) >> 8));
-    float *dst = cprime + kb0 * N + n;
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      if (i < nv) dst[i * N] = __fmul_rn(t8[code[i]], ((b0 + i) >> 8) == grp0 ? s0 : s1);
-  }
-}
 
 }  // namespace qlora

@@ -70,7 +70,6 @@ struct GemmArgs {
   CUtensorMap tm_pk;  // packed NF4 codes
   CUtensorMap tm_a2;  // low-rank A2
   CUtensorMap tm_b2;  // low-rank B2 [tokens, r]: box {64, B_ROWS}
-  CUtensorMap tm_cp;  // decoded block constants c' [K/64][N] fp32
   // Output: 16-bit (bf16, or fp16 when f16) out[col * out_ld + row] (the transposed tile).
   void *out;
   int64_t out_ld;
@@ -89,7 +88,13 @@ struct GemmArgs {
   int tail_subtiles;
   int lora_kblocks;       // 64-deep K blocks of the low-rank product (last split only)
   int f16;                // operands, decoded weight and output are fp16 (else bf16)
+  // Block constants, decoded by the producers: c'_b = t8[q_b] * scale2[b / 256]
+  // for block b = n * wkb + kb of the row-major weight W [N, wkb * 64].
+  const uint8_t *q;
+  const float *scale2;
+  int64_t wkb;
   float nf4[16];
+  float t8[256];
 };
 
 template <int BN_, int ASRC_, int L2_, int BKB_, int SB_, int SA_, int SP_, int NPW_, bool PAIR_, int NTT_ = 1>
@@ -120,12 +125,11 @@ struct GemmCfg {
   static constexpr int B_BYTES = KB_BYTES * BKB;
   // P slot: the packed codes of KSUP consecutive 64-deep K blocks of the
   // 128-row weight tile (128 contiguous bytes per weight row: forward;
-  // 64 bytes of 4 x 64 rows: backward), then their 4 x 128 decoded block
-  // constants c'; both by TMA, shared by KSUP consecutive MMA jobs.
+  // 64 bytes of 4 x 64 rows: backward), by TMA, shared by KSUP consecutive
+  // MMA jobs. (The block constants come from q and scale2 directly.)
   static constexpr int KSUP = 4;
   static constexpr int PK_BYTES = 4096 * KSUP;
-  static constexpr int P_CP = PK_BYTES;
-  static constexpr int P_BYTES = P_CP + 512 * KSUP;
+  static constexpr int P_BYTES = PK_BYTES;
   static constexpr int OFF_B = 0;
   static constexpr int OFF_A = OFF_B + SB * B_BYTES;
   static constexpr int OFF_P = OFF_A + SA * A_BYTES;
@@ -133,9 +137,11 @@ struct GemmCfg {
   // b_full[SB] b_empty[SB] a_full[SA] a_empty[SA] p_full[SP] p_empty[SP]
   // tmem_full[2] tmem_empty[2] drain
   static constexpr int NBARS = 2 * SB + 2 * SA + 2 * SP + 5;
-  // misc: tmem base, abort flag, last-CTA flag (16 B), then the 16 NF4 levels
+  // misc: tmem base, abort flag, last-CTA flag (16 B), the 16 NF4 levels,
+  // then the 256-entry 8-bit constant table
   static constexpr int OFF_MISC = ((OFF_BAR + NBARS * 8) + 15) & ~15;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 64;
+  static constexpr int OFF_T8 = OFF_MISC + 16 + 64;
+  static constexpr int SMEM_BYTES = OFF_T8 + 1024;
   static constexpr int WARPS = 7 + NPW_;
   static constexpr int THREADS = WARPS * 32;
   // two accumulators of BN columns: double-buffered tiles (NTT = 1) or the
@@ -239,15 +245,13 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     fence_barrier_init();
   }
   if (threadIdx.x < 16) reinterpret_cast<float *>(smem + C::OFF_MISC + 16)[threadIdx.x] = args.nf4[threadIdx.x];
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) reinterpret_cast<float *>(smem + C::OFF_T8)[i] = args.t8[i];
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&args.tm_b);
     tma_prefetch_desc(&args.tm_a2);
     tma_prefetch_desc(&args.tm_b2);
   }
-  if (warp == 6 && lane == 0) {
-    tma_prefetch_desc(&args.tm_pk);
-    tma_prefetch_desc(&args.tm_cp);
-  }
+  if (warp == 6 && lane == 0) tma_prefetch_desc(&args.tm_pk);
   if (warp == 5) {
     if constexpr (C::PAIR) {
       tmem_alloc_pair(smem_u32(s_tmem), C::TMEM_COLS);
@@ -279,10 +283,17 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
   auto wait_warp = [&](uint32_t bar, uint32_t par) -> bool {
     return __all_sync(0xFFFFFFFFu, mbar_wait(bar, par, s_abort));
   };
-  // everything above overlaps the previous kernel's tail; its outputs are
-  // read only below
-  grid_dep_wait();
-  grid_dep_launch();
+  // Programmatic launch. The kernel before this one in the stream is the
+  // call's low-rank launch (X A or dY B^T), and everything before that is
+  // complete when this kernel starts (that launch waits for it before it
+  // lets this one start). This kernel reads that launch's outputs only in
+  // two places: the low-rank operand (the token TMA warp, before its first
+  // low-rank stage) and the split-K tile counters it zeroes (the epilogue,
+  // before its first counter); everything else (tokens, packed codes and
+  // constants, the adapter weights) is an input of the call, so the main K
+  // loop runs while that launch is still working. The TMA warp alone lets
+  // the next kernel start, and only after its own wait, so a started
+  // dependent still implies that this call's earlier launches are complete.
 
   // tiles of TILE_ROWS weight rows x BN tokens; a pair (cluster) takes every
   // (number of pairs)-th tile
@@ -299,6 +310,14 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     if (lane == 0) {
       uint32_t job = 0, bs = 0;  // A-ring job and B-ring stage counters
       bool ok = true;
+      bool waited = false;
+      auto wait_prior = [&]() {
+        if (!waited) {
+          grid_dep_wait();
+          grid_dep_launch();
+          waited = true;
+        }
+      };
       // one stage load: into this CTA's slot, counted on the leader's barrier
       auto load = [&](uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
         if constexpr (C::PAIR) tma_load_2d_pair(dst, map, map_cluster(bar, 0u), x, y);
@@ -321,6 +340,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
             job += (st + 1 < nbm) ? C::BKB : t.nmain - st * C::BKB;
           } else {
             // low-rank K block: B2 into the stage, A2 into this job's A slot
+            wait_prior();  // B2 is the previous launch's output
             const int lk = st - nbm;
             const int sa = job % C::SA;
             if (!mbar_wait(a_empty(sa), ((job / C::SA) & 1u) ^ 1u, s_abort)) { ok = false; break; }
@@ -337,6 +357,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
           }
         }
       }
+      wait_prior();
       // wait (bounded) for this thread's copies still in flight (a pair's
       // copies complete on the leader's barriers, which count both halves;
       // the peer stays resident until the leader is past this point: the
@@ -526,6 +547,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
         if (lane == 0) arrive_leader(tmem_empty(u & 1u));  // accumulator free (its partial is in memory)
       }
       if (!ok || t.nsplit == 1) continue;
+      grid_dep_wait();  // the tile counters are zeroed by the previous launch
       __threadfence();
       named_bar_sync(1, 128);
       if (warp == 0 && lane == 0) {
@@ -554,9 +576,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
   } else if (warp == 6) {
     // ------------------------------------------------ P ring: TMA issue --
     // Runs up to SP superjobs ahead of the producers, gated only by them:
-    // the packed codes of the 128 x (64 KSUP) weight tile and its decoded
-    // block constants (c' is block-major, so they are contiguous 512-byte
-    // rows for the forward and 256-byte rows for the backward).
+    // the packed codes of the 128 x (64 KSUP) weight tile.
     if (lane == 0) {
       uint32_t ms = 0;  // superjob counter (KSUP main jobs each, per tile)
       bool ok = true;
@@ -568,13 +588,8 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
           const int kb0 = t.kb_begin + u * C::KSUP;
           const uint32_t p_dst = sbase + C::OFF_P + sp * C::P_BYTES;
           mbar_arrive_expect_tx(p_full(sp), C::P_BYTES);
-          if (C::ASRC == A_DEQ_K) {
-            tma_load_2d(p_dst, &args.tm_pk, p_full(sp), kb0 * 32, t.row0);
-            tma_load_2d(p_dst + C::P_CP, &args.tm_cp, p_full(sp), t.row0, kb0);
-          } else {
-            tma_load_2d(p_dst, &args.tm_pk, p_full(sp), t.row0 / 2, kb0 * 64);
-            tma_load_2d(p_dst + C::P_CP, &args.tm_cp, p_full(sp), kb0 * 64, t.row0 / 64);
-          }
+          if (C::ASRC == A_DEQ_K) tma_load_2d(p_dst, &args.tm_pk, p_full(sp), kb0 * 32, t.row0);
+          else tma_load_2d(p_dst, &args.tm_pk, p_full(sp), t.row0 / 2, kb0 * 64);
         }
       }
       // wait (bounded) for this thread's own copies still in flight
@@ -604,6 +619,28 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
       for (int jj = 0; jj < njobs; ++jj, ++job) {
         const bool main_job = jj < t.nmain;
         if ((int)(job % C::NGROUPS) != group) continue;
+        // this thread's block constant for the job, c' = t8[q] * S (the same
+        // fp32 product as the dequantization), loaded before the waits below
+        uint32_t qv = 0u;
+        float sv = 0.0f;  // rows past the weight: c' = 0, the rows decode to zeros
+        if (main_job) {
+          int64_t n, kblk;  // W row and 64-block of this thread's codes
+          bool valid;
+          if (C::ASRC == A_DEQ_K) {
+            n = t.row0 + p;
+            kblk = t.kb_begin + jj;
+            valid = n < args.rows;
+          } else {
+            n = static_cast<int64_t>(t.kb_begin + jj) * 64 + (p & 63);
+            kblk = t.row0 / 64 + (p >> 6);
+            valid = kblk < args.wkb;
+          }
+          if (valid) {
+            const int64_t b = n * args.wkb + kblk;
+            qv = __ldg(args.q + b);
+            sv = __ldg(args.scale2 + (b >> 8));
+          }
+        }
         const int sa = job % C::SA;
         if (!wait_warp(a_empty(sa), ((job / C::SA) & 1u) ^ 1u)) { ok = false; break; }
         if (main_job) {
@@ -616,19 +653,17 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
           // for the forward, 64-byte swizzle on 64-byte rows for the
           // backward): 16-byte chunk c of a row sits at c ^ (row bits), so
           // the 8 threads of each quarter-warp read 8 different bank groups.
-          uint32_t p_off0, p_off1, c_idx;
-          if (C::ASRC == A_DEQ_K) {  // [128 rows][KSUP x 32 B], c' [KSUP][128]
+          uint32_t p_off0, p_off1;
+          if (C::ASRC == A_DEQ_K) {  // [128 rows][KSUP x 32 B]
             const uint32_t x = p & 7;
             p_off0 = p * (32 * C::KSUP) + (((2 * sub) ^ x) << 4);
             p_off1 = p * (32 * C::KSUP) + (((2 * sub + 1) ^ x) << 4);
-            c_idx = sub * 128 + p;
-          } else {  // [KSUP x 64 rows][2 x 32 B], c' [2][KSUP x 64]
+          } else {  // [KSUP x 64 rows][2 x 32 B]
             const uint32_t row = sub * 64 + (p & 63), x = (row >> 1) & 3, c0 = 2 * (p >> 6);
             p_off0 = row * 64 + ((c0 ^ x) << 4);
             p_off1 = row * 64 + (((c0 + 1) ^ x) << 4);
-            c_idx = (p >> 6) * (64 * C::KSUP) + sub * 64 + (p & 63);
           }
-          const float cp = reinterpret_cast<const float *>(pslot + C::P_CP)[c_idx];
+          const float cp = __fmul_rn(reinterpret_cast<const float *>(smem + C::OFF_T8)[qv], sv);
           const uint4 w0 = *reinterpret_cast<const uint4 *>(pslot + p_off0);
           const uint4 w1 = *reinterpret_cast<const uint4 *>(pslot + p_off1);
           __syncwarp();

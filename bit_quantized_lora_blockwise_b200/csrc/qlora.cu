@@ -400,7 +400,6 @@ int resident_pairs() {
 
 // Block constants c' = t8[q] * S, block-major [K/64][N] fp32 (GEMM operand
 // staging), decoded once per call by extra CTAs of the first skinny launch.
-size_t cprime_bytes(int64_t N, int64_t K) { return align256(static_cast<size_t>(N) * (K / 64) * 4); }
 
 // Layer sizes shared by forward and backward.
 struct Shape {
@@ -539,14 +538,6 @@ qlora_status run_skinny(const SkinnyArgs &a, int bn, int grid, cudaStream_t st) 
   return run_skinny_bn<256, AMN, BMN>(a, grid, st);
 }
 
-// Constants pass folded into a skinny launch (extra CTAs, see SkinnyArgs).
-struct DecodeSpec {
-  const uint8_t *q;
-  const float *scale2;
-  float *cprime;
-  int64_t N, KB;
-  const float *t8;  // host table
-};
 
 // kind: SK_XA   Aop = X [M,K] (K-major),   Bop = A  [K,r] (MN-major), rows = M, kdim = K
 //       SK_G    Aop = dY [M,N] (K-major),  Bop = B  [r,N] (K-major),  rows = M, kdim = N
@@ -573,10 +564,10 @@ struct SkinnyOperands {
 };
 
 // Launch one or two products of the same kind (same operand layouts and
-// reduction length) as one grid; optionally with the constants pass.
+// reduction length) as one grid.
 qlora_status skinny_launch(SkinnyKind kind, const SkinnyOperands *ops, int nprob, int r, int sms,
                            cudaStream_t st, unsigned int *zero_words, int nzero, bool early,
-                           const DecodeSpec *dc, bool late = false) {
+                           bool late = false) {
   int row_tiles[2] = {0, 0};
   for (int i = 0; i < nprob; ++i) row_tiles[i] = static_cast<int>(cdiv(ops[i].rows, 128));
   // the split is chosen for all row tiles of the launch together
@@ -626,23 +617,7 @@ qlora_status skinny_launch(SkinnyKind kind, const SkinnyOperands *ops, int nprob
   a.early = early ? 1 : 0;
   a.late = late ? 1 : 0;
   a.f16 = t_f16 ? 1 : 0;
-  a.gemm_ctas = (row_tiles[0] + row_tiles[1]) * p.splits;
-  int grid = a.gemm_ctas;
-  if (dc != nullptr) {
-    // one item (16 constants of a row) per thread, on the CTA slots the GEMM
-    // CTAs leave free, in whole clusters
-    const int64_t want = cdiv(dc->N * cdiv(dc->KB, 16), 256);
-    const int64_t free_slots = static_cast<int64_t>(p.per_sm) * sms - a.gemm_ctas;
-    int64_t n = std::min(want, std::max<int64_t>(free_slots, p.splits));
-    n = cdiv(std::max<int64_t>(n, 1), p.splits) * p.splits;
-    grid += static_cast<int>(n);
-    a.dc_q = dc->q;
-    a.dc_scale2 = dc->scale2;
-    a.dc_cprime = dc->cprime;
-    a.dc_N = dc->N;
-    a.dc_KB = dc->KB;
-    std::memcpy(a.dc_t8, dc->t8, sizeof a.dc_t8);
-  }
+  const int grid = (row_tiles[0] + row_tiles[1]) * p.splits;
   switch (kind) {
     case SK_XA: return run_skinny<false, true>(a, p.bn, grid, st);
     case SK_G: return run_skinny<false, false>(a, p.bn, grid, st);
@@ -653,9 +628,9 @@ qlora_status skinny_launch(SkinnyKind kind, const SkinnyOperands *ops, int nprob
 qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a_outer, const void *bop,
                     int64_t b_inner, int64_t b_outer, int64_t rows, int64_t kdim, int r, const OutSpec &o,
                     int sms, cudaStream_t st, unsigned int *zero_words = nullptr, int nzero = 0,
-                    bool early = false, const DecodeSpec *dc = nullptr) {
+                    bool early = false) {
   const SkinnyOperands op{aop, a_inner, a_outer, bop, b_inner, b_outer, rows, kdim, o};
-  return skinny_launch(kind, &op, 1, r, sms, st, zero_words, nzero, early, dc);
+  return skinny_launch(kind, &op, 1, r, sms, st, zero_words, nzero, early);
 }
 
 // -------------------------------------------------------- fused GEMMs --
@@ -812,9 +787,9 @@ qlora_status run_smallm(const SmallmArgs &a, const SmallmPlan &p, cudaStream_t s
   return p.nt == 1 ? run_smallm_nt<1, false>(a, p.grid, st) : run_smallm_nt<2, false>(a, p.grid, st);
 }
 
-// Workspace carve-up: [tile counters][bf16 M x r][bf16 M x r (backward)][c'][fp32 partials]
+// Workspace carve-up: [tile counters][bf16 M x r][bf16 M x r (backward)][fp32 partials]
 struct WsLayout {
-  size_t counters, mr, cprime, part, total;
+  size_t counters, mr, part, total;
   int64_t ncounters;
 };
 
@@ -823,16 +798,15 @@ WsLayout ws_layout(const Shape &s, int sms, bool backward) {
   w.ncounters = counters_needed(s);
   w.counters = align256(static_cast<size_t>(w.ncounters) * 4);
   w.mr = align256(static_cast<size_t>(s.M) * s.r * 2);
-  w.cprime = cprime_bytes(s.N, s.K);
   if (!backward) {
     w.part = s.M <= kSmallmMaxTokens ? plan_smallm(s.M, s.N, s.K, sms, 0).part_bytes
                                      : fused_part_bound(s.M, s.N, s.K / 64, sms);
-    w.total = w.counters + w.mr + w.cprime + w.part;
+    w.total = w.counters + w.mr + w.part;
   } else {
     // the skinny GEMMs reduce their split-K partials in shared memory
     const size_t part = fused_part_bound(s.M, s.K, s.N / 64, sms);   // dX split-K
     w.part = part;
-    w.total = w.counters + 2 * w.mr + w.cprime + w.part;
+    w.total = w.counters + 2 * w.mr + w.part;
   }
   return w;
 }
@@ -1084,8 +1058,7 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   unsigned int *counters = reinterpret_cast<unsigned int *>(ws);
   qlora_bf16 *xas = reinterpret_cast<qlora_bf16 *>(ws + w.counters);
-  float *cprime = reinterpret_cast<float *>(ws + w.counters + w.mr);
-  float *part = reinterpret_cast<float *>(ws + w.counters + w.mr + w.cprime);
+  float *part = reinterpret_cast<float *>(ws + w.counters + w.mr);
 
   if (M <= kSmallmMaxTokens) {
     // Few tokens: XA (which also zeroes the band counters), then one pass over
@@ -1120,13 +1093,12 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   }
 
   // 1) XA = X A -> XA_out = bf16(XA) (if wanted), xas = bf16(s XA); the same
-  //    launch decodes the block constants c' for the GEMM producers and
-  //    zeroes the split-K tile counters. The first ring stages may go out
-  //    before the wait only when the launch before it is one of this call's.
+  //    launch zeroes the split-K tile counters. The GEMM after it decodes
+  //    the block constants itself and waits for this launch only before its
+  //    low-rank K-steps and its counters, so its main loop overlaps it.
   {
     OutSpec o{xas, r, scl, XA_out, r, 1.0f, false};
-    const DecodeSpec dc{q, scale2, cprime, N, K / 64, t8};
-    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs, counters, static_cast<int>(w.ncounters), false, &dc);
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs, counters, static_cast<int>(w.ncounters), false);
     if (st != QLORA_OK) return st;
   }
 
@@ -1138,7 +1110,6 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   std::memset(&a, 0, sizeof a);
   if (!map_tokens_3d(&a.tm_b, X, M, K, b_rows, bkb) ||
       !make_map(&a.tm_pk, packed, MAP_U8, K / 2, N, K / 2, 128, 128, SW_128B) ||
-      !make_map(&a.tm_cp, cprime, MAP_F32, N, K / 64, N * 4, 128, 4, SW_NONE) ||
       !map_mnmajor(&a.tm_a2, B, N, r) || !map_kmajor(&a.tm_b2, xas, r, M, b_rows))
     return QLORA_ERR_CUDA;
   a.rows = static_cast<int>(N);
@@ -1153,6 +1124,10 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   a.part = part;
   a.counters = counters;
   std::memcpy(a.nf4, nf4, sizeof a.nf4);
+  std::memcpy(a.t8, t8, sizeof a.t8);
+  a.q = q;
+  a.scale2 = scale2;
+  a.wkb = K / 64;
   a.f16 = t_f16 ? 1 : 0;
   trace_begin(cs);
   st = fp.pair ? (fp.ntt == 2 ? run_fused_pair<FwdPair2Cfg>(a, d.sms, fp.slots, cs)
@@ -1186,15 +1161,13 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   unsigned int *counters = reinterpret_cast<unsigned int *>(ws);
   qlora_bf16 *gs = reinterpret_cast<qlora_bf16 *>(ws + w.counters);
   qlora_bf16 *xa_ws = reinterpret_cast<qlora_bf16 *>(ws + w.counters + w.mr);
-  float *cprime = reinterpret_cast<float *>(ws + w.counters + 2 * w.mr);
-  float *part = reinterpret_cast<float *>(ws + w.counters + 2 * w.mr + w.cprime);
+  float *part = reinterpret_cast<float *>(ws + w.counters + 2 * w.mr);
 
-  // 1) Gs = bf16(s * dY B^T); the same launch decodes c' and zeroes the
-  //    tile counters (first kernel of the call: it waits before loading)
+  // 1) Gs = bf16(s * dY B^T); the same launch zeroes the tile counters
+  //    (first kernel of the call: it waits before loading)
   {
     OutSpec o{gs, r, scl, nullptr, 0, 0.0f, false};
-    const DecodeSpec dc{q, scale2, cprime, N, K / 64, t8};
-    st = skinny(SK_G, dY, N, M, B, N, r, M, N, r, o, d.sms, cs, counters, static_cast<int>(w.ncounters), false, &dc);
+    st = skinny(SK_G, dY, N, M, B, N, r, M, N, r, o, d.sms, cs, counters, static_cast<int>(w.ncounters), false);
     if (st != QLORA_OK) return st;
   }
 
@@ -1216,7 +1189,6 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   std::memset(&a, 0, sizeof a);
   if (!map_tokens_3d(&a.tm_b, dY, M, N, b_rows, bkb) ||
       !make_map(&a.tm_pk, packed, MAP_U8, K / 2, N, K / 2, 64, 256, SW_64B) ||
-      !make_map(&a.tm_cp, cprime, MAP_F32, N, K / 64, N * 4, 256, 2, SW_NONE) ||
       !map_kmajor(&a.tm_a2, A, r, K, 128) || !map_kmajor(&a.tm_b2, gs, r, M, b_rows))
     return QLORA_ERR_CUDA;
   a.rows = static_cast<int>(K);
@@ -1231,6 +1203,10 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   a.part = part;
   a.counters = counters;
   std::memcpy(a.nf4, nf4, sizeof a.nf4);
+  std::memcpy(a.t8, t8, sizeof a.t8);
+  a.q = q;
+  a.scale2 = scale2;
+  a.wkb = K / 64;
   a.f16 = t_f16 ? 1 : 0;
   trace_begin(cs);
   st = fp.pair ? (fp.ntt == 2 ? run_fused_pair<BwdPair2Cfg>(a, d.sms, fp.slots, cs)
@@ -1250,7 +1226,7 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   const SkinnyOperands ops[2] = {
       {X, K, M, gs, r, M, K, M, OutSpec{dA, r, 1.0f, nullptr, 0, 0.0f, false}},
       {dY, N, M, xa, r, M, N, M, OutSpec{dB, N, scl, nullptr, 0, 0.0f, true}}};
-  return skinny_launch(SK_DA, ops, 2, r, d.sms, cs, nullptr, 0, true, nullptr, true);
+  return skinny_launch(SK_DA, ops, 2, r, d.sms, cs, nullptr, 0, true, true);
 }
 
 qlora_status qlora_dequant_dt(const uint8_t *packed, const uint8_t *q, const float *scale2, int64_t N, int64_t K,

@@ -51,14 +51,6 @@ struct SkinnyArgs {
               // the kernel before it, so the whole product runs without waiting for that kernel; each
               // thread waits for it only before exiting, so this grid still completes after it
   int f16;   // operands and outputs are fp16 (else bf16)
-  // Optional constants pass for the fused GEMM that follows, run by the CTAs
-  // from gemm_ctas on (whole clusters): cprime[kb * dc_N + n] = t8[q] * S.
-  int gemm_ctas;
-  const uint8_t *dc_q;
-  const float *dc_scale2;
-  float *dc_cprime;
-  int64_t dc_N, dc_KB;
-  float dc_t8[256];
 };
 
 template <int BN_, bool A_MN_, bool B_MN_, int STAGES_>
@@ -86,17 +78,6 @@ template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1) skinny_kernel(const __grid_constant__ SkinnyArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = smem_raw;  // 1024-byte aligned: the 128-byte swizzle atoms need it
-  if (static_cast<int>(blockIdx.x) >= args.gemm_ctas) {
-    // constants pass (no TMEM, no cluster barrier; these CTAs just return)
-    float *s_t8 = reinterpret_cast<float *>(smem);
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) s_t8[i] = args.dc_t8[i];
-    __syncthreads();
-    grid_dep_wait();
-    const int64_t stride = static_cast<int64_t>(gridDim.x - args.gemm_ctas) * blockDim.x;
-    const int64_t first = static_cast<int64_t>(blockIdx.x - args.gemm_ctas) * blockDim.x + threadIdx.x;
-    decode_constants_range(args.dc_q, args.dc_scale2, args.dc_N, args.dc_KB, args.dc_cprime, s_t8, first, stride);
-    return;
-  }
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
