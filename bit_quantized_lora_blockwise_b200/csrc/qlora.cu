@@ -755,7 +755,10 @@ SmallmPlan plan_smallm(int64_t M, int64_t N, int64_t K, int sms, int busy_sms) {
   p.kc = static_cast<int>(cdiv(K, 256));
   p.units = p.bands * p.kc;
   const int avail = std::max(1, sms - busy_sms);
-  p.grid = std::min(p.units, avail);
+  // at least two units per CTA: a band then spans half as many CTAs, whose
+  // serial reduction at the end costs more on small weights than the
+  // parallelism it buys (4096 x 4096 at 16 tokens: 20.5 us against 26.8)
+  p.grid = std::min(std::max(1, p.units / 2), avail);
   // two partial slots per CTA: its pieces of the bands shared with other CTAs
   p.part_bytes = align256(static_cast<size_t>(p.grid) * 2 * SmallmCfg<1>::WARPS * p.nt * 32 * 16);
   return p;
