@@ -612,33 +612,56 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
     const uint32_t swz = p & 7;
     uint32_t job = 0, ms = 0;  // ms: superjob counter at the start of the tile
     bool ok = true;
+    // the 8-bit code and second-level scale of this thread's block in main
+    // job jj of tile t (0 and 0.0 past the weight)
+    auto load_consts = [&](const TileCoord &t, int jj, uint32_t &qv, float &sv) {
+      int64_t n, kblk;  // W row and 64-block of this thread's codes
+      bool valid;
+      if (C::ASRC == A_DEQ_K) {
+        n = t.row0 + p;
+        kblk = t.kb_begin + jj;
+        valid = n < args.rows;
+      } else {
+        n = static_cast<int64_t>(t.kb_begin + jj) * 64 + (p & 63);
+        kblk = t.row0 / 64 + (p >> 6);
+        valid = kblk < args.wkb;
+      }
+      qv = 0u;
+      sv = 0.0f;
+      if (valid) {
+        const int64_t b = n * args.wkb + kblk;
+        qv = __ldg(args.q + b);
+        sv = __ldg(args.scale2 + (b >> 8));
+      }
+    };
+    int pf_jj = -1;  // main job of the current tile whose constants are in pf_q, pf_s
+    uint32_t pf_q = 0u;
+    float pf_s = 0.0f;
     for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
       const TileCoord t = coord(tile);
       const int njobs = t.nmain + t.nlora;
+      pf_jj = -1;
       const int nsup = (t.nmain + C::KSUP - 1) / C::KSUP;
       for (int jj = 0; jj < njobs; ++jj, ++job) {
         const bool main_job = jj < t.nmain;
         if ((int)(job % C::NGROUPS) != group) continue;
         // this thread's block constant for the job, c' = t8[q] * S (the same
-        // fp32 product as the dequantization), loaded before the waits below
+        // fp32 product as the dequantization): its code and scale were loaded
+        // one of this group's jobs ahead (or here, for a tile's first jobs)
         uint32_t qv = 0u;
         float sv = 0.0f;  // rows past the weight: c' = 0, the rows decode to zeros
         if (main_job) {
-          int64_t n, kblk;  // W row and 64-block of this thread's codes
-          bool valid;
-          if (C::ASRC == A_DEQ_K) {
-            n = t.row0 + p;
-            kblk = t.kb_begin + jj;
-            valid = n < args.rows;
+          if (pf_jj == jj) {
+            qv = pf_q;
+            sv = pf_s;
           } else {
-            n = static_cast<int64_t>(t.kb_begin + jj) * 64 + (p & 63);
-            kblk = t.row0 / 64 + (p >> 6);
-            valid = kblk < args.wkb;
+            load_consts(t, jj, qv, sv);
           }
-          if (valid) {
-            const int64_t b = n * args.wkb + kblk;
-            qv = __ldg(args.q + b);
-            sv = __ldg(args.scale2 + (b >> 8));
+          if (jj + C::NGROUPS < t.nmain) {  // this group's next job of the tile
+            load_consts(t, jj + C::NGROUPS, pf_q, pf_s);
+            pf_jj = jj + C::NGROUPS;
+          } else {
+            pf_jj = -1;
           }
         }
         const int sa = job % C::SA;
