@@ -454,6 +454,8 @@ def workload_phases(dev, hbm_gbs, tc_tflops, quick=False):
       single_1024          one 1024x1024 linear, M = 16, r = 8: fwd + bwd latency
       llama13b_quant_sweep quantize + double quant, and dequant, over 40 layers x 7 linears
       llama65b_fwd         7 linears: few-token forwards (M = 1, 4, 16) and M = 4096
+      llama7b_f16          the 7B set's fused fwd + bwd with fp16 operands
+      paged_adamw_7b_adapters  one AdamW step over the 7B adapters, state on the device / paged out
       llama33b_block       7 linears, M = 2048: block fwd + block bwd recomputing XA (and one by one)
     Rates are against the measured peaks and the spec ones (8 TB/s HBM,
     2.25 PFLOP/s dense bf16)."""
@@ -577,6 +579,56 @@ def workload_phases(dev, hbm_gbs, tc_tflops, quick=False):
             c4[f"M{m}"] = {"ms": round(ms, 4), **frac_tc(flops / (ms * 1e-3) / 1e12)}
     out["llama65b_fwd"] = c4
     del packed, acts, Ybuf, XAbuf, ws
+
+    # -- 7B set in fp16 (the pages' other 16-bit compute type): fused fwd + bwd
+    wl = WORKLOADS["llama7b_set"]
+    M = wl.M[0]
+    f16 = []
+    for li, lin in enumerate(wl.linears):
+        inp = layer_inputs(wl, li, M, device=dev)
+        pk, q, s2 = quantized(inp["W"])
+        h = {k: inp[k].to(torch.float16) for k in ("X", "A", "B", "dY")}
+        del inp
+        f16.append((lin, pk, q, s2, h, torch.empty((M, lin.N), dtype=torch.float16, device=dev),
+                    torch.empty((M, wl.r), dtype=torch.float16, device=dev),
+                    torch.empty((M, lin.K), dtype=torch.float16, device=dev),
+                    torch.empty((lin.K, wl.r), dtype=torch.float16, device=dev),
+                    torch.empty((wl.r, lin.N), dtype=torch.float16, device=dev)))
+    ws = torch.empty(max(binding.workspace_bytes(M, lin.N, lin.K, wl.r) for lin, *_ in f16),
+                     dtype=torch.uint8, device=dev)
+
+    def fwd_bwd_f16():
+        for lin, pk, q, s2, h, Y, XA, dX, dA, dB in f16:
+            binding.linear_fwd(pk, q, s2, h["X"], h["A"], h["B"], wl.alpha, lin.N, lin.K, Y=Y, XA_out=XA,
+                               workspace=ws)
+            binding.linear_bwd(pk, q, s2, h["X"], h["dY"], h["A"], h["B"], wl.alpha, lin.N, lin.K, XA=XA, dX=dX,
+                               dA=dA, dB=dB, workspace=ws)
+    ms = device_ms(fwd_bwd_f16, 5)
+    flops = sum(linear_flops(M, lin.N, lin.K, wl.r) for lin, *_ in f16)
+    out["llama7b_f16"] = {"what": "7 linears of the 7B set, M=2048, r=64, fp16 operands and outputs: "
+                                  "qlora_linear_fwd + qlora_linear_bwd (the _dt calls)",
+                          "ms": round(ms, 4), **frac_tc(flops / (ms * 1e-3) / 1e12)}
+
+    # -- paged AdamW over the 7B set's adapters: state on the device, and paged out to the host
+    grads = [t for *_, dA, dB in f16 for t in (dA, dB)]
+    params = [t.clone() for lin, pk, q, s2, h, *_ in f16 for t in (h["A"], h["B"])]
+    n_el = sum(t.numel() for t in params)
+    adamw = {}
+    for where, reserve in (("device", 0), ("host", 1 << 62)):
+        opt = binding.PagedAdamW(params, lr=1e-4, weight_decay=0.01)
+        opt.set_reserve(reserve)
+        opt.step(grads)  # places the state
+        torch.cuda.synchronize()
+        ms = device_ms(lambda: opt.step(grads), 10)
+        gbs = n_el * 28 / (ms * 1e-3) / 1e9  # 2 B grad + 12 B state read + 12 B written + 2 B param
+        adamw[where] = {"ms": round(ms, 4), "placement": opt.location, "GB/s": round(gbs, 1),
+                        **({"frac_hbm": round(gbs / hbm_gbs, 3)} if where == "device" else {})}
+        opt.close()
+    out["paged_adamw_7b_adapters"] = {"what": f"one AdamW step over the 14 adapter tensors of the 7B set "
+                                              f"({n_el / 1e6:.2f} M fp16 parameters, fp32 state in managed memory)",
+                                      **adamw}
+    del f16, ws, grads, params
+    torch.cuda.empty_cache()
 
     # -- 33B-shaped block: forward saving XA, backward recomputing XA (checkpoint style)
     wl = WORKLOADS["llama33b_block"]
