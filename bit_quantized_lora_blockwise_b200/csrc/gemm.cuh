@@ -50,9 +50,10 @@
 //   warp 6     TMA issue for the packed-code ring (one lane)
 //   warps 7..  dequant producers (NPW warps, in groups of 4 that take turns)
 // Rings (mbarrier-guarded): B (SB stages), dequantized A (SA stages, one per
-// 64-deep job), packed codes + block constants (SP slots of KSUP jobs); two
-// TMEM accumulators (tmem_full, tmem_empty) so the epilogue of one tile
-// overlaps the mainloop of the next. Every wait is bounded (mbar_wait); on a
+// 64-deep job), packed codes (SP slots of KSUP jobs; each producer thread
+// reads its block's 8-bit constant code and second-level scale from global
+// memory one job ahead); two TMEM accumulators (tmem_full, tmem_empty) so the
+// epilogue of one tile overlaps the mainloop of the next. Every wait is bounded (mbar_wait); on a
 // timeout the CTA drains its own copies and MMAs, frees TMEM and returns with
 // the device error word set.
 #pragma once
