@@ -61,6 +61,10 @@ def parse():
     ap.add_argument("--no-compare", action="store_true",
                     help="skip the dequantize-then-cuBLAS comparison leg")
     ap.add_argument("--linears", default="", help="comma list of linear names to keep (profiling runs)")
+    ap.add_argument("--phase", default="",
+                    help="run only this diagnostic workload phase (no headline step; a profiling aid): "
+                         "single_1024, llama13b_quant_sweep, llama65b_fwd, llama7b_f16, "
+                         "paged_adamw_7b_adapters or llama33b_block")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the diagnostic rows of the other workloads (single linear, 13B codec sweep, "
                          "65B forwards, 33B block)")
@@ -448,7 +452,7 @@ def device_ms(fn, reps, warm=2):
     return e0.elapsed_time(e1) / reps
 
 
-def workload_phases(dev, hbm_gbs, tc_tflops, quick=False):
+def workload_phases(dev, hbm_gbs, tc_tflops, quick=False, only=None):
     """Every other workload the hot path is specified on, timed on the
     device after the headline (diagnostic rows, not the headline):
       single_1024          one 1024x1024 linear, M = 16, r = 8: fwd + bwd latency
@@ -464,6 +468,9 @@ def workload_phases(dev, hbm_gbs, tc_tflops, quick=False):
     from bit_quantized_lora_blockwise_b200.inputs import WORKLOADS, layer_inputs, weight_bf16, seed_for
     out = {}
 
+    def want(name):
+        return only is None or only == name
+
     def frac_hbm(gbs):
         return {"GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm_gbs, 3), "frac_8tbs": round(gbs / SPEC_HBM_GBS, 3)}
 
@@ -476,205 +483,210 @@ def workload_phases(dev, hbm_gbs, tc_tflops, quick=False):
         q, s2 = binding.double_quant(am)
         return pk, q, s2
 
-    # -- single linear (latency; every tensor L2-resident)
-    wl = WORKLOADS["single_1024"]
-    inp = layer_inputs(wl, 0, wl.M[0], device=dev)
-    N, K, M, r = wl.linears[0].N, wl.linears[0].K, wl.M[0], wl.r
-    pk, q, s2 = quantized(inp["W"])
-    ws = torch.empty(binding.workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
-    Y, XA = torch.empty((M, N), dtype=torch.bfloat16, device=dev), torch.empty((M, r), dtype=torch.bfloat16, device=dev)
-    dX, dA, dB = (torch.empty(sh, dtype=torch.bfloat16, device=dev) for sh in ((M, K), (K, r), (r, N)))
-
-    def c1():
-        binding.linear_fwd(pk, q, s2, inp["X"], inp["A"], inp["B"], wl.alpha, N, K, Y=Y, XA_out=XA, workspace=ws)
-        binding.linear_bwd(pk, q, s2, inp["X"], inp["dY"], inp["A"], inp["B"], wl.alpha, N, K, XA=XA, dX=dX,
-                           dA=dA, dB=dB, workspace=ws)
-    ms = device_ms(c1, 50)
-    out["single_1024"] = {"what": "qlora_linear_fwd + qlora_linear_bwd, 1024x1024, M=16, r=8 (L2-resident)",
-                          "us_per_fwd_bwd": round(ms * 1e3, 2),
-                          "TFLOP/s": round(linear_flops(M, N, K, r) / (ms * 1e-3) / 1e12, 3)}
-    del inp, pk, q, s2, ws
-
-    # -- 13B-equivalent codec sweep: one layer's buffers, refilled per layer (outside the timed calls)
-    wl = WORKLOADS["llama13b_quant_sweep"]
-    layers = 4 if quick else wl.layers
-    bufs = []
-    for lin in wl.linears:
-        n = lin.N * lin.K
-        bufs.append({"N": lin.N, "K": lin.K, "W": torch.empty((lin.N, lin.K), dtype=torch.bfloat16, device=dev),
-                     "pk": torch.empty(n // 2, dtype=torch.uint8, device=dev),
-                     "am": torch.empty(n // 64, dtype=torch.float32, device=dev),
-                     "q": torch.empty(n // 64, dtype=torch.uint8, device=dev),
-                     "s2": torch.empty((n // 64 + 255) // 256, dtype=torch.float32, device=dev),
-                     "Wq": torch.empty((lin.N, lin.K), dtype=torch.bfloat16, device=dev)})
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 2x L2: written between timed calls
-    t_q = t_dq = t_d = t_qdq = 0.0
-    params = 0
-    for layer in range(layers):
-        for li, b in enumerate(bufs):
-            b["W"].copy_(weight_bf16(b["N"], b["K"], wl.w_std, seed_for(wl.index, li, 0, layer), device=dev))
-        flush.zero_()
-        t_q += device_ms(lambda: [binding.quantize_nf4(b["W"], packed=b["pk"], absmax=b["am"]) for b in bufs], 1, 0)
-        flush.zero_()
-        t_dq += device_ms(lambda: [binding.double_quant(b["am"], q=b["q"], scale2=b["s2"]) for b in bufs], 1, 0)
-        flush.zero_()
-        t_qdq += device_ms(lambda: [binding.quantize_dq(b["W"], packed=b["pk"], q=b["q"], scale2=b["s2"])
-                                    for b in bufs], 1, 0)
-        flush.zero_()
-        t_d += device_ms(lambda: [binding.dequant(b["pk"], b["q"], b["s2"], b["N"], b["K"], out=b["Wq"])
-                                  for b in bufs], 1, 0)
-        params += sum(b["N"] * b["K"] for b in bufs)
-    n = params
-    q_in, q_out = 2 * n, n // 2 + n // 64 * 4
-    dq_in, dq_out = n // 64 * 4, n // 64 + n // 16384 * 4
-    d_in, d_out = n // 2 + n // 64 + n // 16384 * 4, 2 * n
-    out["llama13b_quant_sweep"] = {
-        "what": f"{layers} layers x 7 linears (d=5120, ffn=13824), {n / 1e9:.3f} G params, per-call events summed",
-        "quantize": {"ms": round(t_q, 3), "GB_in": round(q_in / 1e9, 3), "GB_out": round(q_out / 1e9, 3),
-                     **frac_hbm((q_in + q_out) / (t_q * 1e-3) / 1e9)},
-        "double_quant": {"ms": round(t_dq, 3), **frac_hbm((dq_in + dq_out) / (t_dq * 1e-3) / 1e9)},
-        "quantize_plus_double_quant": {"ms": round(t_q + t_dq, 3),
-                                       **frac_hbm((q_in + q_out + dq_in + dq_out) / ((t_q + t_dq) * 1e-3) / 1e9)},
-        "quantize_dq_one_pass": {"ms": round(t_qdq, 3), "GB_in": round(q_in / 1e9, 3),
-                                 "GB_out": round((n // 2 + n // 64 + n // 16384 * 4) / 1e9, 3),
-                                 **frac_hbm((q_in + n // 2 + n // 64 + n // 16384 * 4) / (t_qdq * 1e-3) / 1e9)},
-        "dequant": {"ms": round(t_d, 3), "GB_in": round(d_in / 1e9, 3), "GB_out": round(d_out / 1e9, 3),
-                    **frac_hbm((d_in + d_out) / (t_d * 1e-3) / 1e9)}}
-    del bufs, flush
-
-    # -- 65B-shaped forwards: few tokens (HBM-bound) and M = 4096 (tensor-bound)
-    wl = WORKLOADS["llama65b_fwd"]
-    packed = []
-    for li, lin in enumerate(wl.linears):
-        W = weight_bf16(lin.N, lin.K, wl.w_std, seed_for(wl.index, li, 0), device=dev)
-        packed.append((lin, *quantized(W)))
-        del W
-    torch.cuda.synchronize()
-    Mmax = max(wl.M)
-    Kmax = max(lin.K for lin in wl.linears)
-    Nmax = max(lin.N for lin in wl.linears)
-    acts = []
-    for li, (lin, _, _, _) in enumerate(packed):
-        acts.append({"X": torch.randn((Mmax, lin.K), device=dev).to(torch.bfloat16),
-                     "A": (torch.randn((lin.K, wl.r), device=dev) * 0.01).to(torch.bfloat16),
-                     "B": (torch.randn((wl.r, lin.N), device=dev) * 0.01).to(torch.bfloat16)})
-    Ybuf = torch.empty(Mmax * Nmax, dtype=torch.bfloat16, device=dev)
-    XAbuf = torch.empty(Mmax * wl.r, dtype=torch.bfloat16, device=dev)
-    ws = torch.empty(max(binding.workspace_bytes(m, lin.N, lin.K, wl.r) for m in wl.M for lin, *_ in packed),
-                     dtype=torch.uint8, device=dev)
-    c4 = {"what": "7 linears (d=8192, ffn=22016), r=64: one qlora_linear_fwd per linear, summed"}
-    for m in wl.M:
-        def fwd_all(m=m):
-            for (lin, pk, q, s2), a in zip(packed, acts):
-                binding.linear_fwd(pk, q, s2, a["X"][:m], a["A"], a["B"], wl.alpha, lin.N, lin.K,
-                                   Y=Ybuf[:m * lin.N].view(m, lin.N), XA_out=XAbuf[:m * wl.r].view(m, wl.r),
-                                   workspace=ws)
-        ms = device_ms(fwd_all, 3 if m > 16 else 10)
-        flops = sum(2 * m * lin.N * lin.K + 2 * m * wl.r * (lin.N + lin.K) for lin, *_ in packed)
-        if m <= 16:
-            nbytes = sum(lin.N * lin.K // 2 + lin.N * lin.K // 64 + (lin.N * lin.K // 16384) * 4 +
-                         2 * (m * lin.K + lin.K * wl.r + wl.r * lin.N + m * lin.N + m * wl.r) for lin, *_ in packed)
-            c4[f"M{m}"] = {"ms": round(ms, 4), "MB": round(nbytes / 1e6, 1), **frac_hbm(nbytes / (ms * 1e-3) / 1e9)}
-        else:
-            c4[f"M{m}"] = {"ms": round(ms, 4), **frac_tc(flops / (ms * 1e-3) / 1e12)}
-    out["llama65b_fwd"] = c4
-    del packed, acts, Ybuf, XAbuf, ws
-
-    # -- 7B set in fp16 (the pages' other 16-bit compute type): fused fwd + bwd
-    wl = WORKLOADS["llama7b_set"]
-    M = wl.M[0]
-    f16 = []
-    for li, lin in enumerate(wl.linears):
-        inp = layer_inputs(wl, li, M, device=dev)
+    if want("single_1024"):
+        # -- single linear (latency; every tensor L2-resident)
+        wl = WORKLOADS["single_1024"]
+        inp = layer_inputs(wl, 0, wl.M[0], device=dev)
+        N, K, M, r = wl.linears[0].N, wl.linears[0].K, wl.M[0], wl.r
         pk, q, s2 = quantized(inp["W"])
-        h = {k: inp[k].to(torch.float16) for k in ("X", "A", "B", "dY")}
-        del inp
-        f16.append((lin, pk, q, s2, h, torch.empty((M, lin.N), dtype=torch.float16, device=dev),
-                    torch.empty((M, wl.r), dtype=torch.float16, device=dev),
-                    torch.empty((M, lin.K), dtype=torch.float16, device=dev),
-                    torch.empty((lin.K, wl.r), dtype=torch.float16, device=dev),
-                    torch.empty((wl.r, lin.N), dtype=torch.float16, device=dev)))
-    ws = torch.empty(max(binding.workspace_bytes(M, lin.N, lin.K, wl.r) for lin, *_ in f16),
-                     dtype=torch.uint8, device=dev)
+        ws = torch.empty(binding.workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+        Y, XA = torch.empty((M, N), dtype=torch.bfloat16, device=dev), torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+        dX, dA, dB = (torch.empty(sh, dtype=torch.bfloat16, device=dev) for sh in ((M, K), (K, r), (r, N)))
 
-    def fwd_bwd_f16():
-        for lin, pk, q, s2, h, Y, XA, dX, dA, dB in f16:
-            binding.linear_fwd(pk, q, s2, h["X"], h["A"], h["B"], wl.alpha, lin.N, lin.K, Y=Y, XA_out=XA,
-                               workspace=ws)
-            binding.linear_bwd(pk, q, s2, h["X"], h["dY"], h["A"], h["B"], wl.alpha, lin.N, lin.K, XA=XA, dX=dX,
+        def c1():
+            binding.linear_fwd(pk, q, s2, inp["X"], inp["A"], inp["B"], wl.alpha, N, K, Y=Y, XA_out=XA, workspace=ws)
+            binding.linear_bwd(pk, q, s2, inp["X"], inp["dY"], inp["A"], inp["B"], wl.alpha, N, K, XA=XA, dX=dX,
                                dA=dA, dB=dB, workspace=ws)
-    ms = device_ms(fwd_bwd_f16, 5)
-    flops = sum(linear_flops(M, lin.N, lin.K, wl.r) for lin, *_ in f16)
-    out["llama7b_f16"] = {"what": "7 linears of the 7B set, M=2048, r=64, fp16 operands and outputs: "
-                                  "qlora_linear_fwd + qlora_linear_bwd (the _dt calls)",
-                          "ms": round(ms, 4), **frac_tc(flops / (ms * 1e-3) / 1e12)}
+        ms = device_ms(c1, 50)
+        out["single_1024"] = {"what": "qlora_linear_fwd + qlora_linear_bwd, 1024x1024, M=16, r=8 (L2-resident)",
+                              "us_per_fwd_bwd": round(ms * 1e3, 2),
+                              "TFLOP/s": round(linear_flops(M, N, K, r) / (ms * 1e-3) / 1e12, 3)}
+        del inp, pk, q, s2, ws
 
-    # -- paged AdamW over the 7B set's adapters: state on the device, and paged out to the host
-    grads = [t for *_, dA, dB in f16 for t in (dA, dB)]
-    params = [t.clone() for lin, pk, q, s2, h, *_ in f16 for t in (h["A"], h["B"])]
-    n_el = sum(t.numel() for t in params)
-    adamw = {}
-    for where, reserve in (("device", 0), ("host", 1 << 62)):
-        opt = binding.PagedAdamW(params, lr=1e-4, weight_decay=0.01)
-        opt.set_reserve(reserve)
-        opt.step(grads)  # places the state
+    if want("llama13b_quant_sweep"):
+        # -- 13B-equivalent codec sweep: one layer's buffers, refilled per layer (outside the timed calls)
+        wl = WORKLOADS["llama13b_quant_sweep"]
+        layers = 4 if quick else wl.layers
+        bufs = []
+        for lin in wl.linears:
+            n = lin.N * lin.K
+            bufs.append({"N": lin.N, "K": lin.K, "W": torch.empty((lin.N, lin.K), dtype=torch.bfloat16, device=dev),
+                         "pk": torch.empty(n // 2, dtype=torch.uint8, device=dev),
+                         "am": torch.empty(n // 64, dtype=torch.float32, device=dev),
+                         "q": torch.empty(n // 64, dtype=torch.uint8, device=dev),
+                         "s2": torch.empty((n // 64 + 255) // 256, dtype=torch.float32, device=dev),
+                         "Wq": torch.empty((lin.N, lin.K), dtype=torch.bfloat16, device=dev)})
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 2x L2: written between timed calls
+        t_q = t_dq = t_d = t_qdq = 0.0
+        params = 0
+        for layer in range(layers):
+            for li, b in enumerate(bufs):
+                b["W"].copy_(weight_bf16(b["N"], b["K"], wl.w_std, seed_for(wl.index, li, 0, layer), device=dev))
+            flush.zero_()
+            t_q += device_ms(lambda: [binding.quantize_nf4(b["W"], packed=b["pk"], absmax=b["am"]) for b in bufs], 1, 0)
+            flush.zero_()
+            t_dq += device_ms(lambda: [binding.double_quant(b["am"], q=b["q"], scale2=b["s2"]) for b in bufs], 1, 0)
+            flush.zero_()
+            t_qdq += device_ms(lambda: [binding.quantize_dq(b["W"], packed=b["pk"], q=b["q"], scale2=b["s2"])
+                                        for b in bufs], 1, 0)
+            flush.zero_()
+            t_d += device_ms(lambda: [binding.dequant(b["pk"], b["q"], b["s2"], b["N"], b["K"], out=b["Wq"])
+                                      for b in bufs], 1, 0)
+            params += sum(b["N"] * b["K"] for b in bufs)
+        n = params
+        q_in, q_out = 2 * n, n // 2 + n // 64 * 4
+        dq_in, dq_out = n // 64 * 4, n // 64 + n // 16384 * 4
+        d_in, d_out = n // 2 + n // 64 + n // 16384 * 4, 2 * n
+        out["llama13b_quant_sweep"] = {
+            "what": f"{layers} layers x 7 linears (d=5120, ffn=13824), {n / 1e9:.3f} G params, per-call events summed",
+            "quantize": {"ms": round(t_q, 3), "GB_in": round(q_in / 1e9, 3), "GB_out": round(q_out / 1e9, 3),
+                         **frac_hbm((q_in + q_out) / (t_q * 1e-3) / 1e9)},
+            "double_quant": {"ms": round(t_dq, 3), **frac_hbm((dq_in + dq_out) / (t_dq * 1e-3) / 1e9)},
+            "quantize_plus_double_quant": {"ms": round(t_q + t_dq, 3),
+                                           **frac_hbm((q_in + q_out + dq_in + dq_out) / ((t_q + t_dq) * 1e-3) / 1e9)},
+            "quantize_dq_one_pass": {"ms": round(t_qdq, 3), "GB_in": round(q_in / 1e9, 3),
+                                     "GB_out": round((n // 2 + n // 64 + n // 16384 * 4) / 1e9, 3),
+                                     **frac_hbm((q_in + n // 2 + n // 64 + n // 16384 * 4) / (t_qdq * 1e-3) / 1e9)},
+            "dequant": {"ms": round(t_d, 3), "GB_in": round(d_in / 1e9, 3), "GB_out": round(d_out / 1e9, 3),
+                        **frac_hbm((d_in + d_out) / (t_d * 1e-3) / 1e9)}}
+        del bufs, flush
+
+    if want("llama65b_fwd"):
+        # -- 65B-shaped forwards: few tokens (HBM-bound) and M = 4096 (tensor-bound)
+        wl = WORKLOADS["llama65b_fwd"]
+        packed = []
+        for li, lin in enumerate(wl.linears):
+            W = weight_bf16(lin.N, lin.K, wl.w_std, seed_for(wl.index, li, 0), device=dev)
+            packed.append((lin, *quantized(W)))
+            del W
         torch.cuda.synchronize()
-        ms = device_ms(lambda: opt.step(grads), 10)
-        gbs = n_el * 28 / (ms * 1e-3) / 1e9  # 2 B grad + 12 B state read + 12 B written + 2 B param
-        adamw[where] = {"ms": round(ms, 4), "placement": opt.location, "GB/s": round(gbs, 1),
-                        **({"frac_hbm": round(gbs / hbm_gbs, 3)} if where == "device" else {})}
-        opt.close()
-    out["paged_adamw_7b_adapters"] = {"what": f"one AdamW step over the 14 adapter tensors of the 7B set "
-                                              f"({n_el / 1e6:.2f} M fp16 parameters, fp32 state in managed memory)",
-                                      **adamw}
-    del f16, ws, grads, params
-    torch.cuda.empty_cache()
+        Mmax = max(wl.M)
+        Kmax = max(lin.K for lin in wl.linears)
+        Nmax = max(lin.N for lin in wl.linears)
+        acts = []
+        for li, (lin, _, _, _) in enumerate(packed):
+            acts.append({"X": torch.randn((Mmax, lin.K), device=dev).to(torch.bfloat16),
+                         "A": (torch.randn((lin.K, wl.r), device=dev) * 0.01).to(torch.bfloat16),
+                         "B": (torch.randn((wl.r, lin.N), device=dev) * 0.01).to(torch.bfloat16)})
+        Ybuf = torch.empty(Mmax * Nmax, dtype=torch.bfloat16, device=dev)
+        XAbuf = torch.empty(Mmax * wl.r, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(binding.workspace_bytes(m, lin.N, lin.K, wl.r) for m in wl.M for lin, *_ in packed),
+                         dtype=torch.uint8, device=dev)
+        c4 = {"what": "7 linears (d=8192, ffn=22016), r=64: one qlora_linear_fwd per linear, summed"}
+        for m in wl.M:
+            def fwd_all(m=m):
+                for (lin, pk, q, s2), a in zip(packed, acts):
+                    binding.linear_fwd(pk, q, s2, a["X"][:m], a["A"], a["B"], wl.alpha, lin.N, lin.K,
+                                       Y=Ybuf[:m * lin.N].view(m, lin.N), XA_out=XAbuf[:m * wl.r].view(m, wl.r),
+                                       workspace=ws)
+            ms = device_ms(fwd_all, 3 if m > 16 else 10)
+            flops = sum(2 * m * lin.N * lin.K + 2 * m * wl.r * (lin.N + lin.K) for lin, *_ in packed)
+            if m <= 16:
+                nbytes = sum(lin.N * lin.K // 2 + lin.N * lin.K // 64 + (lin.N * lin.K // 16384) * 4 +
+                             2 * (m * lin.K + lin.K * wl.r + wl.r * lin.N + m * lin.N + m * wl.r) for lin, *_ in packed)
+                c4[f"M{m}"] = {"ms": round(ms, 4), "MB": round(nbytes / 1e6, 1), **frac_hbm(nbytes / (ms * 1e-3) / 1e9)}
+            else:
+                c4[f"M{m}"] = {"ms": round(ms, 4), **frac_tc(flops / (ms * 1e-3) / 1e12)}
+        out["llama65b_fwd"] = c4
+        del packed, acts, Ybuf, XAbuf, ws
 
-    # -- 33B-shaped block: forward saving XA, backward recomputing XA (checkpoint style)
-    wl = WORKLOADS["llama33b_block"]
-    M = wl.M[0]
-    state = []
-    for li, lin in enumerate(wl.linears):
-        inp = layer_inputs(wl, li, M, device=dev)
-        pk, q, s2 = quantized(inp["W"])
-        del inp["W"]
-        state.append((lin, pk, q, s2, inp, torch.empty((M, lin.N), dtype=torch.bfloat16, device=dev),
-                      torch.empty((M, wl.r), dtype=torch.bfloat16, device=dev),
-                      torch.empty((M, lin.K), dtype=torch.bfloat16, device=dev),
-                      torch.empty((lin.K, wl.r), dtype=torch.bfloat16, device=dev),
-                      torch.empty((wl.r, lin.N), dtype=torch.bfloat16, device=dev)))
-    ws = torch.empty(max(binding.workspace_bytes(M, lin.N, lin.K, wl.r) for lin, *_ in state),
-                     dtype=torch.uint8, device=dev)
+    if want("llama7b_f16") or want("paged_adamw_7b_adapters"):
+        # -- 7B set in fp16 (the pages' other 16-bit compute type): fused fwd + bwd
+        wl = WORKLOADS["llama7b_set"]
+        M = wl.M[0]
+        f16 = []
+        for li, lin in enumerate(wl.linears):
+            inp = layer_inputs(wl, li, M, device=dev)
+            pk, q, s2 = quantized(inp["W"])
+            h = {k: inp[k].to(torch.float16) for k in ("X", "A", "B", "dY")}
+            del inp
+            f16.append((lin, pk, q, s2, h, torch.empty((M, lin.N), dtype=torch.float16, device=dev),
+                        torch.empty((M, wl.r), dtype=torch.float16, device=dev),
+                        torch.empty((M, lin.K), dtype=torch.float16, device=dev),
+                        torch.empty((lin.K, wl.r), dtype=torch.float16, device=dev),
+                        torch.empty((wl.r, lin.N), dtype=torch.float16, device=dev)))
+        ws = torch.empty(max(binding.workspace_bytes(M, lin.N, lin.K, wl.r) for lin, *_ in f16),
+                         dtype=torch.uint8, device=dev)
 
-    def block():
-        for lin, pk, q, s2, inp, Y, XA, dX, dA, dB in state:
-            binding.linear_fwd(pk, q, s2, inp["X"], inp["A"], inp["B"], wl.alpha, lin.N, lin.K, Y=Y, XA_out=XA,
-                               workspace=ws)
-        for lin, pk, q, s2, inp, Y, XA, dX, dA, dB in reversed(state):
-            binding.linear_bwd(pk, q, s2, inp["X"], inp["dY"], inp["A"], inp["B"], wl.alpha, lin.N, lin.K, XA=None,
-                               dX=dX, dA=dA, dB=dB, workspace=ws)
-    ms_seq = device_ms(block, 3)
-    # the same work through the block executor (qlora_block_fwd/bwd: one call
-    # per pass, linears over two streams), checkpoint schedule: the forward
-    # saves nothing and the backward recomputes X A
-    lins = [{"packed": pk, "q": q, "scale2": s2, "N": lin.N, "K": lin.K, "X": inp["X"], "A": inp["A"],
-             "B": inp["B"], "Y": Y, "XA": XA, "dY": inp["dY"], "dX": dX, "dA": dA, "dB": dB}
-            for lin, pk, q, s2, inp, Y, XA, dX, dA, dB in state]
-    bws = torch.empty(binding.block_workspace_bytes(lins, M, wl.r), dtype=torch.uint8, device=dev)
-    rev = lins[::-1]
+        def fwd_bwd_f16():
+            for lin, pk, q, s2, h, Y, XA, dX, dA, dB in f16:
+                binding.linear_fwd(pk, q, s2, h["X"], h["A"], h["B"], wl.alpha, lin.N, lin.K, Y=Y, XA_out=XA,
+                                   workspace=ws)
+                binding.linear_bwd(pk, q, s2, h["X"], h["dY"], h["A"], h["B"], wl.alpha, lin.N, lin.K, XA=XA, dX=dX,
+                                   dA=dA, dB=dB, workspace=ws)
+        ms = device_ms(fwd_bwd_f16, 5)
+        flops = sum(linear_flops(M, lin.N, lin.K, wl.r) for lin, *_ in f16)
+        out["llama7b_f16"] = {"what": "7 linears of the 7B set, M=2048, r=64, fp16 operands and outputs: "
+                                      "qlora_linear_fwd + qlora_linear_bwd (the _dt calls)",
+                              "ms": round(ms, 4), **frac_tc(flops / (ms * 1e-3) / 1e12)}
 
-    def block_exec():
-        binding.block_fwd(lins, M, wl.r, wl.alpha, save_xa=False, workspace=bws)
-        binding.block_bwd(rev, M, wl.r, wl.alpha, save_xa=False, workspace=bws)
-    ms = device_ms(block_exec, 3)
-    flops = sum(linear_flops(M, lin.N, lin.K, wl.r) + 2 * M * lin.K * wl.r for lin, *_ in state)
-    out["llama33b_block"] = {"what": "7 linears (d=6656, ffn=17920), M=2048, r=64: block forward saving nothing, "
-                                     "block backward recomputing XA and re-dequantizing W (qlora_block_fwd/bwd, "
-                                     "2 streams)",
-                             "ms": round(ms, 4), "ms_linears_one_by_one": round(ms_seq, 4),
-                             "GFLOP": round(flops / 1e9, 1), **frac_tc(flops / (ms * 1e-3) / 1e12)}
-    del state, ws, bws, lins, rev
-    torch.cuda.empty_cache()
+        # -- paged AdamW over the 7B set's adapters: state on the device, and paged out to the host
+        grads = [t for *_, dA, dB in f16 for t in (dA, dB)]
+        params = [t.clone() for lin, pk, q, s2, h, *_ in f16 for t in (h["A"], h["B"])]
+        n_el = sum(t.numel() for t in params)
+        adamw = {}
+        for where, reserve in (("device", 0), ("host", 1 << 62)):
+            opt = binding.PagedAdamW(params, lr=1e-4, weight_decay=0.01)
+            opt.set_reserve(reserve)
+            opt.step(grads)  # places the state
+            torch.cuda.synchronize()
+            ms = device_ms(lambda: opt.step(grads), 10)
+            gbs = n_el * 28 / (ms * 1e-3) / 1e9  # 2 B grad + 12 B state read + 12 B written + 2 B param
+            adamw[where] = {"ms": round(ms, 4), "placement": opt.location, "GB/s": round(gbs, 1),
+                            **({"frac_hbm": round(gbs / hbm_gbs, 3)} if where == "device" else {})}
+            opt.close()
+        out["paged_adamw_7b_adapters"] = {"what": f"one AdamW step over the 14 adapter tensors of the 7B set "
+                                                  f"({n_el / 1e6:.2f} M fp16 parameters, fp32 state in managed memory)",
+                                          **adamw}
+        del f16, ws, grads, params
+        torch.cuda.empty_cache()
+
+    if want("llama33b_block"):
+        # -- 33B-shaped block: forward saving XA, backward recomputing XA (checkpoint style)
+        wl = WORKLOADS["llama33b_block"]
+        M = wl.M[0]
+        state = []
+        for li, lin in enumerate(wl.linears):
+            inp = layer_inputs(wl, li, M, device=dev)
+            pk, q, s2 = quantized(inp["W"])
+            del inp["W"]
+            state.append((lin, pk, q, s2, inp, torch.empty((M, lin.N), dtype=torch.bfloat16, device=dev),
+                          torch.empty((M, wl.r), dtype=torch.bfloat16, device=dev),
+                          torch.empty((M, lin.K), dtype=torch.bfloat16, device=dev),
+                          torch.empty((lin.K, wl.r), dtype=torch.bfloat16, device=dev),
+                          torch.empty((wl.r, lin.N), dtype=torch.bfloat16, device=dev)))
+        ws = torch.empty(max(binding.workspace_bytes(M, lin.N, lin.K, wl.r) for lin, *_ in state),
+                         dtype=torch.uint8, device=dev)
+
+        def block():
+            for lin, pk, q, s2, inp, Y, XA, dX, dA, dB in state:
+                binding.linear_fwd(pk, q, s2, inp["X"], inp["A"], inp["B"], wl.alpha, lin.N, lin.K, Y=Y, XA_out=XA,
+                                   workspace=ws)
+            for lin, pk, q, s2, inp, Y, XA, dX, dA, dB in reversed(state):
+                binding.linear_bwd(pk, q, s2, inp["X"], inp["dY"], inp["A"], inp["B"], wl.alpha, lin.N, lin.K, XA=None,
+                                   dX=dX, dA=dA, dB=dB, workspace=ws)
+        ms_seq = device_ms(block, 3)
+        # the same work through the block executor (qlora_block_fwd/bwd: one call
+        # per pass, linears over two streams), checkpoint schedule: the forward
+        # saves nothing and the backward recomputes X A
+        lins = [{"packed": pk, "q": q, "scale2": s2, "N": lin.N, "K": lin.K, "X": inp["X"], "A": inp["A"],
+                 "B": inp["B"], "Y": Y, "XA": XA, "dY": inp["dY"], "dX": dX, "dA": dA, "dB": dB}
+                for lin, pk, q, s2, inp, Y, XA, dX, dA, dB in state]
+        bws = torch.empty(binding.block_workspace_bytes(lins, M, wl.r), dtype=torch.uint8, device=dev)
+        rev = lins[::-1]
+
+        def block_exec():
+            binding.block_fwd(lins, M, wl.r, wl.alpha, save_xa=False, workspace=bws)
+            binding.block_bwd(rev, M, wl.r, wl.alpha, save_xa=False, workspace=bws)
+        ms = device_ms(block_exec, 3)
+        flops = sum(linear_flops(M, lin.N, lin.K, wl.r) + 2 * M * lin.K * wl.r for lin, *_ in state)
+        out["llama33b_block"] = {"what": "7 linears (d=6656, ffn=17920), M=2048, r=64: block forward saving nothing, "
+                                         "block backward recomputing XA and re-dequantizing W (qlora_block_fwd/bwd, "
+                                         "2 streams)",
+                                 "ms": round(ms, 4), "ms_linears_one_by_one": round(ms_seq, 4),
+                                 "GFLOP": round(flops / 1e9, 1), **frac_tc(flops / (ms * 1e-3) / 1e12)}
+        del state, ws, bws, lins, rev
+        torch.cuda.empty_cache()
     return out
 
 
@@ -692,6 +704,12 @@ def run_native(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     build()
     binding.load()
+    if args.phase:
+        pk, _ = peaks()
+        res = workload_phases(dev, pk["hbm_gbs"], pk["bf16_tflops"], only=args.phase)
+        if rank == 0:
+            print(json.dumps({"phase": args.phase, "workloads": res, "device_error": binding.device_error()}))
+        return
     wl = WORKLOADS[WORKLOAD]
     M = wl.M[0]
     keep = [n for n in args.linears.split(",") if n]

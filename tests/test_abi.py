@@ -131,3 +131,38 @@ def test_dtype_argument_is_checked_first(lib):
     assert lib.qlora_linear_fwd_dt(_fake(), _fake(), _fake(), tb.nf4, tb.t8, 1, 16, 128, 128, _fake(), _fake(),
                                    _fake(), 0, 16.0, _fake(), None, _fake(), 1 << 30, s) == 4
     assert lib.qlora_dequant_dt(None, _fake(), _fake(), 64, 64, tb.nf4, tb.t8, 1, _fake(), s) == 1
+
+
+def test_quantize_dq_argument_checks(lib):
+    """The one-pass quantize checks its arguments like the two calls it
+    replaces, before any launch."""
+    tb = binding._tables(None, None)
+    s = ctypes.c_void_p(0)
+    f = lib.qlora_quantize_dq
+    assert f(None, 64, 64, tb.nf4, tb.t8, _fake(), _fake(), _fake(), None, s) == 1
+    assert f(_fake(), 64, 64, tb.nf4, tb.t8, _fake(), None, _fake(), None, s) == 1
+    assert f(_fake(), 64, 96, tb.nf4, tb.t8, _fake(), _fake(), _fake(), None, s) == 2
+    assert f(_fake(), 0, 64, tb.nf4, tb.t8, _fake(), _fake(), _fake(), None, s) == 2
+    assert f(_fake(0x10008), 64, 64, tb.nf4, tb.t8, _fake(), _fake(), _fake(), None, s) == 3
+    assert f(_fake(), 64, 64, tb.nf4, tb.t8, _fake(), _fake(), _fake(), _fake(0x10004), s) == 3
+    bad = (ctypes.c_float * 16)(*np.linspace(-1, 1, 16).astype(np.float32))  # no exact 0
+    assert f(_fake(), 64, 64, bad, tb.t8, _fake(), _fake(), _fake(), None, s) == 8
+
+
+def test_block_and_optimizer_argument_checks(lib):
+    """Block executor and paged optimizer: null, shape and range checks that
+    need no device."""
+    tb = binding._tables(None, None)
+    s = ctypes.c_void_p(0)
+    assert lib.qlora_block_fwd(0, None, tb.nf4, tb.t8, 0, 16, 8, 16.0, 1, _fake(), 1 << 20, s) == 2
+    assert lib.qlora_block_bwd(1, None, tb.nf4, tb.t8, 0, 16, 8, 16.0, 1, _fake(), 1 << 20, s) == 1
+    assert lib.qlora_block_fwd(1, None, tb.nf4, tb.t8, 5, 16, 8, 16.0, 1, _fake(), 1 << 20, s) == 4
+    assert lib.qlora_block_workspace_bytes(0, None, 16, 8) == 0
+    counts = (ctypes.c_int64 * 2)(10, 0)
+    h = ctypes.c_void_p()
+    assert lib.qlora_paged_adamw_create(2, counts, ctypes.byref(h)) == 2
+    assert lib.qlora_paged_adamw_create(0, counts, ctypes.byref(h)) == 2
+    assert lib.qlora_paged_adamw_create(1, None, ctypes.byref(h)) == 1
+    assert lib.qlora_paged_adamw_location(None) == -1
+    assert lib.qlora_paged_adamw_state_bytes(None) == 0
+    lib.qlora_paged_adamw_destroy(None)  # a no-op
