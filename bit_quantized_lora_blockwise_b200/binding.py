@@ -38,7 +38,8 @@ EXPORTS = ("qlora_status_string", "qlora_abi_version", "qlora_nf4_levels", "qlor
            "qlora_paged_adamw_create", "qlora_paged_adamw_destroy", "qlora_paged_adamw_init",
            "qlora_paged_adamw_step", "qlora_paged_adamw_set_reserve", "qlora_paged_adamw_placement",
            "qlora_paged_adamw_location", "qlora_paged_adamw_state_bytes", "qlora_paged_adamw_state",
-           "qlora_block_workspace_bytes", "qlora_block_fwd", "qlora_block_bwd", "qlora_quantize_dq")
+           "qlora_block_workspace_bytes", "qlora_block_fwd", "qlora_block_bwd", "qlora_quantize_dq",
+           "qlora_debug_fail_allocs")
 
 BLOCK_STREAMS = 2
 
@@ -133,6 +134,8 @@ def load(path: str | None = None):
         lib.qlora_launch_count.restype = ctypes.c_uint64
         lib.qlora_selftest_bounded_wait.argtypes = [P]
         lib.qlora_selftest_bounded_wait.restype = I32
+        lib.qlora_debug_fail_allocs.argtypes = [I32, I32]
+        lib.qlora_debug_fail_allocs.restype = I32
         for fn in ("qlora_quantize_nf4", "qlora_double_quant", "qlora_dequant", "qlora_linear_fwd",
                    "qlora_linear_bwd"):
             getattr(lib, fn).restype = I32
@@ -255,6 +258,15 @@ def selftest_bounded_wait():
     limit and sets bit 0 of the device error word (read it with
     device_error)."""
     _check(load().qlora_selftest_bounded_wait(_stream()), "qlora_selftest_bounded_wait")
+
+
+def debug_fail_allocs(n: int, skip: int = 0) -> int:
+    """Host-side allocation fault injection: after `skip` more of the
+    library's resource allocations succeed (managed optimizer state, the
+    block executor's streams and events), the next `n` fail as if the driver
+    were out of memory. n = 0 cancels. Returns the failures still pending
+    before the call."""
+    return int(load().qlora_debug_fail_allocs(int(skip), int(n)))
 
 
 def launch_count() -> int:

@@ -12,6 +12,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <new>
 #include <vector>
 
 #include "qlora.h"
@@ -41,6 +42,22 @@ struct DeviceInfo {
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 std::atomic<uint64_t> g_launches{0};
+// Injected allocation failures: after g_inject_skip more allocations
+// succeed, the next g_inject_fail fail.
+std::mutex g_inject_mu;
+int g_inject_skip = 0, g_inject_fail = 0;
+
+// True when this allocation is to fail (consumes one injected failure).
+bool inject_alloc_failure() {
+  std::lock_guard<std::mutex> lock(g_inject_mu);
+  if (g_inject_fail <= 0) return false;
+  if (g_inject_skip > 0) {
+    --g_inject_skip;
+    return false;
+  }
+  --g_inject_fail;
+  return true;
+}
 thread_local cudaEvent_t t_trace_start = nullptr;
 thread_local cudaEvent_t t_trace_stop = nullptr;
 // Compute type of the call in progress on this thread (set by the entry
@@ -1340,6 +1357,14 @@ void qlora_set_trace_events(void *start, void *stop) {
 
 uint64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+int qlora_debug_fail_allocs(int skip, int n) {
+  std::lock_guard<std::mutex> lock(g_inject_mu);
+  const int pending = g_inject_fail;
+  g_inject_skip = std::max(skip, 0);
+  g_inject_fail = std::max(n, 0);
+  return pending;
+}
+
 qlora_status qlora_selftest_bounded_wait(qlora_stream_t stream) {
   qlora_status st;
   DeviceInfo d;
@@ -1375,16 +1400,40 @@ struct BlockStreams {
 };
 thread_local BlockStreams t_block[kMaxDevices];
 
+cudaError_t make_event(cudaEvent_t *e) {
+  if (inject_alloc_failure()) return cudaErrorMemoryAllocation;
+  return cudaEventCreateWithFlags(e, cudaEventDisableTiming);
+}
+
+cudaError_t make_stream(cudaStream_t *s) {
+  if (inject_alloc_failure()) return cudaErrorMemoryAllocation;
+  return cudaStreamCreateWithFlags(s, cudaStreamNonBlocking);
+}
+
+// Destroys whatever a failed first-use setup had created, so that the next
+// call starts from nothing.
+void release_block_streams(BlockStreams &b) {
+  if (b.fork) cudaEventDestroy(b.fork);
+  for (int i = 0; i < QLORA_BLOCK_STREAMS - 1; ++i) {
+    if (b.side[i]) cudaStreamDestroy(b.side[i]);
+    if (b.join[i]) cudaEventDestroy(b.join[i]);
+  }
+  b = BlockStreams{};
+}
+
 qlora_status block_streams(BlockStreams **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ERR_CUDA;
   BlockStreams &b = t_block[dev];
   if (!b.init) {
-    if (cudaEventCreateWithFlags(&b.fork, cudaEventDisableTiming) != cudaSuccess) return QLORA_ERR_CUDA;
-    for (int i = 0; i < QLORA_BLOCK_STREAMS - 1; ++i)
-      if (cudaStreamCreateWithFlags(&b.side[i], cudaStreamNonBlocking) != cudaSuccess ||
-          cudaEventCreateWithFlags(&b.join[i], cudaEventDisableTiming) != cudaSuccess)
-        return QLORA_ERR_CUDA;
+    bool ok = make_event(&b.fork) == cudaSuccess;
+    for (int i = 0; ok && i < QLORA_BLOCK_STREAMS - 1; ++i)
+      ok = make_stream(&b.side[i]) == cudaSuccess && make_event(&b.join[i]) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      release_block_streams(b);
+      return QLORA_ERR_CUDA;
+    }
     b.init = true;
   }
   *out = &b;
@@ -1534,8 +1583,14 @@ qlora_status qlora_paged_adamw_create(int nseg, const int64_t *counts, qlora_pag
   if (!counts || !out) return QLORA_ERR_NULL;
   *out = nullptr;
   if (nseg < 1) return QLORA_ERR_SHAPE;
-  auto *o = new qlora_paged_adamw();
-  o->offset.resize(static_cast<size_t>(nseg) + 1);
+  auto *o = new (std::nothrow) qlora_paged_adamw();
+  if (!o) return QLORA_ERR_CUDA;
+  try {
+    o->offset.resize(static_cast<size_t>(nseg) + 1);
+  } catch (const std::bad_alloc &) {
+    delete o;
+    return QLORA_ERR_CUDA;
+  }
   o->offset[0] = 0;
   for (int i = 0; i < nseg; ++i) {
     if (counts[i] < 1) {
@@ -1558,7 +1613,7 @@ qlora_status qlora_paged_adamw_create(int nseg, const int64_t *counts, qlora_pag
   cudaDeviceGetAttribute(&cma, cudaDevAttrConcurrentManagedAccess, o->device);
   o->hints = cma != 0;
   void *p = nullptr;
-  if (cudaMallocManaged(&p, o->bytes, cudaMemAttachGlobal) != cudaSuccess) {
+  if (inject_alloc_failure() || cudaMallocManaged(&p, o->bytes, cudaMemAttachGlobal) != cudaSuccess) {
     cudaGetLastError();
     delete o;
     return QLORA_ERR_CUDA;

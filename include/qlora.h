@@ -272,6 +272,24 @@ QLORA_API uint32_t qlora_device_error(int clear);
 QLORA_API qlora_status qlora_selftest_bounded_wait(qlora_stream_t stream);
 
 /*
+ * Host-side allocation fault injection (no counterpart on the pages; the
+ * paged optimizers exist so that a memory spike does not end the run, and
+ * this lets a test make the library's own allocations fail without touching
+ * the GPU). After `skip` more resource allocations succeed, the next `n`
+ * fail with the driver's out-of-memory result, without calling the driver.
+ * The library's resource allocations are the managed optimizer state of
+ * qlora_paged_adamw_create, and the side streams and fork/join events that
+ * the block executor creates on a thread's first qlora_block_fwd /
+ * qlora_block_bwd on a device (in the order: fork event, then per side
+ * stream the stream and its join event). The failing call returns
+ * QLORA_ERR_CUDA, launches nothing, frees what it had made and leaves no
+ * half-built state: the same call succeeds once the injected failures are
+ * used up. n <= 0 cancels the pending failures. Thread-safe; returns the
+ * number of injected failures that were still pending before this call.
+ */
+QLORA_API int qlora_debug_fail_allocs(int skip, int n);
+
+/*
  * Forward without a caller workspace (the QLoRA pages have no counterpart:
  * this is an integration convenience, not part of the method).
  *

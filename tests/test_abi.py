@@ -166,3 +166,14 @@ def test_block_and_optimizer_argument_checks(lib):
     assert lib.qlora_paged_adamw_location(None) == -1
     assert lib.qlora_paged_adamw_state_bytes(None) == 0
     lib.qlora_paged_adamw_destroy(None)  # a no-op
+
+
+def test_alloc_fault_injection_counter(lib):
+    """The injector's pending count: set, read back by the next call, and
+    cancelled by n <= 0 (no allocation is made on a CPU-only host)."""
+    assert binding.debug_fail_allocs(0) == 0
+    assert binding.debug_fail_allocs(3, skip=2) == 0
+    assert binding.debug_fail_allocs(-1) == 3
+    assert binding.debug_fail_allocs(1) == 0
+    assert binding.debug_fail_allocs(0) == 1
+    assert binding.debug_fail_allocs(0) == 0
