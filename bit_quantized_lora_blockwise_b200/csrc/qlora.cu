@@ -584,7 +584,7 @@ struct SkinnyOperands {
 // reduction length) as one grid.
 qlora_status skinny_launch(SkinnyKind kind, const SkinnyOperands *ops, int nprob, int r, int sms,
                            cudaStream_t st, unsigned int *zero_words, int nzero, bool early,
-                           bool late = false, int max_ctas = 0) {
+                           bool late = false) {
   int row_tiles[2] = {0, 0};
   for (int i = 0; i < nprob; ++i) row_tiles[i] = static_cast<int>(cdiv(ops[i].rows, 128));
   // the split is chosen for all row tiles of the launch together
@@ -594,11 +594,6 @@ qlora_status skinny_launch(SkinnyKind kind, const SkinnyOperands *ops, int nprob
                      : kind == SK_G ? plan_skinny_v<false, false>(plan_rows, ops[0].kdim, r, &p)
                                     : plan_skinny_v<true, true>(plan_rows, ops[0].kdim, r, &p);
   if (pst != QLORA_OK) return pst;
-  // at most max_ctas CTAs when that still leaves a CTA per row tile: fewer
-  // K splits, a longer launch on fewer SMs (see fused_spare_sms)
-  const int all_tiles = row_tiles[0] + row_tiles[1];
-  if (max_ctas > 0 && all_tiles <= max_ctas)
-    while (p.splits > 1 && all_tiles * p.splits > max_ctas) p.splits >>= 1;
   SkinnyArgs a;
   std::memset(&a, 0, sizeof a);
   for (int i = 0; i < nprob; ++i) {
@@ -650,9 +645,9 @@ qlora_status skinny_launch(SkinnyKind kind, const SkinnyOperands *ops, int nprob
 qlora_status skinny(SkinnyKind kind, const void *aop, int64_t a_inner, int64_t a_outer, const void *bop,
                     int64_t b_inner, int64_t b_outer, int64_t rows, int64_t kdim, int r, const OutSpec &o,
                     int sms, cudaStream_t st, unsigned int *zero_words = nullptr, int nzero = 0,
-                    bool early = false, int max_ctas = 0) {
+                    bool early = false) {
   const SkinnyOperands op{aop, a_inner, a_outer, bop, b_inner, b_outer, rows, kdim, o};
-  return skinny_launch(kind, &op, 1, r, sms, st, zero_words, nzero, early, false, max_ctas);
+  return skinny_launch(kind, &op, 1, r, sms, st, zero_words, nzero, early);
 }
 
 // -------------------------------------------------------- fused GEMMs --
@@ -736,20 +731,6 @@ FusedPlan plan_fused(int64_t M, int64_t rows, int64_t kblocks, int sms, int pair
   p.part_bytes = splits > 1 ? align256(static_cast<size_t>(splits) * tail * tile_rows * p.ntt * cdiv(p.bn, 32) * 32 * 4)
                             : 0;
   return p;
-}
-
-// SMs a fused GEMM of plan fp leaves idle: it runs one CTA per SM, on
-// min(units, slots) pairs (or CTAs). The low-rank launch before it in the
-// call is capped to those SMs, so that every GEMM CTA starts at once and the
-// low-rank launch runs under the GEMM's main loop (the GEMM waits for it
-// only before its low-rank K-steps).
-int fused_spare_sms(const FusedPlan &fp, int64_t M, int64_t rows, int sms) {
-  const int64_t tile_rows = fp.pair ? 256 : 128;
-  const int64_t tiles = cdiv(rows, tile_rows) * cdiv(M, static_cast<int64_t>(fp.bn) * fp.ntt);
-  const int64_t units = fp.full_tiles + (tiles - fp.full_tiles) * (fp.tail_subtiles > 1 ? fp.tail_subtiles
-                                                                                         : fp.tail_splits);
-  const int64_t used = fp.pair ? 2 * std::min<int64_t>(units, fp.slots) : std::min<int64_t>(units, sms);
-  return static_cast<int>(std::max<int64_t>(0, sms - used));
 }
 
 // Partial bytes of the plan the call will run on this device.
@@ -1135,15 +1116,14 @@ qlora_status qlora_linear_fwd(const uint8_t *packed, const uint8_t *q, const flo
   //    launch zeroes the split-K tile counters. The GEMM after it decodes
   //    the block constants itself and waits for this launch only before its
   //    low-rank K-steps and its counters, so its main loop overlaps it.
-  const FusedPlan fp = plan_fused(M, N, K / 64, d.sms, fused_pair_slots(d.sms));
   {
     OutSpec o{xas, r, scl, XA_out, r, 1.0f, false};
-    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs, counters, static_cast<int>(w.ncounters), false,
-                fused_spare_sms(fp, M, N, d.sms));
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs, counters, static_cast<int>(w.ncounters), false);
     if (st != QLORA_OK) return st;
   }
 
   // 2) Y^T[n, m] = W'[n, :] . X[m, :] + B^T[n, :] . xas[m, :]
+  const FusedPlan fp = plan_fused(M, N, K / 64, d.sms, fused_pair_slots(d.sms));
   const uint32_t b_rows = fp.cta_tokens();
   const uint32_t bkb = static_cast<uint32_t>(!fp.pair ? single_bkb(fp.bn) : fp.ntt == 2 ? kPair2Bkb : kPairBkb);
   GemmArgs a;
@@ -1204,14 +1184,10 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   float *part = reinterpret_cast<float *>(ws + w.counters + 2 * w.mr);
 
   // 1) Gs = bf16(s * dY B^T); the same launch zeroes the tile counters
-  //    (first kernel of the call: it waits before loading). It and the
-  //    X A recompute are capped to the SMs the dX GEMM leaves idle.
-  const FusedPlan fp = plan_fused(M, K, N / 64, d.sms, fused_pair_slots(d.sms));
-  const int spare = fused_spare_sms(fp, M, K, d.sms);
+  //    (first kernel of the call: it waits before loading)
   {
     OutSpec o{gs, r, scl, nullptr, 0, 0.0f, false};
-    st = skinny(SK_G, dY, N, M, B, N, r, M, N, r, o, d.sms, cs, counters, static_cast<int>(w.ncounters), false,
-                spare);
+    st = skinny(SK_G, dY, N, M, B, N, r, M, N, r, o, d.sms, cs, counters, static_cast<int>(w.ncounters), false);
     if (st != QLORA_OK) return st;
   }
 
@@ -1220,12 +1196,13 @@ qlora_status qlora_linear_bwd(const uint8_t *packed, const uint8_t *q, const flo
   const qlora_bf16 *xa = XA;
   if (xa == nullptr) {
     OutSpec o{xa_ws, r, 1.0f, nullptr, 0, 0.0f, false};
-    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs, nullptr, 0, true, spare);
+    st = skinny(SK_XA, X, K, M, A, r, K, M, K, r, o, d.sms, cs, nullptr, 0, true);
     if (st != QLORA_OK) return st;
     xa = xa_ws;
   }
 
   // 2) dX^T[k, m] = W'^T[k, :] . dY[m, :] + A[k, :] . Gs[m, :]
+  const FusedPlan fp = plan_fused(M, K, N / 64, d.sms, fused_pair_slots(d.sms));
   const uint32_t b_rows = fp.cta_tokens();
   const uint32_t bkb = static_cast<uint32_t>(!fp.pair ? single_bkb(fp.bn) : fp.ntt == 2 ? kPair2Bkb : kPairBkb);
   GemmArgs a;
