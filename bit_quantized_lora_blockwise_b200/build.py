@@ -18,7 +18,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libqlora.so")
-SOURCES = ["qlora.cu", "codec.cuh", "gemm.cuh", "skinny.cuh", "smallm.cuh", "ptx.cuh"]
+SOURCES = ["qlora.cu", "codec.cuh", "gemm.cuh", "skinny.cuh", "smallm.cuh", "adamw.cuh", "ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
