@@ -136,8 +136,8 @@ struct GemmCfg {
   static constexpr int OFF_P = OFF_A + SA * A_BYTES;
   static constexpr int OFF_BAR = OFF_P + SP * P_BYTES;
   // b_full[SB] b_empty[SB] a_full[SA] a_empty[SA] p_full[SP] p_empty[SP]
-  // tmem_full[2] tmem_empty[2] drain
-  static constexpr int NBARS = 2 * SB + 2 * SA + 2 * SP + 5;
+  // tmem_full[2] tmem_empty[2] drain epilogue-group
+  static constexpr int NBARS = 2 * SB + 2 * SA + 2 * SP + 6;
   // misc: tmem base, abort flag, last-CTA flag (16 B), the 16 NF4 levels,
   // then the 256-entry 8-bit constant table
   static constexpr int OFF_MISC = ((OFF_BAR + NBARS * 8) + 15) & ~15;
@@ -221,6 +221,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
   auto tmem_full = [&](int a) { return bar0 + 8u * (TB + a); };
   auto tmem_empty = [&](int a) { return bar0 + 8u * (TB + 2 + a); };
   const uint32_t drain_bar = bar0 + 8u * (TB + 4);
+  const uint32_t epi_bar = bar0 + 8u * (TB + 5);  // the four epilogue warps' group barrier
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
   volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -242,6 +243,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
       mbar_init(tmem_empty(a), C::GROUP_ARRIVALS);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(epi_bar, 4);
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -479,7 +481,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
       return args.part + (static_cast<int64_t>(sp) * ntail + ti) * TILE_PCOLS * C::TILE_ROWS + rank * 128 +
              qrow_of(warp, lane);
     };
-    uint32_t iter = 0;
+    uint32_t iter = 0, epi_phase = 0;
     const int qrow = qrow_of(warp, lane);  // TMEM lane of this thread
     // chunk ch of the accumulator row (32 columns; a 16-column tail is zero-padded)
     auto load_chunk = [&](uint32_t tcol, int ch, uint32_t (&u)[32]) {
@@ -550,14 +552,14 @@ __global__ void __launch_bounds__(C::THREADS, 1) qgemm_kernel(const __grid_const
       if (!ok || t.nsplit == 1) continue;
       grid_dep_wait();  // the tile counters are zeroed by the previous launch
       __threadfence();
-      named_bar_sync(1, 128);
+      if (!warp_group_sync(epi_bar, epi_phase, s_abort)) { ok = false; continue; }
       if (warp == 0 && lane == 0) {
         const unsigned int prev = atomicAdd(args.counters + t.rc, 1u);
         const int last = prev == static_cast<unsigned int>(t.nsplit - 1);
         if (last) args.counters[t.rc] = 0u;  // every split has arrived: reset for the next use
         *s_last = last;
       }
-      named_bar_sync(1, 128);
+      if (!warp_group_sync(epi_bar, epi_phase, s_abort)) { ok = false; continue; }
       if (*s_last) {
         __threadfence();
 #pragma unroll 1

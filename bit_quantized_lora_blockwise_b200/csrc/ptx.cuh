@@ -161,6 +161,21 @@ __device__ __forceinline__ bool warp_wait_all(uint32_t bar, uint32_t parity, vol
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
+// Barrier of a group of warps on an mbarrier initialised with one arrival
+// per warp: each warp's lane 0 arrives (a release, after the warp's own
+// shared and global accesses are ordered by __syncwarp) and the warp waits
+// for the phase with the bounded wait. Unlike bar.sync it cannot block for
+// good when a member has left after a failed wait: the others give up after
+// the limit (or at once once the abort flag is up) and it returns false.
+// `phase` is this warp's count of completed uses, parity in bit 0.
+__device__ __forceinline__ bool warp_group_sync(uint32_t bar, uint32_t &phase, volatile int *abort_flag) {
+  __syncwarp();
+  if ((threadIdx.x & 31u) == 0) mbar_arrive(bar);
+  const bool ok = warp_wait_all(bar, phase & 1u, abort_flag);
+  ++phase;
+  return ok;
+}
+
 // ------------------------------------------------------------------ TMA --
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

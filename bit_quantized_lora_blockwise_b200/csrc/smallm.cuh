@@ -73,7 +73,8 @@ struct SmallmCfg {
   static constexpr int STAGE = W_BYTES + X_BYTES;
   static constexpr int SX = NT == 1 ? 6 : 5;     // stages
   static constexpr int OFF_BAR = SX * STAGE;
-  static constexpr int OFF_T8 = OFF_BAR + 2 * SX * 8;
+  // full[SX] empty[SX], then the CTA's group barrier (one arrival per warp)
+  static constexpr int OFF_T8 = OFF_BAR + (2 * SX + 2) * 8;
   static constexpr int OFF_MISC = OFF_T8 + 256 * 4;  // abort flag, two completed-band flags
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SLOT_FLOATS = WARPS * NT * 32 * 4;
@@ -100,6 +101,7 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
   volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC);
   auto full_bar = [&](int s) { return sbase + C::OFF_BAR + 8u * s; };
   auto empty_bar = [&](int s) { return sbase + C::OFF_BAR + 8u * (C::SX + s); };
+  const uint32_t group_bar = sbase + C::OFF_BAR + 8u * (2 * C::SX);
 
   const int grid = gridDim.x;
   const int u_begin = smallm_unit_begin(blockIdx.x, a.units, grid);
@@ -141,6 +143,7 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), C::WARPS);
     }
+    mbar_init(group_bar, C::WARPS);
     *s_abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&a.tm_w);
@@ -388,7 +391,10 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
   // band's number of pieces sums the slots of CTAs c0 .. c1 in CTA order
   // (so the result does not depend on which CTA finishes last), applies the
   // low-rank term and stores Y. No CTA waits for another.
-  named_bar_sync(1, C::WARPS * 32);  // every warp's parked pieces are stored
+  // A bounded group barrier rather than bar.sync: a warp that left after a
+  // failed wait (the error word is then set) cannot hold the others for good.
+  uint32_t group_phase = 0;
+  if (!warp_group_sync(group_bar, group_phase, s_abort)) return;  // every warp's parked pieces are stored
   volatile int *s_last = s_abort + 1;  // [0]: first_band completed here, [1]: last_band
   if (threadIdx.x == 0) {
     __threadfence();
@@ -406,7 +412,7 @@ __global__ void __launch_bounds__(SmallmCfg<NT>::THREADS, 1) smallm_kernel(const
       s_last[k] = last;
     }
   }
-  named_bar_sync(1, C::WARPS * 32);
+  if (!warp_group_sync(group_bar, group_phase, s_abort)) return;
 #pragma unroll 1
   for (int k = 0; k < 2; ++k) {
     const int band = k == 0 ? first_band : last_band;
