@@ -51,6 +51,13 @@ def test_bounded_wait_reports_and_context_survives(cuda_device):
 # return QLORA_ERR_CUDA, launch nothing, leave no half-built state, and the
 # same call must then succeed with the results of an undisturbed run.
 
+@pytest.fixture(autouse=True)
+def _no_pending_injection():
+    """No injected allocation failure outlives the test that set it."""
+    yield
+    binding.debug_fail_allocs(0)
+
+
 def _adapter_params(seed):
     shapes = ((256, 16), (16, 512), (320, 8))
     params = [normal_bf16(s, 0.05, seed + i).cuda() for i, s in enumerate(shapes)]
